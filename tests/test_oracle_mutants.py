@@ -1,0 +1,52 @@
+"""Plant plausible mistakes in a copy of the oracle (CPU only) and check that
+the pins catch every one of them: a dropped term, a wrong scale, sign or
+index, a transposed operand, a wrong head mapping or layout."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moda_oracle.c")
+
+# (name, text in the oracle, planted replacement)
+MUTANTS = [
+    ("seq_scale_dropped", "row[j] = scale * dot(", "row[j] = dot("),
+    ("depth_scale_dropped", "row[t + 1 + l] = scale * dot(", "row[t + 1 + l] = dot("),
+    ("depth_of_previous_token", "kd_off(b, hk, t, 0, Hk, T, L, d) : NULL;\n                const double* vd",
+     "kd_off(b, hk, t > 0 ? t - 1 : 0, 0, Hk, T, L, d) : NULL;\n                const double* vd"),
+    ("gqa_head_tiled", "const int hk = h / G;   /* [GQA] */", "const int hk = h % Hk;"),
+    ("depth_value_dropped", "o[c] += w * Vdep[", "o[c] += 0.0 * Vdep["),
+    ("lse_without_max", "*lse = m + log(Z);", "*lse = log(Z);"),
+    ("bwd_ds_sign", "const double ds = p * (dot(go, v, d) - Dr[r]);\n                        for (int c = 0; c < d; ++c) dq",
+     "const double ds = p * (dot(go, v, d) + Dr[r]);\n                        for (int c = 0; c < d; ++c) dq"),
+    ("bwd_dkd_unscaled", "dKd[o + c] += scale * ds * q[c];", "dKd[o + c] += ds * q[c];"),
+    ("bwd_dv_uses_ds", "dv[c] += p * go[c];", "dv[c] += ds * go[c];"),
+    ("bwd_dk_diagonal_dropped", "for (int t = j; t < T; ++t)", "for (int t = j + 1; t < T; ++t)"),
+    ("bwd_dq_transposed_operand", "dq[c] += scale * ds * k[c];", "dq[c] += scale * ds * q[c];"),
+    ("repack_layer_major_kept", "const size_t o = (((size_t)b * Hk + hk) * T + t) * L + l;",
+     "const size_t o = (((size_t)b * Hk + hk) * L + l) * T + t;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(tmp_path, name, old, new):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation anchor for {name} not unique"
+    src = tmp_path / "mutant.c"
+    src.write_text(text.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", str(src), "-o", str(so), "-lm"])
+    lib = oracle.load_library(str(so))
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
