@@ -1,0 +1,170 @@
+/*
+ * moda.h -- C ABI of libmoda, the fused Mixture-of-Depths Attention (MoDA)
+ * operator for NVIDIA B200 (sm_100a).
+ *
+ * The operator (paper summary of arXiv 2603.15619, section "Mixture-of-Depths
+ * Attention (MoDA): The Unified Operator", joint-softmax equation and its two
+ * masks): for batch b, query head h, token t, with KV head hk = floor(h / G)
+ * and G = Hq / Hk (GQA by repeat_interleave, "moda-attention 0.1.0" PyPI page,
+ * "Key Design Choices"),
+ *
+ *   s_j  = scale * <Q[b,h,t], K[b,hk,j]>              j = 0..t   (causal, incl. t)
+ *   s'_l = scale * <Q[b,h,t], Kd[b,hk,t*L + l]>       l = 0..L-1 (own token only)
+ *   P    = softmax over the concatenated row [s_0..s_t | s'_0..s'_{L-1}]
+ *   O[b,h,t]   = sum_j P_j V[b,hk,j] + sum_l P'_l Vd[b,hk,t*L + l]
+ *   LSE[b,h,t] = natural-log log-sum-exp of the row
+ *
+ * scale = 1/sqrt(d) unless moda_shape.softmax_scale > 0.  The operator is
+ * causal only (the pages list the non-causal kernel as unreleased).
+ *
+ * Conventions for every entry point:
+ *  - Tensors are dense, contiguous, row-major, in device memory, with base
+ *    addresses aligned to 16 bytes.  Layouts ("moda-attention 0.1.0" PyPI
+ *    page, "Using the Kernel Directly"):
+ *        Q, O, dO, dQ          [B, Hq, T, d]
+ *        K, V, dK, dV          [B, Hk, T, d]
+ *        Kd, Vd, dKd, dVd      [B, Hk, T*L, d], row t*L + l = layer l of token t
+ *        LSE                   [B, Hq, T] float32
+ *    Element type of every tensor but LSE is moda_shape.dtype.
+ *  - The caller allocates and owns every buffer, including the workspace.
+ *    The library never allocates, frees or synchronises; all work is queued
+ *    on the caller's stream (NULL = legacy default stream).  Outputs are
+ *    fully overwritten (no accumulate-into).  Inputs and outputs must not
+ *    alias.
+ *  - Errors are returned as moda_status; nothing is thrown across the ABI.
+ *    On any error nothing has been queued.  moda_last_error_message() gives a
+ *    one-line detail for the calling thread's most recent failure.
+ *  - Kernel-side waits are bounded.  A wait that runs out sets a device
+ *    status word and the kernel returns early; moda_check_status() reports it
+ *    as MODA_ERR_TIMEOUT.
+ *  - Thread-safe; calls on different streams may run concurrently.
+ */
+#ifndef MODA_H_
+#define MODA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* moda_stream_t;
+
+typedef enum moda_status {
+    MODA_OK = 0,
+    MODA_ERR_INVALID_ARG = 1,   /* NULL pointer, bad shape or enum value   */
+    MODA_ERR_MISALIGNED = 2,    /* a pointer is not 16-byte aligned         */
+    MODA_ERR_UNSUPPORTED = 3,   /* valid but not implemented (e.g. d=96 bf16) */
+    MODA_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than required  */
+    MODA_ERR_CUDA = 5,          /* a CUDA runtime / driver call failed      */
+    MODA_ERR_TIMEOUT = 6        /* a kernel-side bounded wait ran out        */
+} moda_status;
+
+typedef enum moda_dtype {
+    MODA_BF16 = 0,   /* bf16 in/out, fp32 accumulation and softmax statistics */
+    MODA_FP32 = 1    /* fp32 everywhere (CUDA-core path)                       */
+} moda_dtype;
+
+/*
+ * Depth layouts.  FLAT is the flash-compatible layout of the paper summary,
+ * "Hardware-Efficient Implementation": token t's L rows contiguous at
+ * [t*L, (t+1)*L).  CHUNKED is the chunk-aware view [B, Hk, T/C, C*L, d]: with
+ * C counted in tokens, chunk c holds rows [c*C*L, (c+1)*C*L) of the FLAT
+ * tensor, so it is the same bytes; CHUNKED only adds the check T % C == 0.
+ * Results are bitwise identical for both layouts and every C.
+ */
+typedef enum moda_depth_layout {
+    MODA_DEPTH_FLAT = 0,
+    MODA_DEPTH_CHUNKED = 1
+} moda_depth_layout;
+
+typedef struct moda_shape {
+    int B;            /* batch, >= 0 (0 = nothing to do)                   */
+    int Hq;           /* query heads, >= 1                                  */
+    int Hk;           /* KV heads, >= 1, Hq % Hk == 0, G = Hq/Hk <= 128       */
+    int T;            /* tokens, >= 0 (0 = nothing to do)                   */
+    int d;            /* head dim: 64 or 128 for BF16; 1..128 for FP32       */
+    int L;            /* depth rows per token, >= 0 (0: Kd/Vd may be NULL)  */
+    int C;            /* chunk size in tokens (CHUNKED only; >= 1, T % C == 0) */
+    moda_dtype dtype;
+    moda_depth_layout depth_layout;
+    float softmax_scale;  /* <= 0 selects 1/sqrt(d) */
+} moda_shape;
+
+/*
+ * Bytes of workspace moda_fwd (for_bwd = 0) or moda_bwd (for_bwd = 1) needs
+ * for this shape; 0 means ws may be NULL.  Returns (size_t)-1 for a shape
+ * that the corresponding call would reject.
+ */
+size_t moda_workspace_size(const moda_shape* shape, int for_bwd);
+
+/*
+ * Depth-KV repack (paper summary, "Hardware-Efficient Implementation": the
+ * natural depth cache is layer-major with stride T*d between layers; the
+ * flash-compatible layout puts each token's L rows contiguously).
+ *   src  [L, B, Hk, T, d]  layer-major cache (one tensor: K or V)
+ *   dst  [B, Hk, T*L, d]   token-major; dst row t*L + l = src[l, b, hk, t]
+ * A bytewise permutation: exact for any dtype.  Call once for K_depth and
+ * once for V_depth.  L = 0, B = 0 or T = 0 is a no-op.
+ */
+moda_status moda_repack_depth(const moda_shape* shape, const void* src, void* dst,
+                              moda_stream_t stream);
+
+/*
+ * Forward (the operator above, fused: one online softmax over the causal
+ * sequence keys and the token's own depth rows).
+ *   Q, K, V, Kd, Vd   inputs as laid out above (Kd, Vd may be NULL if L = 0)
+ *   O                 output [B, Hq, T, d], dtype of the shape
+ *   LSE               output [B, Hq, T] float32, natural log; needed by moda_bwd
+ *   ws, ws_bytes      workspace of at least moda_workspace_size(shape, 0) bytes
+ */
+moda_status moda_fwd(const moda_shape* shape,
+                     const void* Q, const void* K, const void* V,
+                     const void* Kd, const void* Vd,
+                     void* O, float* LSE,
+                     void* ws, size_t ws_bytes, moda_stream_t stream);
+
+/*
+ * Backward of moda_fwd.  The pages give no backward formulas; this is the
+ * derivative of the forward definition (one softmax over [seq | depth]):
+ *   D = rowsum(dO * O),  dS = P * (dO . v - D),
+ *   dQ = scale * (sum_j dS_j K_j + sum_l dS'_l Kd_l),
+ *   dK[hk,j]  = scale * sum over the group's heads h and rows t >= j of dS q,
+ *   dV[hk,j]  = sum over the same rows of P dO,
+ *   dKd[hk,t*L+l] = scale * sum over the group's heads of dS' q[h,t],
+ *   dVd[hk,t*L+l] = sum over the group's heads of P' dO[h,t].
+ *   O, LSE            the outputs of moda_fwd for the same inputs
+ *   dO                incoming gradient [B, Hq, T, d]
+ *   dQ, dK, dV, dKd, dVd   outputs (fully overwritten; dKd/dVd may be NULL if L = 0)
+ *   ws, ws_bytes      workspace of at least moda_workspace_size(shape, 1) bytes
+ * Deterministic: no floating-point atomics; repeated calls give identical bits.
+ */
+moda_status moda_bwd(const moda_shape* shape,
+                     const void* Q, const void* K, const void* V,
+                     const void* Kd, const void* Vd,
+                     const void* O, const float* LSE, const void* dO,
+                     void* dQ, void* dK, void* dV, void* dKd, void* dVd,
+                     void* ws, size_t ws_bytes, moda_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's kernel
+ * status word.  MODA_ERR_TIMEOUT if a kernel's bounded wait ran out since the
+ * last check, MODA_ERR_CUDA if the stream reports an error, else MODA_OK.
+ */
+moda_status moda_check_status(moda_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* moda_status_string(moda_status status);
+
+/* Detail of the calling thread's most recent failed call ("" if none). */
+const char* moda_last_error_message(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int moda_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MODA_H_ */

@@ -1,0 +1,162 @@
+"""ctypes binding of libmoda (include/moda.h): argument marshalling only.
+
+Every function here has the name of the C entry point it wraps and takes
+torch tensors (or raw integer device pointers) plus an optional stream.  No
+arithmetic of the operator happens in Python; if the shared library is
+missing the first call raises, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libmoda.so")
+
+MODA_OK = 0
+MODA_ERR_INVALID_ARG = 1
+MODA_ERR_MISALIGNED = 2
+MODA_ERR_UNSUPPORTED = 3
+MODA_ERR_WORKSPACE = 4
+MODA_ERR_CUDA = 5
+MODA_ERR_TIMEOUT = 6
+
+MODA_BF16 = 0
+MODA_FP32 = 1
+MODA_DEPTH_FLAT = 0
+MODA_DEPTH_CHUNKED = 1
+
+# Every symbol include/moda.h declares.
+EXPORTED = ("moda_workspace_size", "moda_repack_depth", "moda_fwd", "moda_bwd",
+            "moda_check_status", "moda_status_string", "moda_last_error_message", "moda_version")
+
+
+class moda_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hk", ctypes.c_int),
+                ("T", ctypes.c_int), ("d", ctypes.c_int), ("L", ctypes.c_int),
+                ("C", ctypes.c_int), ("dtype", ctypes.c_int), ("depth_layout", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float)]
+
+
+class MoDAError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {status_name(status)} ({detail})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: Optional[str] = None):
+    """Load libmoda.so.  Raises if it has not been built (no fallback)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"libmoda.so not found at {p}; build it with "
+                               "`python -m sequence_depth_attention_moda_b200.build`")
+        lib = ctypes.CDLL(p)
+        vp, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        sp = ctypes.POINTER(moda_shape)
+        lib.moda_workspace_size.argtypes = [sp, i]
+        lib.moda_workspace_size.restype = sz
+        lib.moda_repack_depth.argtypes = [sp, vp, vp, vp]
+        lib.moda_repack_depth.restype = i
+        lib.moda_fwd.argtypes = [sp] + [vp] * 7 + [vp, sz, vp]
+        lib.moda_fwd.restype = i
+        lib.moda_bwd.argtypes = [sp] + [vp] * 13 + [vp, sz, vp]
+        lib.moda_bwd.restype = i
+        lib.moda_check_status.argtypes = [vp]
+        lib.moda_check_status.restype = i
+        lib.moda_status_string.argtypes = [i]
+        lib.moda_status_string.restype = ctypes.c_char_p
+        lib.moda_last_error_message.argtypes = []
+        lib.moda_last_error_message.restype = ctypes.c_char_p
+        lib.moda_version.argtypes = []
+        lib.moda_version.restype = i
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_name(status: int) -> str:
+    try:
+        return load().moda_status_string(status).decode()
+    except Exception:  # library missing: still give a readable name
+        return f"status {status}"
+
+
+def make_shape(B, Hq, Hk, T, d, L, C=0, dtype=MODA_BF16, depth_layout=MODA_DEPTH_FLAT,
+               softmax_scale=0.0) -> moda_shape:
+    return moda_shape(int(B), int(Hq), int(Hk), int(T), int(d), int(L), int(C), int(dtype),
+                      int(depth_layout), float(softmax_scale))
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != MODA_OK:
+        detail = load().moda_last_error_message().decode()
+        raise MoDAError(rc, where, detail)
+
+
+def moda_workspace_size(shape: moda_shape, for_bwd: bool) -> int:
+    n = load().moda_workspace_size(ctypes.byref(shape), 1 if for_bwd else 0)
+    if n == ctypes.c_size_t(-1).value:
+        _check(load().moda_fwd(ctypes.byref(shape), *([None] * 7), None, 0, None), "moda_workspace_size")
+    return int(n)
+
+
+def moda_repack_depth(shape: moda_shape, src, dst, stream=None):
+    _check(load().moda_repack_depth(ctypes.byref(shape), _ptr(src), _ptr(dst), _stream(stream)),
+           "moda_repack_depth")
+
+
+def moda_fwd(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, ws=None, ws_bytes: int = 0, stream=None):
+    _check(load().moda_fwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd),
+                           _ptr(O), _ptr(LSE), _ptr(ws), int(ws_bytes), _stream(stream)), "moda_fwd")
+
+
+def moda_bwd(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, ws,
+             ws_bytes: int, stream=None):
+    _check(load().moda_bwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd),
+                           _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dKd),
+                           _ptr(dVd), _ptr(ws), int(ws_bytes), _stream(stream)), "moda_bwd")
+
+
+def moda_check_status(stream=None):
+    _check(load().moda_check_status(_stream(stream)), "moda_check_status")
+
+
+def moda_status_string(status: int) -> str:
+    return load().moda_status_string(int(status)).decode()
+
+
+def moda_last_error_message() -> str:
+    return load().moda_last_error_message().decode()
+
+
+def moda_version() -> int:
+    return int(load().moda_version())

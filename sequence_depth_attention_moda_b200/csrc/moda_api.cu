@@ -1,0 +1,235 @@
+// moda_api.cu -- the C ABI declared in include/moda.h: argument validation,
+// workspace sizing, dispatch to the kernel launchers, status reporting.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "moda.h"
+#include "moda_internal.h"
+
+namespace moda {
+namespace {
+
+// Kernel-side status word, one per device (this is a device variable: every
+// device that loads the library gets its own copy).
+__device__ unsigned int g_status_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+unsigned int* g_status_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+
+thread_local std::string g_last_error;
+
+moda_status fail(moda_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+moda_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(MODA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validate a shape; fill *p.  `tensor_core` selects the bf16 limits.
+moda_status validate(const moda_shape* s, Problem* p) {
+    if (!s) return fail(MODA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->dtype != MODA_BF16 && s->dtype != MODA_FP32)
+        return fail(MODA_ERR_INVALID_ARG, "unknown dtype %d", (int)s->dtype);
+    if (s->depth_layout != MODA_DEPTH_FLAT && s->depth_layout != MODA_DEPTH_CHUNKED)
+        return fail(MODA_ERR_INVALID_ARG, "unknown depth layout %d", (int)s->depth_layout);
+    if (s->B < 0 || s->T < 0 || s->L < 0)
+        return fail(MODA_ERR_INVALID_ARG, "B=%d T=%d L=%d must be >= 0", s->B, s->T, s->L);
+    if (s->Hq < 1 || s->Hk < 1 || s->Hq % s->Hk != 0)
+        return fail(MODA_ERR_INVALID_ARG, "need Hq >= 1, Hk >= 1 and Hq %% Hk == 0 (Hq=%d Hk=%d)",
+                    s->Hq, s->Hk);
+    if (s->d < 1) return fail(MODA_ERR_INVALID_ARG, "d=%d must be >= 1", s->d);
+    if (!(s->softmax_scale >= 0.0f) || std::isinf(s->softmax_scale))
+        return fail(MODA_ERR_INVALID_ARG, "softmax_scale must be finite (<= 0 for 1/sqrt(d))");
+    if (s->depth_layout == MODA_DEPTH_CHUNKED) {
+        if (s->C < 1) return fail(MODA_ERR_INVALID_ARG, "chunked layout needs C >= 1 (C=%d)", s->C);
+        if (s->T % s->C != 0)
+            return fail(MODA_ERR_INVALID_ARG, "chunked layout needs T %% C == 0 (T=%d C=%d)", s->T,
+                        s->C);
+    } else if (s->C < 0) {
+        return fail(MODA_ERR_INVALID_ARG, "C=%d must be >= 0", s->C);
+    }
+    const int G = s->Hq / s->Hk;
+    if (s->dtype == MODA_BF16) {
+        if (s->d != 64 && s->d != 128)
+            return fail(MODA_ERR_UNSUPPORTED, "bf16 path supports d in {64, 128} (d=%d)", s->d);
+        if (G > 128) return fail(MODA_ERR_UNSUPPORTED, "bf16 path supports G <= 128 (G=%d)", G);
+    } else if (s->d > 128) {
+        return fail(MODA_ERR_UNSUPPORTED, "fp32 path supports d <= 128 (d=%d)", s->d);
+    }
+    // 64-bit element counts must stay addressable; the kernels index rows with
+    // 32-bit (b*H + h) and token coordinates.
+    const double rows_q = double(s->B) * s->Hq * s->T;
+    const double rows_d = double(s->B) * s->Hk * s->T * double(s->L);
+    if (rows_q > 2147483647.0 || rows_d > 2147483647.0 || double(s->T) * s->L > 2147483647.0)
+        return fail(MODA_ERR_UNSUPPORTED, "problem too large for 32-bit row indices");
+    p->B = s->B; p->Hq = s->Hq; p->Hk = s->Hk; p->T = s->T; p->d = s->d; p->L = s->L; p->G = G;
+    p->scale = s->softmax_scale > 0.0f ? s->softmax_scale : 1.0f / std::sqrt(float(s->d));
+    p->scale_log2 = p->scale * 1.4426950408889634f;
+    p->elem_bytes = s->dtype == MODA_BF16 ? 2 : 4;
+    return MODA_OK;
+}
+
+moda_status check_ptrs(std::initializer_list<std::pair<const void*, const char*>> ptrs) {
+    for (auto& pr : ptrs) {
+        if (!pr.first) return fail(MODA_ERR_INVALID_ARG, "%s is NULL", pr.second);
+        if (!aligned16(pr.first))
+            return fail(MODA_ERR_MISALIGNED, "%s is not 16-byte aligned", pr.second);
+    }
+    return MODA_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+size_t bwd_workspace_bytes(const Problem& p) {
+    return round_up(size_t(p.B) * p.Hq * p.T * sizeof(float), 256);
+}
+
+unsigned int* device_status_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_dev_mutex);
+    if (!g_status_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<unsigned int*>(ptr);
+    }
+    return g_status_ptr[dev];
+}
+
+int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lk(g_dev_mutex);
+    if (!g_sm_count[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        g_sm_count[dev] = n > 0 ? n : 148;
+    }
+    return g_sm_count[dev];
+}
+
+}  // namespace moda
+
+using namespace moda;
+
+extern "C" {
+
+size_t moda_workspace_size(const moda_shape* shape, int for_bwd) {
+    Problem p;
+    if (validate(shape, &p) != MODA_OK) return static_cast<size_t>(-1);
+    if (!for_bwd) return 0;
+    return bwd_workspace_bytes(p);
+}
+
+moda_status moda_repack_depth(const moda_shape* shape, const void* src, void* dst,
+                              moda_stream_t stream) {
+    Problem p;
+    moda_status st = validate(shape, &p);
+    if (st != MODA_OK) return st;
+    if (p.B == 0 || p.T == 0 || p.L == 0) return MODA_OK;
+    if ((st = check_ptrs({{src, "src"}, {dst, "dst"}})) != MODA_OK) return st;
+    if (src == dst) return fail(MODA_ERR_INVALID_ARG, "repack cannot run in place");
+    cudaError_t e = launch_repack(p.B, p.Hk, p.T, p.d, p.L, p.elem_bytes, src, dst,
+                                  reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MODA_OK : cuda_fail(e, "repack launch");
+}
+
+moda_status moda_fwd(const moda_shape* shape, const void* Q, const void* K, const void* V,
+                     const void* Kd, const void* Vd, void* O, float* LSE, void* ws,
+                     size_t ws_bytes, moda_stream_t stream) {
+    (void)ws; (void)ws_bytes;
+    Problem p;
+    moda_status st = validate(shape, &p);
+    if (st != MODA_OK) return st;
+    if (p.B == 0 || p.T == 0) return MODA_OK;
+    if ((st = check_ptrs({{Q, "Q"}, {K, "K"}, {V, "V"}, {O, "O"}, {LSE, "LSE"}})) != MODA_OK)
+        return st;
+    if (p.L > 0 && (st = check_ptrs({{Kd, "Kd"}, {Vd, "Vd"}})) != MODA_OK) return st;
+    if (!device_status_word()) return fail(MODA_ERR_CUDA, "no usable CUDA device");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = p.elem_bytes == 2
+                        ? launch_fwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, s)
+                        : launch_fwd_simt(p, Q, K, V, Kd, Vd, O, LSE, s);
+    return e == cudaSuccess ? MODA_OK : cuda_fail(e, "forward launch");
+}
+
+moda_status moda_bwd(const moda_shape* shape, const void* Q, const void* K, const void* V,
+                     const void* Kd, const void* Vd, const void* O, const float* LSE,
+                     const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
+                     void* ws, size_t ws_bytes, moda_stream_t stream) {
+    Problem p;
+    moda_status st = validate(shape, &p);
+    if (st != MODA_OK) return st;
+    if (p.B == 0 || p.T == 0) return MODA_OK;
+    if ((st = check_ptrs({{Q, "Q"}, {K, "K"}, {V, "V"}, {O, "O"}, {LSE, "LSE"}, {dO, "dO"},
+                          {dQ, "dQ"}, {dK, "dK"}, {dV, "dV"}})) != MODA_OK)
+        return st;
+    if (p.L > 0 &&
+        (st = check_ptrs({{Kd, "Kd"}, {Vd, "Vd"}, {dKd, "dKd"}, {dVd, "dVd"}})) != MODA_OK)
+        return st;
+    const size_t need = bwd_workspace_bytes(p);
+    if (!ws || ws_bytes < need)
+        return fail(MODA_ERR_WORKSPACE, "backward needs %zu workspace bytes (got %zu%s)", need,
+                    ws_bytes, ws ? "" : ", NULL");
+    if (!aligned16(ws)) return fail(MODA_ERR_MISALIGNED, "ws is not 16-byte aligned");
+    if (!device_status_word()) return fail(MODA_ERR_CUDA, "no usable CUDA device");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* Dws = static_cast<float*>(ws);
+    cudaError_t e =
+        p.elem_bytes == 2
+            ? launch_bwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, s)
+            : launch_bwd_simt(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, s);
+    return e == cudaSuccess ? MODA_OK : cuda_fail(e, "backward launch");
+}
+
+moda_status moda_check_status(moda_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned int* w = device_status_word();
+    if (!w) return fail(MODA_ERR_CUDA, "no usable CUDA device");
+    unsigned int v = 0;
+    e = cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (v) {
+        const unsigned int zero = 0;
+        e = cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "status clear");
+        if (v & kStatusTimeout) return fail(MODA_ERR_TIMEOUT, "a kernel wait timed out");
+    }
+    return MODA_OK;
+}
+
+const char* moda_status_string(moda_status status) {
+    switch (status) {
+        case MODA_OK: return "MODA_OK";
+        case MODA_ERR_INVALID_ARG: return "MODA_ERR_INVALID_ARG";
+        case MODA_ERR_MISALIGNED: return "MODA_ERR_MISALIGNED";
+        case MODA_ERR_UNSUPPORTED: return "MODA_ERR_UNSUPPORTED";
+        case MODA_ERR_WORKSPACE: return "MODA_ERR_WORKSPACE";
+        case MODA_ERR_CUDA: return "MODA_ERR_CUDA";
+        case MODA_ERR_TIMEOUT: return "MODA_ERR_TIMEOUT";
+    }
+    return "MODA_ERR_UNKNOWN";
+}
+
+const char* moda_last_error_message(void) { return g_last_error.c_str(); }
+
+int moda_version(void) { return 100; }
+
+}  // extern "C"

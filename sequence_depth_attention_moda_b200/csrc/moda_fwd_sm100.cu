@@ -1,0 +1,389 @@
+// moda_fwd_sm100.cu -- fused MoDA forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// Operator: paper summary of arXiv 2603.15619, "Mixture-of-Depths Attention
+// (MoDA): The Unified Operator" -- one softmax over the causal sequence keys
+// (j <= t) and the token's own L depth rows, scaled by 1/sqrt(d); the online
+// form is "Fused online-softmax (Algorithm 1)" (running max / sum / output in
+// base 2, sequence blocks then depth blocks, o / acc at the end).
+//
+// Work unit: one query tile of 128 rows = the G heads of one KV head times
+// Tq = 128/G consecutive tokens (row r -> head g = r / Tq, token t0 + r % Tq).
+// This is the pages' group-aware idea in B200 form: every K/V tile and every
+// depth tile is loaded once into shared memory and used by all G heads of the
+// group, and the depth rows of the tile's Tq tokens are one contiguous range
+// [t0*L, (t0+Tq)*L) of the token-major depth tensor.
+//
+// CTA roles (192 threads):
+//   warp 0      TMA producer: Q once, then K/V (or K_depth/V_depth) tiles
+//               through a 2-stage ring of mbarriers.
+//   warp 1      TMEM allocator and MMA issuer (one thread):
+//               S_i = Q K_i^T into one of two TMEM S buffers, then
+//               O += P_{i-1} V_{i-1} with P read from TMEM.
+//   warps 2..5  softmax, one thread per tile row: tcgen05.ld of S, masks,
+//               running max, exp2, row sum, P (bf16) written back over S with
+//               tcgen05.st; O in TMEM is rescaled only when the running max
+//               grew by more than 2^8 (exact: the final o / acc cancels it).
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "moda_internal.h"
+#include "moda_ptx.cuh"
+
+namespace moda {
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = 128;          // query rows per tile
+constexpr int BN = 128;          // sequence keys per block
+constexpr int kStages = 2;       // K/V shared-memory stages
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kSlabBytes = 128 * 128;   // 128 rows x 64 bf16
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;
+
+struct FwdArgs {
+    TmaMap tq, tk, tv, tkd, tvd;
+    __nv_bfloat16* O;
+    float* LSE;
+    unsigned int* status;
+    int B, Hq, Hk, T, L, G, Tq, n_qt, dep_rows;
+    float scale_log2;
+};
+
+template <int D>
+struct Layout {
+    static constexpr int kSlabs = D / 64;
+    static constexpr uint32_t kTile = kSlabs * kSlabBytes;
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kK = kTile;
+    static constexpr uint32_t kV = kK + kStages * kTile;
+    static constexpr uint32_t kBar = kV + kStages * kTile;
+    static constexpr uint32_t kBytes = kBar + 256;
+    // + alignment slack; never below 120 KB so that one CTA (and one 512-column
+    // TMEM allocation) is resident per SM.
+    static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
+};
+
+// Barrier slots.
+enum { kQFull = 0, kKFull = 1, kVFull = 3, kKVEmpty = 5, kSFull = 7, kPReady = 9, kOReady = 11,
+       kOFinal = 12, kNumBars = 13 };
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __grid_constant__ FwdArgs a) {
+    using Lay = Layout<D>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    unsigned char* sQ = smem + Lay::kQ;
+    unsigned char* sK = smem + Lay::kK;
+    unsigned char* sV = smem + Lay::kV;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Longest tiles first: block 0.. take the last query tiles of every head.
+    const int nbh = a.B * a.Hk;
+    const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / nbh;
+    const int bh = static_cast<int>(blockIdx.x) % nbh;
+    const int b = bh / a.Hk;
+    const int hk = bh - b * a.Hk;
+    const int t0 = qt * a.Tq;
+    const int R = a.G * a.Tq;
+    const int t_end = min(t0 + a.Tq, a.T);           // one past the last real token
+    const int n_seq = (t_end - 1) / BN + 1;
+    const int n_dep = a.L > 0 ? ((t_end - t0) * a.L + a.dep_rows - 1) / a.dep_rows : 0;
+    const int nb = n_seq + n_dep;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[kQFull], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars[kKFull + s], 1);
+            mbar_init(&bars[kVFull + s], 1);
+            mbar_init(&bars[kKVEmpty + s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kSFull + s], 1);
+            mbar_init(&bars[kPReady + s], kSoftmaxThreads);
+        }
+        mbar_init(&bars[kOReady], 1);
+        mbar_init(&bars[kOFinal], 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (R < BM) {  // rows the Q box does not cover: make them finite (zeros)
+        for (int i = threadIdx.x; i < Lay::kSlabs * (BM - R) * 8; i += kThreads) {
+            const int slab = i / ((BM - R) * 8);
+            const int rem = i - slab * (BM - R) * 8;
+            const int row = R + rem / 8;
+            reinterpret_cast<uint4*>(sQ + slab * kSlabBytes + row * 128)[rem % 8] =
+                make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer ----
+        if (lane == 0) {
+            prefetch_tmap(&a.tq);
+            prefetch_tmap(&a.tk);
+            prefetch_tmap(&a.tv);
+            if (a.L > 0) { prefetch_tmap(&a.tkd); prefetch_tmap(&a.tvd); }
+            const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
+            mbar_arrive_expect_tx(&bars[kQFull], q_bytes);
+            for (int s = 0; s < Lay::kSlabs; ++s)
+                tma_load_3d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, t0, b * a.Hq + hk * a.G);
+            int issued = 0;
+            for (int i = 0; i < nb; ++i) {
+                const int st = i % kStages;
+                if (i >= kStages &&
+                    !mbar_wait(&bars[kKVEmpty + st], ((i / kStages) - 1) & 1, a.status, abort_flag))
+                    break;
+                unsigned char* dk = sK + st * Lay::kTile;
+                unsigned char* dv = sV + st * Lay::kTile;
+                if (i < n_seq) {
+                    const uint32_t bytes = Lay::kTile;
+                    mbar_arrive_expect_tx(&bars[kKFull + st], bytes);
+                    for (int s = 0; s < Lay::kSlabs; ++s)
+                        tma_load_3d(dk + s * kSlabBytes, &a.tk, &bars[kKFull + st], s * 64, i * BN, bh);
+                    mbar_arrive_expect_tx(&bars[kVFull + st], bytes);
+                    for (int s = 0; s < Lay::kSlabs; ++s)
+                        tma_load_3d(dv + s * kSlabBytes, &a.tv, &bars[kVFull + st], s * 64, i * BN, bh);
+                } else {
+                    const int row0 = t0 * a.L + (i - n_seq) * a.dep_rows;
+                    const uint32_t bytes = Lay::kSlabs * 128u * a.dep_rows;
+                    mbar_arrive_expect_tx(&bars[kKFull + st], bytes);
+                    for (int s = 0; s < Lay::kSlabs; ++s)
+                        tma_load_3d(dk + s * kSlabBytes, &a.tkd, &bars[kKFull + st], s * 64, row0, bh);
+                    mbar_arrive_expect_tx(&bars[kVFull + st], bytes);
+                    for (int s = 0; s < Lay::kSlabs; ++s)
+                        tma_load_3d(dv + s * kSlabBytes, &a.tvd, &bars[kVFull + st], s * 64, row0, bh);
+                }
+                issued = i + 1;
+            }
+            // Let every load this thread started land before the CTA retires.
+            mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
+            for (int i = max(0, issued - kStages); i < issued; ++i) {
+                mbar_wait(&bars[kKFull + i % kStages], (i / kStages) & 1, a.status, abort_flag);
+                mbar_wait(&bars[kVFull + i % kStages], (i / kStages) & 1, a.status, abort_flag);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer --
+        if (lane == 0) {
+            const uint32_t id_seq = idesc_bf16(128, BN, false, false);
+            const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
+            const uint32_t id_pv = idesc_bf16(128, D, false, true);
+            const uint32_t q_addr = smem_u32(sQ);
+            bool ok = mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
+            auto issue_pv = [&](int j) -> bool {
+                const int st = j % kStages;
+                const int sb = j & 1;
+                if (!mbar_wait(&bars[kPReady + sb], (j >> 1) & 1, a.status, abort_flag)) return false;
+                if (!mbar_wait(&bars[kVFull + st], (j / kStages) & 1, a.status, abort_flag)) return false;
+                tc_fence_after();
+                const int krows = j < n_seq ? BN : a.dep_rows;
+                const uint32_t v_addr = smem_u32(sV + st * Lay::kTile);
+                for (int kk = 0; kk < krows / 16; ++kk) {
+                    const uint64_t bdesc = desc_mnmajor_sw128(v_addr + kk * 2048, kSlabBytes);
+                    umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, bdesc, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&bars[kKVEmpty + st]);
+                umma_commit(&bars[kOReady]);
+                return true;
+            };
+            for (int i = 0; ok && i < nb; ++i) {
+                const int st = i % kStages;
+                const int sb = i & 1;
+                if (!mbar_wait(&bars[kKFull + st], (i / kStages) & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(sK + st * Lay::kTile);
+                const uint32_t id = i < n_seq ? id_seq : id_dep;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    umma_ss(tmem + sb * 128, desc_kmajor_sw128(q_addr + off),
+                            desc_kmajor_sw128(k_addr + off), id, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[kSFull + sb]);
+                if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+            }
+            if (ok) ok = issue_pv(nb - 1);
+            umma_commit(&bars[kOFinal]);
+        }
+    } else {
+        // ------------------------------------------------------ softmax -----
+        const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
+        const int r = quarter * 32 + lane;            // tile row
+        const bool row_real = r < R;
+        const int g = row_real ? r / a.Tq : 0;
+        const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const float sl2 = a.scale_log2;
+        float m = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int i = 0; i < nb; ++i) {
+            const int sb = i & 1;
+            if (!mbar_wait(&bars[kSFull + sb], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[128];
+            const uint32_t s_addr = lane_base + sb * 128;
+            tmem_ld32(s_addr, sr);
+            tmem_ld32(s_addr + 32, sr + 32);
+            tmem_ld32(s_addr + 64, sr + 64);
+            tmem_ld32(s_addr + 96, sr + 96);
+            tmem_wait_ld();
+            float mx = -INFINITY;
+            if (i < n_seq) {
+                const int kb = i * BN;
+                if (kb + BN - 1 <= t_row) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        if (kb + c > t_row) sr[c] = __float_as_uint(-INFINITY);
+                        mx = fmaxf(mx, __uint_as_float(sr[c]));
+                    }
+                }
+            } else {
+                const int lo = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows);
+                const int hi = min(lo + a.L, a.dep_rows);
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    if (c < lo || c >= hi) sr[c] = __float_as_uint(-INFINITY);
+                    mx = fmaxf(mx, __uint_as_float(sr[c]));
+                }
+            }
+            const float m_new = fmaxf(m, mx * sl2);
+            if (i == 0) {
+                m = m_new;
+            } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
+                // O must hold P_{i-1} V_{i-1} before it is rescaled.  S_i was
+                // issued after PV_{i-2}, so at most PV_{i-1} is in flight.
+                if (!mbar_wait(&bars[kOReady], (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const float alpha = ex2(m - m_new);
+                l *= alpha;
+                m = m_new;
+#pragma unroll
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_base + kColO + c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(lane_base + kColO + c, o);
+                }
+                tmem_wait_st();
+            }
+            float rs = 0.0f;
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -m));
+                const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m));
+                rs += p0 + p1;
+                pk[c] = pack_bf16(p0, p1);
+            }
+            l += rs;
+            tmem_st32(s_addr, pk);
+            tmem_st32(s_addr + 32, pk + 32);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[kPReady + sb]);
+        }
+        // ---------------------------------------------------- epilogue ------
+        if (ok) ok = mbar_wait(&bars[kOFinal], 0, a.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            uint32_t o[D];
+#pragma unroll
+            for (int c = 0; c < D; c += 32) tmem_ld32(lane_base + kColO + c, o + c);
+            tmem_wait_ld();
+            if (row_real && t_row < a.T) {
+                const float inv = 1.0f / l;
+                const size_t qrow = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T + t_row;
+                uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D);
+#pragma unroll
+                for (int c = 0; c < D; c += 8) {
+                    uint4 v;
+                    v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv, __uint_as_float(o[c + 1]) * inv);
+                    v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+                    v.z = pack_bf16(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
+                    v.w = pack_bf16(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
+                    dst[c / 8] = v;
+                }
+                a.LSE[qrow] = (m + log2f(l)) * 0.6931471805599453f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D>
+cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void* V,
+                     const void* Kd, const void* Vd, void* O, float* LSE, cudaStream_t stream) {
+    FwdArgs a;
+    a.B = p.B; a.Hq = p.Hq; a.Hk = p.Hk; a.T = p.T; a.L = p.L; a.G = p.G;
+    a.Tq = BM / p.G;
+    a.n_qt = (p.T + a.Tq - 1) / a.Tq;
+    const int dep = a.Tq * p.L;
+    a.dep_rows = dep >= 128 ? 128 : ((dep + 15) / 16) * 16;
+    if (a.dep_rows < 16) a.dep_rows = 16;
+    a.scale_log2 = p.scale_log2;
+    a.O = static_cast<__nv_bfloat16*>(O);
+    a.LSE = LSE;
+    a.status = device_status_word();
+    cudaError_t e;
+    if ((e = make_tma_3d_bf16(&a.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, a.Tq, p.G)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&a.tk, K, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&a.tv, V, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
+    if (p.L > 0) {
+        const uint64_t rows = (uint64_t)p.T * p.L;
+        if ((e = make_tma_3d_bf16(&a.tkd, Kd, D, rows, (uint64_t)p.B * p.Hk, a.dep_rows, 1)) != cudaSuccess) return e;
+        if ((e = make_tma_3d_bf16(&a.tvd, Vd, D, rows, (uint64_t)p.B * p.Hk, a.dep_rows, 1)) != cudaSuccess) return e;
+    } else {
+        a.tkd = a.tk;
+        a.tvd = a.tv;
+    }
+    const uint32_t smem = Layout<D>::kDynSmem;
+    e = cudaFuncSetAttribute(moda_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long grid = (long long)p.B * p.Hk * a.n_qt;
+    moda_fwd_sm100_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
+                             const void* Kd, const void* Vd, void* O, float* LSE,
+                             cudaStream_t stream) {
+    if (p.d == 128) return launch_d<128>(p, Q, K, V, Kd, Vd, O, LSE, stream);
+    if (p.d == 64) return launch_d<64>(p, Q, K, V, Kd, Vd, O, LSE, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace moda

@@ -1,0 +1,63 @@
+// moda_internal.h -- interface between the C-ABI host layer (moda_api.cu) and
+// the kernel launchers.  Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moda {
+
+// A validated problem.  Index conventions follow the C ABI (include/moda.h).
+struct Problem {
+    int B, Hq, Hk, T, d, L, G;
+    float scale;        // softmax scale on the natural-log scale
+    float scale_log2;   // scale * log2(e): scores go straight into exp2
+    int elem_bytes;     // 2 (bf16) or 4 (fp32)
+};
+
+// Kernel-side status bits written into the per-device status word.
+enum : unsigned int {
+    kStatusTimeout = 1u,   // a bounded mbarrier / flag wait ran out
+};
+
+// Address of the calling device's status word (device memory), or nullptr.
+unsigned int* device_status_word();
+
+// SM count of the current device (cached).
+int device_sm_count();
+
+// ---- depth repack (moda_repack.cu) -----------------------------------------
+cudaError_t launch_repack(int B, int Hk, int T, int d, int L, int elem_bytes,
+                          const void* src, void* dst, cudaStream_t stream);
+
+// ---- CUDA-core path (moda_simt.cu): fp32 dtype; bf16 inputs for debugging --
+cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
+                            const void* Kd, const void* Vd, void* O, float* LSE,
+                            cudaStream_t stream);
+cudaError_t launch_bwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
+                            const void* Kd, const void* Vd, const void* O, const float* LSE,
+                            const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
+                            float* Dws, cudaStream_t stream);
+
+// ---- tensor-core path, sm_100a (moda_fwd_sm100.cu, moda_bwd_sm100.cu) -------
+// Each returns cudaSuccess, or an error; on error nothing was launched.
+cudaError_t launch_fwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
+                             const void* Kd, const void* Vd, void* O, float* LSE,
+                             cudaStream_t stream);
+cudaError_t launch_bwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
+                             const void* Kd, const void* Vd, const void* O, const float* LSE,
+                             const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
+                             float* Dws, cudaStream_t stream);
+
+// Workspace bytes the backward needs: D = rowsum(dO * O), fp32 [B, Hq, T].
+size_t bwd_workspace_bytes(const Problem& p);
+
+// ---- TMA descriptors (moda_tma.cu) -------------------------------------------
+// A 3-D bf16 tensor map over a row-major [outer, rows, d] tensor, box
+// [box_outer, box_rows, 64] with 128-byte swizzle (d split in 64-wide slabs).
+struct TmaMap { alignas(64) unsigned char bytes[128]; };
+cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t rows,
+                             uint64_t outer, uint32_t box_rows, uint32_t box_outer);
+
+}  // namespace moda

@@ -1,0 +1,176 @@
+"""Helpers shared by the GPU parity tests, the smoke check and the benchmark.
+
+``run_gpu`` drives the CUDA path through the C ABI (repack, forward, optional
+backward); ``oracle_*`` compute the fp64 CPU references on the same seeded
+inputs, either in full or for sampled rows / sampled (b, hk) slices (rows are
+independent in the forward, whole (b, hk) slices in the backward, so a sample
+is checked exactly).
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Iterable, List, Sequence, Tuple
+
+import numpy as np
+import torch
+
+import oracle
+import sequence_depth_attention_moda_b200 as moda
+from sequence_depth_attention_moda_b200.inputs import Workload, make_inputs
+
+# bf16 in / fp32 accumulate tolerances on the output (stated with the operator)
+BF16_MAX_ABS, BF16_MEAN_ABS = 2e-2, 2e-3
+FP32_MAX_ABS = 1e-4
+# LSE is fp32 statistics of exactly representable scores: tight.
+LSE_MAX_ABS = 1e-3
+# gradients: max |g - ref| <= 2e-2 * max(1, max|ref|), mean <= 2e-3 * max(1, mean|ref|)
+GRAD_MAX_REL, GRAD_MEAN_REL = 2e-2, 2e-3
+
+
+def shape_of(w: Workload, layout=moda.MODA_DEPTH_FLAT, C=None):
+    return moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C if C is None else C,
+                           moda.MODA_BF16 if w.dtype == "bf16" else moda.MODA_FP32, layout)
+
+
+def run_gpu(w: Workload, x: Dict[str, torch.Tensor], backward=None, layout=moda.MODA_DEPTH_FLAT,
+            C=None, null_depth_if_empty=True):
+    """Repack the depth cache, run the forward (and backward) on the current
+    stream; returns a dict of device tensors."""
+    sh = shape_of(w, layout, C)
+    dev = x["Q"].device
+    dt = x["Q"].dtype
+    out = {}
+    if w.L > 0:
+        Kd = torch.empty(w.B, w.Hk, w.T * w.L, w.d, device=dev, dtype=dt)
+        Vd = torch.empty_like(Kd)
+        moda.moda_repack_depth(sh, x["Kd_layer"], Kd)
+        moda.moda_repack_depth(sh, x["Vd_layer"], Vd)
+    else:
+        Kd = Vd = None if null_depth_if_empty else torch.empty(0, device=dev, dtype=dt)
+    out["Kd"], out["Vd"] = Kd, Vd
+    O = torch.empty_like(x["Q"])
+    LSE = torch.empty(w.B, w.Hq, w.T, device=dev, dtype=torch.float32)
+    moda.moda_fwd(sh, x["Q"], x["K"], x["V"], Kd, Vd, O, LSE)
+    out["O"], out["LSE"] = O, LSE
+    if backward if backward is not None else w.backward:
+        nws = moda.moda_workspace_size(sh, True)
+        ws = torch.empty(max(nws, 16), device=dev, dtype=torch.uint8)
+        dQ = torch.empty_like(x["Q"])
+        dK = torch.empty_like(x["K"])
+        dV = torch.empty_like(x["V"])
+        dKd = torch.empty_like(Kd) if Kd is not None else None
+        dVd = torch.empty_like(Vd) if Vd is not None else None
+        moda.moda_bwd(sh, x["Q"], x["K"], x["V"], Kd, Vd, O, LSE, x["dO"], dQ, dK, dV, dKd, dVd,
+                      ws, nws)
+        out.update(dQ=dQ, dK=dK, dV=dV, dKd=dKd, dVd=dVd)
+    return out
+
+
+def token_major(x: Dict[str, torch.Tensor], w: Workload) -> Tuple[torch.Tensor, torch.Tensor]:
+    """CPU token-major depth tensors via the oracle's repack (bytewise)."""
+    if w.L == 0:
+        e = torch.zeros(w.B, w.Hk, 0, w.d)
+        return e, e
+    res = []
+    for k in ("Kd_layer", "Vd_layer"):
+        src = x[k].cpu()
+        if src.dtype == torch.bfloat16:
+            u = src.view(torch.int16).numpy()
+            res.append(torch.from_numpy(oracle.repack(u, w.B, w.Hk, w.T, w.d, w.L)).view(torch.bfloat16))
+        else:
+            res.append(torch.from_numpy(oracle.repack(src.numpy(), w.B, w.Hk, w.T, w.d, w.L)))
+    return res[0], res[1]
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().double().numpy()
+
+
+def oracle_fwd_full(w, x):
+    Kd, Vd = token_major(x, w)
+    return oracle.fwd(f64(x["Q"]), f64(x["K"]), f64(x["V"]), f64(Kd) if w.L else None,
+                      f64(Vd) if w.L else None)
+
+
+def oracle_bwd_full(w, x):
+    Kd, Vd = token_major(x, w)
+    return oracle.bwd(f64(x["Q"]), f64(x["K"]), f64(x["V"]), f64(Kd), f64(Vd), f64(x["dO"]))
+
+
+def sample_rows(w: Workload, n_random: int, seed: int = 7) -> List[Tuple[int, int, int]]:
+    """(b, h, t) rows: first/last token, tile and chunk boundaries, randoms."""
+    rng = np.random.default_rng(seed)
+    Tq = 128 // w.G
+    ts = {0, 1, w.T - 1, w.T - 2, min(w.T - 1, Tq), max(0, Tq - 1), min(w.T - 1, 127),
+          min(w.T - 1, 128), min(w.T - 1, w.C), max(0, w.C - 1)}
+    ts = sorted(t for t in ts if 0 <= t < w.T)
+    rows = [(int(rng.integers(w.B)), int(rng.integers(w.Hq)), t) for t in ts]
+    for _ in range(n_random):
+        rows.append((int(rng.integers(w.B)), int(rng.integers(w.Hq)), int(rng.integers(w.T))))
+    rows.append((w.B - 1, w.Hq - 1, w.T - 1))
+    return rows
+
+
+def oracle_rows(w: Workload, x, Kd_dev, Vd_dev, rows: Sequence[Tuple[int, int, int]]):
+    """Oracle O and LSE for sampled rows; depth rows are read from the
+    token-major tensors gathered through the oracle's index definition."""
+    O = np.zeros((len(rows), w.d))
+    LSE = np.zeros(len(rows))
+    for i, (b, h, t) in enumerate(rows):
+        hk = h // w.G
+        q = f64(x["Q"][b, h, t])
+        Ks = f64(x["K"][b, hk, :t + 1])
+        Vs = f64(x["V"][b, hk, :t + 1])
+        if w.L:
+            # layer-major source: depth row l of token t is Kd_layer[l, b, hk, t]
+            Kdep = f64(x["Kd_layer"][:, b, hk, t])
+            Vdep = f64(x["Vd_layer"][:, b, hk, t])
+        else:
+            Kdep = Vdep = np.zeros((0, w.d))
+        O[i], LSE[i] = oracle.row(q, Ks, Vs, Kdep, Vdep)
+    return O, LSE
+
+
+def slice_workload(w: Workload, x, b: int, hk: int):
+    """The independent (b, hk) slice as a B=1, Hk=1 problem (CPU tensors)."""
+    G = w.G
+    ws = w.with_(B=1, Hq=G, Hk=1)
+    xs = {"Q": x["Q"][b:b + 1, hk * G:(hk + 1) * G].cpu(),
+          "K": x["K"][b:b + 1, hk:hk + 1].cpu(), "V": x["V"][b:b + 1, hk:hk + 1].cpu(),
+          "Kd_layer": x["Kd_layer"][:, b:b + 1, hk:hk + 1].cpu(),
+          "Vd_layer": x["Vd_layer"][:, b:b + 1, hk:hk + 1].cpu()}
+    if "dO" in x:
+        xs["dO"] = x["dO"][b:b + 1, hk * G:(hk + 1) * G].cpu()
+    return ws, xs
+
+
+def err_stats(got, ref) -> Tuple[float, float]:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if got.size == 0:
+        return 0.0, 0.0
+    d = np.abs(got - ref)
+    return float(d.max()), float(d.mean())
+
+
+def assert_out_close(got, ref, dtype: str, what: str):
+    mx, mean = err_stats(got, ref)
+    assert np.all(np.isfinite(np.asarray(got, dtype=np.float64))), f"{what}: non-finite values"
+    if dtype == "fp32":
+        assert mx <= FP32_MAX_ABS, f"{what}: max-abs {mx:.3e} > {FP32_MAX_ABS}"
+    else:
+        assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, \
+            f"{what}: max-abs {mx:.3e} (<= {BF16_MAX_ABS}), mean-abs {mean:.3e} (<= {BF16_MEAN_ABS})"
+
+
+def assert_grad_close(got, ref, what: str):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    if ref.size == 0:
+        return
+    mx, mean = err_stats(got, ref)
+    lim_mx = GRAD_MAX_REL * max(1.0, float(np.abs(ref).max()))
+    lim_mean = GRAD_MEAN_REL * max(1.0, float(np.abs(ref).mean()))
+    assert mx <= lim_mx and mean <= lim_mean, \
+        f"{what}: max-abs {mx:.3e} (<= {lim_mx:.3e}), mean-abs {mean:.3e} (<= {lim_mean:.3e})"

@@ -1,0 +1,110 @@
+"""The C-ABI library on the CPU: it builds, loads, exports every symbol the
+header declares, and its host-side validation rejects bad arguments before
+touching a device (no compute calls here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sequence_depth_attention_moda_b200 as moda
+from sequence_depth_attention_moda_b200 import build as moda_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moda_build.build()
+    return moda.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moda_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert header_functions() == sorted(moda.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", moda.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(moda_\w+)", out))
+    for name in header_functions():
+        assert name in exported, f"{name} declared in moda.h but not exported"
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    names = [moda.moda_status_string(i) for i in range(7)]
+    assert names == ["MODA_OK", "MODA_ERR_INVALID_ARG", "MODA_ERR_MISALIGNED",
+                     "MODA_ERR_UNSUPPORTED", "MODA_ERR_WORKSPACE", "MODA_ERR_CUDA",
+                     "MODA_ERR_TIMEOUT"]
+    assert moda.moda_version() >= 100
+
+
+def call_fwd(lib, sh, ptrs):
+    return lib.moda_fwd(ctypes.byref(sh), *ptrs, None, 0, None)
+
+
+FAKE = 0x10000   # aligned fake device address: never dereferenced (validation fails first)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=6, Hk=4), 1),                                         # Hq % Hk
+    (dict(d=96), 3),                                                     # bf16 d
+    (dict(Hq=256, Hk=1), 3),                                             # G > 128
+    (dict(T=-1), 1),
+    (dict(L=-2), 1),
+    (dict(dtype=7), 1),
+    (dict(depth_layout=1, C=0), 1),                                      # chunked needs C
+    (dict(depth_layout=1, C=48), 1),                                     # T % C
+])
+def test_fwd_rejects_bad_shapes(lib, kw, status):
+    base = dict(B=1, Hq=4, Hk=2, T=64, d=128, L=2, C=16)
+    base.update(kw)
+    sh = moda.make_shape(**base)
+    rc = call_fwd(lib, sh, [FAKE] * 7)
+    assert rc == status, (rc, moda.moda_last_error_message())
+    assert moda.moda_last_error_message()
+
+
+def test_fwd_rejects_null_and_misaligned(lib):
+    sh = moda.make_shape(1, 4, 2, 64, 128, 2, 16)
+    assert call_fwd(lib, sh, [FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE]) == 1
+    assert "V" in moda.moda_last_error_message()
+    assert call_fwd(lib, sh, [FAKE, FAKE + 2, FAKE, FAKE, FAKE, FAKE, FAKE]) == 2
+    assert call_fwd(lib, sh, [FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE]) == 1   # Kd with L > 0
+
+
+def test_bwd_rejects_small_workspace(lib):
+    sh = moda.make_shape(1, 4, 2, 64, 128, 2, 16)
+    need = lib.moda_workspace_size(ctypes.byref(sh), 1)
+    assert need == 4 * 4 * 64  # fp32 D = rowsum(dO * O), [B, Hq, T], 256-byte rounded
+    rc = lib.moda_bwd(ctypes.byref(sh), *([FAKE] * 13), FAKE, need - 1, None)
+    assert rc == 4
+    rc = lib.moda_bwd(ctypes.byref(sh), *([FAKE] * 13), None, need, None)
+    assert rc == 4
+
+
+def test_workspace_sizes(lib):
+    sh = moda.make_shape(2, 16, 4, 4096, 128, 16, 64)
+    assert lib.moda_workspace_size(ctypes.byref(sh), 0) == 0
+    assert lib.moda_workspace_size(ctypes.byref(sh), 1) == 2 * 16 * 4096 * 4
+    bad = moda.make_shape(2, 16, 5, 4096, 128, 16, 64)
+    assert lib.moda_workspace_size(ctypes.byref(bad), 1) == ctypes.c_size_t(-1).value
+
+
+def test_empty_problems_are_noops(lib):
+    # B = 0 or T = 0: valid, nothing queued, NULL pointers allowed
+    for kw in (dict(B=0), dict(T=0)):
+        base = dict(B=1, Hq=4, Hk=2, T=64, d=128, L=2, C=16)
+        base.update(kw)
+        sh = moda.make_shape(**base)
+        assert call_fwd(lib, sh, [None] * 7) == 0
+        assert lib.moda_repack_depth(ctypes.byref(sh), None, None, None) == 0

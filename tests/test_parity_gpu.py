@@ -1,0 +1,234 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle
+on the same seeded inputs.
+
+Tolerances (bf16 in / fp32 accumulate): output max-abs <= 2e-2 and mean-abs
+<= 2e-3; fp32 path max-abs <= 1e-4; LSE max-abs <= 1e-3; gradients max-abs <=
+2e-2 * max(1, max|ref|) and mean-abs <= 2e-3 * max(1, mean|ref|).  Small
+cases are compared element by element in full; the full-size workloads on
+sampled rows (forward) and sampled (b, hk) slices (backward), which the
+oracle computes exactly for what they cover.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sequence_depth_attention_moda_b200 as moda
+from sequence_depth_attention_moda_b200 import inputs as I
+from moda_cases import (LSE_MAX_ABS, assert_grad_close, assert_out_close, err_stats, f64,
+                        oracle_bwd_full, oracle_fwd_full, oracle_rows, run_gpu, sample_rows,
+                        slice_workload, token_major)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+# (B, Hq, Hk, d, T, L): ragged T, every G the tile handles (incl. G not dividing 128), d in {64,128}
+SMALL = [
+    (1, 4, 2, 128, 300, 4),
+    (2, 8, 2, 64, 257, 3),
+    (1, 4, 4, 128, 200, 1),
+    (1, 16, 2, 128, 130, 16),
+    (1, 6, 2, 128, 100, 5),
+    (1, 4, 2, 128, 256, 0),
+    (1, 2, 1, 128, 1, 7),
+    (1, 32, 1, 64, 64, 2),
+    (1, 128, 1, 64, 9, 3),
+    (1, 8, 2, 128, 513, 40),
+]
+
+
+def small_w(B, Hq, Hk, d, T, L, seed=2024, backward=False):
+    return I.Workload(f"small_{B}_{Hq}_{Hk}_{d}_{T}_{L}", B=B, Hq=Hq, Hk=Hk, d=d, T=T, L=L, C=1,
+                      seed=seed, backward=backward)
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    yield
+    moda.moda_check_status()
+
+
+# ------------------------------------------------------------------ repack --
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_repack_bit_exact(dtype):
+    w = I.Workload("rp", B=2, Hq=4, Hk=2, d=128 if dtype == "bf16" else 40, T=37, L=5, C=1,
+                   dtype=dtype, seed=5)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x, backward=False)
+    Kd_ref, Vd_ref = token_major(x, w)
+    assert torch.equal(out["Kd"].cpu(), Kd_ref) and torch.equal(out["Vd"].cpu(), Vd_ref)
+
+
+def test_repack_bit_exact_full_size():
+    w = I.TRAIN_FWD_BWD
+    x = I.make_inputs(w, device=DEV, grad_out=False)
+    sh = moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C)
+    Kd = torch.empty(w.B, w.Hk, w.T * w.L, w.d, device=DEV, dtype=torch.bfloat16)
+    moda.moda_repack_depth(sh, x["Kd_layer"], Kd)
+    rng = np.random.default_rng(3)
+    for _ in range(64):
+        b, hk, t, l = (int(rng.integers(n)) for n in (w.B, w.Hk, w.T, w.L))
+        assert torch.equal(Kd[b, hk, t * w.L + l], x["Kd_layer"][l, b, hk, t])
+    # every byte moved: the multiset of row sums is preserved
+    assert torch.equal(Kd.float().sum(dim=(0, 1, 2)), x["Kd_layer"].float().sum(dim=(0, 1, 2, 3)))
+
+
+# ------------------------------------------------------------------ forward -
+def test_fwd_fp32_tiny_config():
+    w = I.TINY_FP32
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x)
+    O, LSE = oracle_fwd_full(w, x)
+    assert_out_close(f64(out["O"]), O, "fp32", "O")
+    assert err_stats(f64(out["LSE"]), LSE)[0] <= 1e-4
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "B%d_Hq%d_Hk%d_d%d_T%d_L%d" % c)
+def test_fwd_bf16_small(case):
+    w = small_w(*case)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x, backward=False)
+    O, LSE = oracle_fwd_full(w, x)
+    assert_out_close(f64(out["O"]), O, "bf16", "O")
+    assert err_stats(f64(out["LSE"]), LSE)[0] <= LSE_MAX_ABS
+
+
+def test_fwd_qk_scaled_distribution_small():
+    w = small_w(2, 16, 4, 128, 700, 16).with_(qk_scaled=True)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x, backward=False)
+    O, LSE = oracle_fwd_full(w, x)
+    assert_out_close(f64(out["O"]), O, "bf16", "O")
+
+
+def _check_rows(w, x, out, n_random=24):
+    rows = sample_rows(w, n_random)
+    O_ref, LSE_ref = oracle_rows(w, x, out["Kd"], out["Vd"], rows)
+    got = np.stack([f64(out["O"][b, h, t]) for (b, h, t) in rows])
+    lse = np.array([float(out["LSE"][b, h, t]) for (b, h, t) in rows])
+    assert_out_close(got, O_ref, w.dtype, f"{w.name} O rows")
+    assert err_stats(lse, LSE_ref)[0] <= LSE_MAX_ABS, f"{w.name} LSE rows"
+
+
+def test_fwd_layer_T4k_sampled():
+    w = I.LAYER_1P5B
+    x = I.make_inputs(w, device=DEV)
+    _check_rows(w, x, run_gpu(w, x, backward=False))
+
+
+@pytest.mark.parametrize("L", [32, 0])
+def test_fwd_long_context_T64k_sampled(L):
+    w = I.LONG_64K.with_(L=L)
+    x = I.make_inputs(w, device=DEV)
+    _check_rows(w, x, run_gpu(w, x, backward=False), n_random=16)
+
+
+def test_fwd_depth_group_sweep_sampled():
+    for w in I.depth_group_sweep():
+        x = I.make_inputs(w, device=DEV)
+        _check_rows(w, x, run_gpu(w, x, backward=False, layout=moda.MODA_DEPTH_CHUNKED), n_random=6)
+        del x
+        torch.cuda.empty_cache()
+
+
+def test_fwd_train_shape_sampled():
+    w = I.TRAIN_FWD_BWD
+    x = I.make_inputs(w, device=DEV, grad_out=False)
+    _check_rows(w, x, run_gpu(w, x, backward=False))
+
+
+def test_fwd_bitwise_identical_across_layouts_and_C():
+    w = small_w(1, 16, 4, 128, 1024, 8)
+    x = I.make_inputs(w, device=DEV)
+    ref = run_gpu(w, x, backward=False)
+    for C in (32, 64, 128, 1024):
+        o = run_gpu(w, x, backward=False, layout=moda.MODA_DEPTH_CHUNKED, C=C)
+        assert torch.equal(o["O"], ref["O"]) and torch.equal(o["LSE"], ref["LSE"])
+
+
+def test_fwd_deterministic():
+    w = small_w(2, 8, 2, 128, 777, 9)
+    x = I.make_inputs(w, device=DEV)
+    a = run_gpu(w, x, backward=False)
+    b = run_gpu(w, x, backward=False)
+    assert torch.equal(a["O"], b["O"]) and torch.equal(a["LSE"], b["LSE"])
+
+
+# ----------------------------------------------------------------- backward -
+BWD_SMALL = [c for c in SMALL if c[4] > 1] + [(1, 4, 2, 128, 1, 3)]
+
+
+@pytest.mark.parametrize("case", BWD_SMALL, ids=lambda c: "B%d_Hq%d_Hk%d_d%d_T%d_L%d" % c)
+def test_bwd_bf16_small(case):
+    w = small_w(*case, backward=True)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x)
+    ref = oracle_bwd_full(w, x)
+    for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), ref):
+        if out[name] is None:
+            assert r.size == 0
+            continue
+        assert_grad_close(f64(out[name]), r, name)
+
+
+def test_bwd_fp32_tiny():
+    w = I.TINY_FP32.with_(backward=True)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x)
+    ref = oracle_bwd_full(w, x)
+    for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), ref):
+        assert err_stats(f64(out[name]), r)[0] <= 1e-4, name
+
+
+def _check_slices(w, x, out, slices):
+    for (b, hk) in slices:
+        ws, xs = slice_workload(w, x, b, hk)
+        ref = oracle_bwd_full(ws, xs)
+        G = w.G
+        got = {"dQ": out["dQ"][b:b + 1, hk * G:(hk + 1) * G], "dK": out["dK"][b:b + 1, hk:hk + 1],
+               "dV": out["dV"][b:b + 1, hk:hk + 1], "dKd": out["dKd"][b:b + 1, hk:hk + 1],
+               "dVd": out["dVd"][b:b + 1, hk:hk + 1]}
+        for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), ref):
+            assert_grad_close(f64(got[name]), r, f"{w.name} slice ({b},{hk}) {name}")
+
+
+def test_bwd_layer_T4k_sampled_slices():
+    w = I.LAYER_1P5B
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x)
+    _check_rows(w, x, out)
+    _check_slices(w, x, out, [(1, 3)])
+
+
+def test_bwd_train_shape_sampled_slice():
+    w = I.TRAIN_FWD_BWD
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x)
+    _check_slices(w, x, out, [(7, 5)])
+
+
+def test_bwd_deterministic():
+    w = small_w(1, 8, 2, 128, 300, 6, backward=True)
+    x = I.make_inputs(w, device=DEV)
+    a = run_gpu(w, x)
+    b = run_gpu(w, x)
+    for k in ("dQ", "dK", "dV", "dKd", "dVd"):
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_bwd_workspace_error_on_device():
+    w = small_w(1, 4, 2, 128, 64, 2, backward=True)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x, backward=False)
+    sh = moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C)
+    need = moda.moda_workspace_size(sh, True)
+    ws = torch.empty(need, device=DEV, dtype=torch.uint8)
+    g = {k: torch.empty_like(v) for k, v in (("dQ", x["Q"]), ("dK", x["K"]), ("dV", x["V"]),
+                                            ("dKd", out["Kd"]), ("dVd", out["Vd"]))}
+    with pytest.raises(moda.MoDAError) as ei:
+        moda.moda_bwd(sh, x["Q"], x["K"], x["V"], out["Kd"], out["Vd"], out["O"], out["LSE"],
+                      x["dO"], g["dQ"], g["dK"], g["dV"], g["dKd"], g["dVd"], ws, need - 16)
+    assert ei.value.status == 4
