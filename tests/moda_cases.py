@@ -23,8 +23,11 @@ BF16_MAX_ABS, BF16_MEAN_ABS = 2e-2, 2e-3
 FP32_MAX_ABS = 1e-4
 # LSE is fp32 statistics of exactly representable scores: tight.
 LSE_MAX_ABS = 1e-3
-# gradients: max |g - ref| <= 2e-2 * max(1, max|ref|), mean <= 2e-3 * max(1, mean|ref|)
-GRAD_MAX_REL, GRAD_MEAN_REL = 2e-2, 2e-3
+# gradients (the pages state none): max |g - ref| <= 2e-2 * max(1, max|ref|) and
+# mean |g - ref| <= 5e-3 * max(1, mean|ref|).  Rounding a gradient to bf16 on
+# store costs up to 2^-9 relative (about 2e-3 on average over a tensor), and the
+# bf16 P / dS operands of the tensor-core products add the same order again.
+GRAD_MAX_REL, GRAD_MEAN_REL = 2e-2, 5e-3
 
 
 def shape_of(w: Workload, layout=moda.MODA_DEPTH_FLAT, C=None):

@@ -3,7 +3,8 @@ on the same seeded inputs.
 
 Tolerances (bf16 in / fp32 accumulate): output max-abs <= 2e-2 and mean-abs
 <= 2e-3; fp32 path max-abs <= 1e-4; LSE max-abs <= 1e-3; gradients max-abs <=
-2e-2 * max(1, max|ref|) and mean-abs <= 2e-3 * max(1, mean|ref|).  Small
+2e-2 * max(1, max|ref|) and mean-abs <= 5e-3 * max(1, mean|ref|) (storing a
+gradient in bf16 alone costs up to ~2e-3 relative on average).  Small
 cases are compared element by element in full; the full-size workloads on
 sampled rows (forward) and sampled (b, hk) slices (backward), which the
 oracle computes exactly for what they cover.
@@ -72,8 +73,9 @@ def test_repack_bit_exact_full_size():
     for _ in range(64):
         b, hk, t, l = (int(rng.integers(n)) for n in (w.B, w.Hk, w.T, w.L))
         assert torch.equal(Kd[b, hk, t * w.L + l], x["Kd_layer"][l, b, hk, t])
-    # every byte moved: the multiset of row sums is preserved
-    assert torch.equal(Kd.float().sum(dim=(0, 1, 2)), x["Kd_layer"].float().sum(dim=(0, 1, 2, 3)))
+    # the whole tensor, bit for bit, against the library's own permute
+    ref = x["Kd_layer"].permute(1, 2, 3, 0, 4).reshape(w.B, w.Hk, w.T * w.L, w.d)
+    assert torch.equal(Kd, ref)
 
 
 # ------------------------------------------------------------------ forward -
