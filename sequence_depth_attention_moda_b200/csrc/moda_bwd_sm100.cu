@@ -1,13 +1,716 @@
-// moda_bwd_sm100.cu -- backward launcher for the bf16 path.
+// moda_bwd_sm100.cu -- MoDA backward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// The pages give no backward formulas; this is the derivative of the forward
+// definition (paper summary of arXiv 2603.15619, "Mixture-of-Depths Attention
+// (MoDA): The Unified Operator": one softmax over [causal sequence keys |
+// the token's own L depth rows]).  With P the softmax weights recomputed from
+// the saved LSE, and D = rowsum(dO * O):
+//     dS = P * (dO . v - D)
+//     dQ = scale * (sum_j dS_j K_j + sum_l dS'_l Kd_l)
+//     dK_j = scale * sum over the group's heads and rows t >= j of dS q
+//     dV_j = sum over the same rows of P dO
+//     dKd[t*L+l] = scale * sum over the group's heads of dS'_l q[h,t]
+//     dVd[t*L+l] = sum over the group's heads of P'_l dO[h,t]
+//
+// Three launches, no floating-point atomics (bitwise repeatable):
+//  1. rowdot:  D[b,h,t] = sum_c dO * O                      (CUDA cores, HBM)
+//  2. dkdv:    one CTA per 128-key tile of one KV head.  M = 128 keys:
+//              S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and dS^T written
+//              back to TMEM as bf16, then dV += P^T dO and dK += dS^T Q with
+//              the A operand read from TMEM.  The group's G heads are all
+//              iterated inside the CTA, so dK/dV are complete sums.
+//  3. dq:      one CTA per 128-row query tile (G heads x 128/G tokens, as in
+//              the forward).  S = Q K^T, dP = dO V^T, dQ += dS K over the
+//              causal sequence blocks and then the tile's depth blocks.  For
+//              a depth block, P' and dS' (bf16) are also staged in shared
+//              memory, and the token-local depth gradients come out as
+//              dKd^T = Q^T dS' and dVd^T = dO^T P' (M = d, N = depth rows):
+//              each depth row belongs to exactly one query tile, so these
+//              are complete without atomics.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
 #include "moda_internal.h"
+#include "moda_ptx.cuh"
 
 namespace moda {
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kThreads = 192;            // warp 0 TMA, warp 1 MMA, warps 2..5 math
+constexpr int kMathThreads = 128;
+constexpr uint32_t kSlabBytes = 128 * 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------ 1. rowdot ----
+template <int D>
+__global__ void __launch_bounds__(256) rowdot_kernel(long long nrows,
+                                                      const __nv_bfloat16* __restrict__ O,
+                                                      const __nv_bfloat16* __restrict__ dO,
+                                                      float* __restrict__ Dout) {
+    constexpr int kLanesPerRow = D / 8;              // 16 B per lane
+    constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+    const int lane = threadIdx.x & 31;
+    const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const long long row = warp * kRowsPerWarp + lane / kLanesPerRow;
+    float s = 0.0f;
+    if (row < nrows) {
+        const uint4 a = reinterpret_cast<const uint4*>(O + row * D)[lane % kLanesPerRow];
+        const uint4 b = reinterpret_cast<const uint4*>(dO + row * D)[lane % kLanesPerRow];
+        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(pa[e]);
+            const float2 fb = __bfloat1622float2(pb[e]);
+            s = fmaf(fa.x, fb.x, s);
+            s = fmaf(fa.y, fb.y, s);
+        }
+    }
+#pragma unroll
+    for (int o = kLanesPerRow / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (row < nrows && lane % kLanesPerRow == 0) Dout[row] = s;
+}
+
+// -------------------------------------------------------------- 2. dkdv ----
+struct DkdvArgs {
+    TmaMap tk, tv, tq, tdo;
+    const float* LSE;
+    const float* Drow;
+    __nv_bfloat16* dK;
+    __nv_bfloat16* dV;
+    unsigned int* status;
+    int B, Hq, Hk, T, G, n_kt, n_qb;
+    float scale, scale_log2;
+};
+
+template <int D>
+struct DkdvLayout {
+    static constexpr int kSlabs = D / 64;
+    static constexpr uint32_t kTile = kSlabs * kSlabBytes;
+    static constexpr uint32_t kK = 0;
+    static constexpr uint32_t kV = kTile;
+    static constexpr uint32_t kQ = 2 * kTile;            // 2 stages
+    static constexpr uint32_t kDO = 4 * kTile;           // 2 stages
+    static constexpr uint32_t kStat = 6 * kTile;         // 2 x (lse2[128], D[128]) floats
+    static constexpr uint32_t kBar = kStat + 2048;
+    static constexpr uint32_t kBytes = kBar + 256;
+    static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
+};
+
+enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 3, kA_SFull = 5, kA_PReady = 6, kA_Final = 7,
+       kA_NumBars = 8 };
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant__ DkdvArgs a) {
+    using Lay = DkdvLayout<D>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kA_NumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    float* stat = reinterpret_cast<float*>(smem + Lay::kStat);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nbh = a.B * a.Hk;
+    const int kt = static_cast<int>(blockIdx.x) / nbh;     // small kt = most work: first
+    const int bh = static_cast<int>(blockIdx.x) % nbh;
+    const int b = bh / a.Hk;
+    const int hk = bh - b * a.Hk;
+    const int nqb = a.n_qb - kt;                            // query blocks qb = kt .. n_qb-1
+    const int n_it = a.G * nqb;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[kA_KVFull], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kA_QFull + s], 1);
+            mbar_init(&bars[kA_QEmpty + s], 1);
+        }
+        mbar_init(&bars[kA_SFull], 1);
+        mbar_init(&bars[kA_PReady], kMathThreads);
+        mbar_init(&bars[kA_Final], 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&a.tk); prefetch_tmap(&a.tv); prefetch_tmap(&a.tq); prefetch_tmap(&a.tdo);
+            mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * Lay::kTile);
+            for (int s = 0; s < Lay::kSlabs; ++s) {
+                tma_load_3d(smem + Lay::kK + s * kSlabBytes, &a.tk, &bars[kA_KVFull], s * 64, kt * BN, bh);
+                tma_load_3d(smem + Lay::kV + s * kSlabBytes, &a.tv, &bars[kA_KVFull], s * 64, kt * BN, bh);
+            }
+            int issued = 0;
+            for (int it = 0; it < n_it; ++it) {
+                const int st = it & 1;
+                if (it >= 2 && !mbar_wait(&bars[kA_QEmpty + st], ((it >> 1) - 1) & 1, a.status, abort_flag))
+                    break;
+                const int g = it / nqb;
+                const int qb = kt + (it - g * nqb);
+                const int qh = b * a.Hq + hk * a.G + g;
+                mbar_arrive_expect_tx(&bars[kA_QFull + st], 2 * Lay::kTile);
+                for (int s = 0; s < Lay::kSlabs; ++s) {
+                    tma_load_3d(smem + Lay::kQ + st * Lay::kTile + s * kSlabBytes, &a.tq,
+                                &bars[kA_QFull + st], s * 64, qb * BM, qh);
+                    tma_load_3d(smem + Lay::kDO + st * Lay::kTile + s * kSlabBytes, &a.tdo,
+                                &bars[kA_QFull + st], s * 64, qb * BM, qh);
+                }
+                issued = it + 1;
+            }
+            mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
+            for (int it = max(0, issued - 2); it < issued; ++it)
+                mbar_wait(&bars[kA_QFull + (it & 1)], (it >> 1) & 1, a.status, abort_flag);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(128, BM, false, false);
+            const uint32_t id_g = idesc_bf16(128, D, false, true);
+            const uint32_t k_addr = smem_u32(smem + Lay::kK);
+            const uint32_t v_addr = smem_u32(smem + Lay::kV);
+            bool ok = mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
+            for (int it = 0; ok && it < n_it; ++it) {
+                const int st = it & 1;
+                if (!mbar_wait(&bars[kA_QFull + st], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kTile);
+                const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kTile);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    umma_ss(tmem + 0, desc_kmajor_sw128(k_addr + off), desc_kmajor_sw128(q_addr + off),
+                            id_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    umma_ss(tmem + 128, desc_kmajor_sw128(v_addr + off), desc_kmajor_sw128(do_addr + off),
+                            id_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[kA_SFull]);
+                if (!mbar_wait(&bars[kA_PReady], it & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BM / 16; ++kk) {
+                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                    umma_ts(tmem + 256, tmem + 0 + kk * 8,
+                            desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes), id_g, acc);
+                    umma_ts(tmem + 384, tmem + 128 + kk * 8,
+                            desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes), id_g, acc);
+                }
+                umma_commit(&bars[kA_QEmpty + st]);
+            }
+            umma_commit(&bars[kA_Final]);
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int kr = quarter * 32 + lane;               // key row within the tile
+        const int k = kt * BN + kr;
+        const int mt = threadIdx.x - 64;                  // 0..127 among the math threads
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const float sl2 = a.scale_log2;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int g = it / nqb;
+            const int qb = kt + (it - g * nqb);
+            const size_t qrow0 = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T;
+            float* sbuf = stat + (it & 1) * 256;
+            {
+                const int t = qb * BM + mt;
+                sbuf[mt] = t < a.T ? a.LSE[qrow0 + t] * kLog2e : INFINITY;
+                sbuf[128 + mt] = t < a.T ? a.Drow[qrow0 + t] : 0.0f;
+            }
+            named_bar_sync(1, kMathThreads);
+            if (!mbar_wait(&bars[kA_SFull], it & 1, a.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const bool diag = qb == kt;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t s[32], dp[32], pk[16], dk[16];
+                tmem_ld32(lane_base + 32 * c4, s);
+                tmem_ld32(lane_base + 128 + 32 * c4, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float p2[2], d2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int c = 32 * c4 + e + u;
+                        const bool vis = !diag || k <= qb * BM + c;
+                        const float p = vis ? ex2(fmaf(__uint_as_float(s[e + u]), sl2, -sbuf[c])) : 0.0f;
+                        p2[u] = p;
+                        d2[u] = vis ? p * (__uint_as_float(dp[e + u]) - sbuf[128 + c]) : 0.0f;
+                    }
+                    pk[e / 2] = pack_bf16(p2[0], p2[1]);
+                    dk[e / 2] = pack_bf16(d2[0], d2[1]);
+                }
+                tmem_st16(lane_base + 16 * c4, pk);
+                tmem_st16(lane_base + 128 + 16 * c4, dk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[kA_PReady]);
+        }
+        if (ok) ok = mbar_wait(&bars[kA_Final], 0, a.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            // dK (scaled) then dV, one row of D values at a time
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                uint32_t gr[D];
+#pragma unroll
+                for (int c = 0; c < D; c += 32) tmem_ld32(lane_base + (which ? 256 : 384) + c, gr + c);
+                tmem_wait_ld();
+                if (k < a.T) {
+                    const size_t row = static_cast<size_t>(bh) * a.T + k;
+                    uint4* dst = reinterpret_cast<uint4*>((which ? a.dV : a.dK) + row * D);
+                    const float sc = which ? 1.0f : a.scale;
+#pragma unroll
+                    for (int c = 0; c < D; c += 8) {
+                        uint4 u;
+                        u.x = pack_bf16(__uint_as_float(gr[c]) * sc, __uint_as_float(gr[c + 1]) * sc);
+                        u.y = pack_bf16(__uint_as_float(gr[c + 2]) * sc, __uint_as_float(gr[c + 3]) * sc);
+                        u.z = pack_bf16(__uint_as_float(gr[c + 4]) * sc, __uint_as_float(gr[c + 5]) * sc);
+                        u.w = pack_bf16(__uint_as_float(gr[c + 6]) * sc, __uint_as_float(gr[c + 7]) * sc);
+                        dst[c / 8] = u;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- 3. dq ----
+struct DqArgs {
+    TmaMap tq, tdo, tk, tv, tkd, tvd;
+    const float* LSE;
+    const float* Drow;
+    __nv_bfloat16* dQ;
+    __nv_bfloat16* dKd;
+    __nv_bfloat16* dVd;
+    unsigned int* status;
+    int B, Hq, Hk, T, L, G, Tq, n_qt, dep_rows;
+    float scale, scale_log2;
+};
+
+template <int D>
+struct DqLayout {
+    static constexpr int kSlabs = D / 64;
+    static constexpr uint32_t kTile = kSlabs * kSlabBytes;
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kDO = kTile;
+    static constexpr uint32_t kK = 2 * kTile;        // 2 stages
+    static constexpr uint32_t kV = 4 * kTile;        // 2 stages
+    static constexpr uint32_t kDS = 6 * kTile;       // [128 q rows][64 depth] bf16, 128-B swizzle
+    static constexpr uint32_t kP = kDS + kSlabBytes;
+    static constexpr uint32_t kBar = kP + kSlabBytes;
+    static constexpr uint32_t kBytes = kBar + 256;
+    static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
+};
+
+enum { kB_QFull = 0, kB_KFull = 1, kB_VFull = 3, kB_KVEmpty = 5, kB_SFull = 7, kB_PReady = 8,
+       kB_DDFull = 9, kB_Final = 10, kB_NumBars = 11 };
+
+// TMEM columns of the dq kernel.
+constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDKd = 384, kColDVd = 448;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__ DqArgs a) {
+    using Lay = DqLayout<D>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kB_NumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nbh = a.B * a.Hk;
+    const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / nbh;
+    const int bh = static_cast<int>(blockIdx.x) % nbh;
+    const int b = bh / a.Hk;
+    const int hk = bh - b * a.Hk;
+    const int t0 = qt * a.Tq;
+    const int R = a.G * a.Tq;
+    const int t_end = min(t0 + a.Tq, a.T);
+    const int n_seq = (t_end - 1) / BN + 1;
+    const int dep_total = a.L > 0 ? (t_end - t0) * a.L : 0;
+    const int n_dep = (dep_total + a.dep_rows - 1) / a.dep_rows;
+    const int nb = n_seq + n_dep;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[kB_QFull], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kB_KFull + s], 1);
+            mbar_init(&bars[kB_VFull + s], 1);
+            mbar_init(&bars[kB_KVEmpty + s], 1);
+        }
+        mbar_init(&bars[kB_SFull], 1);
+        mbar_init(&bars[kB_PReady], kMathThreads);
+        mbar_init(&bars[kB_DDFull], 1);
+        mbar_init(&bars[kB_Final], 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (R < BM) {  // rows the Q / dO boxes do not cover: zeros
+        for (int i = threadIdx.x; i < 2 * Lay::kSlabs * (BM - R) * 8; i += kThreads) {
+            const int per = (BM - R) * 8;
+            const int which = i / (Lay::kSlabs * per);       // 0: Q, 1: dO
+            const int rem0 = i - which * Lay::kSlabs * per;
+            const int slab = rem0 / per;
+            const int rem = rem0 - slab * per;
+            const int row = R + rem / 8;
+            reinterpret_cast<uint4*>(smem + (which ? Lay::kDO : Lay::kQ) + slab * kSlabBytes +
+                                     row * 128)[rem % 8] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&a.tq); prefetch_tmap(&a.tdo); prefetch_tmap(&a.tk); prefetch_tmap(&a.tv);
+            if (a.L > 0) { prefetch_tmap(&a.tkd); prefetch_tmap(&a.tvd); }
+            const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
+            mbar_arrive_expect_tx(&bars[kB_QFull], 2 * q_bytes);
+            for (int s = 0; s < Lay::kSlabs; ++s) {
+                tma_load_3d(smem + Lay::kQ + s * kSlabBytes, &a.tq, &bars[kB_QFull], s * 64, t0, b * a.Hq + hk * a.G);
+                tma_load_3d(smem + Lay::kDO + s * kSlabBytes, &a.tdo, &bars[kB_QFull], s * 64, t0, b * a.Hq + hk * a.G);
+            }
+            int issued = 0;
+            for (int i = 0; i < nb; ++i) {
+                const int st = i & 1;
+                if (i >= 2 && !mbar_wait(&bars[kB_KVEmpty + st], ((i >> 1) - 1) & 1, a.status, abort_flag))
+                    break;
+                unsigned char* dk = smem + Lay::kK + st * Lay::kTile;
+                unsigned char* dv = smem + Lay::kV + st * Lay::kTile;
+                const bool seq = i < n_seq;
+                const int row0 = seq ? i * BN : t0 * a.L + (i - n_seq) * a.dep_rows;
+                const uint32_t bytes = Lay::kSlabs * 128u * (seq ? BN : a.dep_rows);
+                const void* mk = seq ? static_cast<const void*>(&a.tk) : static_cast<const void*>(&a.tkd);
+                const void* mv = seq ? static_cast<const void*>(&a.tv) : static_cast<const void*>(&a.tvd);
+                mbar_arrive_expect_tx(&bars[kB_KFull + st], bytes);
+                for (int s = 0; s < Lay::kSlabs; ++s)
+                    tma_load_3d(dk + s * kSlabBytes, mk, &bars[kB_KFull + st], s * 64, row0, bh);
+                mbar_arrive_expect_tx(&bars[kB_VFull + st], bytes);
+                for (int s = 0; s < Lay::kSlabs; ++s)
+                    tma_load_3d(dv + s * kSlabBytes, mv, &bars[kB_VFull + st], s * 64, row0, bh);
+                issued = i + 1;
+            }
+            mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag);
+            for (int i = max(0, issued - 2); i < issued; ++i) {
+                mbar_wait(&bars[kB_KFull + (i & 1)], (i >> 1) & 1, a.status, abort_flag);
+                mbar_wait(&bars[kB_VFull + (i & 1)], (i >> 1) & 1, a.status, abort_flag);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_seq = idesc_bf16(128, BN, false, false);
+            const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
+            const uint32_t id_dq = idesc_bf16(128, D, false, true);
+            const uint32_t id_dd = idesc_bf16(128, a.dep_rows, true, true);
+            const uint32_t q_addr = smem_u32(smem + Lay::kQ);
+            const uint32_t do_addr = smem_u32(smem + Lay::kDO);
+            const uint32_t ds_addr = smem_u32(smem + Lay::kDS);
+            const uint32_t p_addr = smem_u32(smem + Lay::kP);
+            bool ok = mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag);
+            for (int i = 0; ok && i < nb; ++i) {
+                const int st = i & 1;
+                const bool seq = i < n_seq;
+                const uint32_t id = seq ? id_seq : id_dep;
+                const int n = seq ? BN : a.dep_rows;
+                const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kTile);
+                const uint32_t v_addr = smem_u32(smem + Lay::kV + st * Lay::kTile);
+                if (!mbar_wait(&bars[kB_KFull + st], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    umma_ss(tmem + kColS, desc_kmajor_sw128(q_addr + off), desc_kmajor_sw128(k_addr + off),
+                            id, kk > 0 ? 1u : 0u);
+                }
+                if (!mbar_wait(&bars[kB_VFull + st], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    umma_ss(tmem + kColDP, desc_kmajor_sw128(do_addr + off), desc_kmajor_sw128(v_addr + off),
+                            id, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[kB_SFull]);
+                if (!mbar_wait(&bars[kB_PReady], i & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int kk = 0; kk < n / 16; ++kk)
+                    umma_ts(tmem + kColDQ, tmem + kColS + kk * 8,
+                            desc_mnmajor_sw128(k_addr + kk * 2048, kSlabBytes), id_dq,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+                if (!seq) {
+#pragma unroll
+                    for (int kk = 0; kk < BM / 16; ++kk) {
+                        umma_ss(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
+                                desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                        umma_ss(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
+                                desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&bars[kB_DDFull]);
+                }
+                umma_commit(&bars[kB_KVEmpty + st]);
+            }
+            umma_commit(&bars[kB_Final]);
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const bool row_real = r < R;
+        const int g = row_real ? r / a.Tq : 0;
+        const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
+        const bool row_live = row_real && t_row < a.T;
+        const size_t qrow = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T + t_row;
+        const float lse2 = row_live ? a.LSE[qrow] * kLog2e : INFINITY;
+        const float Dr = row_live ? a.Drow[qrow] : 0.0f;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const float sl2 = a.scale_log2;
+        unsigned char* sDS = smem + Lay::kDS;
+        unsigned char* sP = smem + Lay::kP;
+        const size_t dep_base = static_cast<size_t>(bh) * a.T * a.L;   // first depth row of (b, hk)
+
+        // Depth epilogue: TMEM lane = d index, columns = depth rows of block jd.
+        auto depth_epilogue = [&](int jd) {
+            uint32_t xk[64], xv[64];
+            tmem_ld32(lane_base + kColDKd, xk);
+            tmem_ld32(lane_base + kColDKd + 32, xk + 32);
+            tmem_ld32(lane_base + kColDVd, xv);
+            tmem_ld32(lane_base + kColDVd + 32, xv + 32);
+            tmem_wait_ld();
+            const int dd = r;                      // d index of this lane
+            const int row0 = jd * a.dep_rows;      // relative to t0*L
+            const int nvalid = min(a.dep_rows, dep_total - row0);
+            if (dd < D) {
+                __nv_bfloat16* pk = a.dKd + (dep_base + static_cast<size_t>(t0) * a.L + row0) * D + dd;
+                __nv_bfloat16* pv = a.dVd + (dep_base + static_cast<size_t>(t0) * a.L + row0) * D + dd;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    if (c < nvalid) {
+                        pk[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
+                        pv[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xv[c]));
+                    }
+                }
+            }
+        };
+
+        bool ok = true;
+        int jd = 0;
+        for (int i = 0; i < nb; ++i) {
+            const bool seq = i < n_seq;
+            if (!seq && jd >= 1) {
+                if (!mbar_wait(&bars[kB_DDFull], (jd - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                depth_epilogue(jd - 1);
+            }
+            if (!mbar_wait(&bars[kB_SFull], i & 1, a.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const int nchunk = seq ? 4 : 2;
+            int lo = 0, hi = BN, kb = 0;
+            if (seq) {
+                kb = i * BN;
+            } else {
+                lo = t_row * a.L - (t0 * a.L + jd * a.dep_rows);
+                hi = min(lo + a.L, a.dep_rows);
+            }
+            for (int c4 = 0; c4 < nchunk; ++c4) {
+                uint32_t s[32], dp[32], dsk[16], pk[16];
+                tmem_ld32(lane_base + kColS + 32 * c4, s);
+                tmem_ld32(lane_base + kColDP + 32 * c4, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float p2[2], d2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int c = 32 * c4 + e + u;
+                        const bool vis = seq ? (kb + c <= t_row) : (c >= lo && c < hi);
+                        const float p = vis ? ex2(fmaf(__uint_as_float(s[e + u]), sl2, -lse2)) : 0.0f;
+                        p2[u] = p;
+                        d2[u] = vis ? p * (__uint_as_float(dp[e + u]) - Dr) : 0.0f;
+                    }
+                    dsk[e / 2] = pack_bf16(d2[0], d2[1]);
+                    pk[e / 2] = pack_bf16(p2[0], p2[1]);
+                }
+                tmem_st16(lane_base + kColS + 16 * c4, dsk);
+                if (!seq) {
+                    // row r of the [q][depth] staging tiles, 128-byte swizzle
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int ch = 4 * c4 + e;
+                        const uint32_t off = r * 128 + ((ch ^ (r & 7)) << 4);
+                        *reinterpret_cast<uint4*>(sDS + off) =
+                            make_uint4(dsk[4 * e], dsk[4 * e + 1], dsk[4 * e + 2], dsk[4 * e + 3]);
+                        *reinterpret_cast<uint4*>(sP + off) =
+                            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
+                }
+            }
+            tmem_wait_st();
+            if (!seq) {
+                fence_proxy_async_smem();
+                ++jd;
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[kB_PReady]);
+        }
+        if (ok && n_dep > 0) {
+            if (mbar_wait(&bars[kB_DDFull], (n_dep - 1) & 1, a.status, abort_flag)) {
+                tc_fence_after();
+                depth_epilogue(n_dep - 1);
+            } else {
+                ok = false;
+            }
+        }
+        if (ok) ok = mbar_wait(&bars[kB_Final], 0, a.status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            uint32_t o[D];
+#pragma unroll
+            for (int c = 0; c < D; c += 32) tmem_ld32(lane_base + kColDQ + c, o + c);
+            tmem_wait_ld();
+            if (row_live) {
+                uint4* dst = reinterpret_cast<uint4*>(a.dQ + qrow * D);
+                const float sc = a.scale;
+#pragma unroll
+                for (int c = 0; c < D; c += 8) {
+                    uint4 v;
+                    v.x = pack_bf16(__uint_as_float(o[c]) * sc, __uint_as_float(o[c + 1]) * sc);
+                    v.y = pack_bf16(__uint_as_float(o[c + 2]) * sc, __uint_as_float(o[c + 3]) * sc);
+                    v.z = pack_bf16(__uint_as_float(o[c + 4]) * sc, __uint_as_float(o[c + 5]) * sc);
+                    v.w = pack_bf16(__uint_as_float(o[c + 6]) * sc, __uint_as_float(o[c + 7]) * sc);
+                    dst[c / 8] = v;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int D>
+cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void* V,
+                     const void* Kd, const void* Vd, const void* O, const float* LSE,
+                     const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
+                     float* Dws, cudaStream_t stream) {
+    cudaError_t e;
+    // 1. D = rowsum(dO * O)
+    const long long nrows = (long long)p.B * p.Hq * p.T;
+    constexpr int kRowsPerBlock = 8 * (32 / (D / 8));
+    rowdot_kernel<D><<<(unsigned)((nrows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(
+        nrows, static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), Dws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    // 2. dK, dV
+    DkdvArgs A;
+    A.B = p.B; A.Hq = p.Hq; A.Hk = p.Hk; A.T = p.T; A.G = p.G;
+    A.n_kt = (p.T + BN - 1) / BN;
+    A.n_qb = (p.T + BM - 1) / BM;
+    A.scale = p.scale; A.scale_log2 = p.scale_log2;
+    A.LSE = LSE; A.Drow = Dws;
+    A.dK = static_cast<__nv_bfloat16*>(dK);
+    A.dV = static_cast<__nv_bfloat16*>(dV);
+    A.status = device_status_word();
+    if ((e = make_tma_3d_bf16(&A.tk, K, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&A.tv, V, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&A.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, BM, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&A.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, BM, 1)) != cudaSuccess) return e;
+    {
+        const uint32_t smem = DkdvLayout<D>::kDynSmem;
+        if ((e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        const long long grid = (long long)p.B * p.Hk * A.n_kt;
+        dkdv_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(A);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+
+    // 3. dQ, dKd, dVd
+    DqArgs B;
+    B.B = p.B; B.Hq = p.Hq; B.Hk = p.Hk; B.T = p.T; B.L = p.L; B.G = p.G;
+    B.Tq = BM / p.G;
+    B.n_qt = (p.T + B.Tq - 1) / B.Tq;
+    const int dep = B.Tq * p.L;
+    B.dep_rows = dep >= 64 ? 64 : ((dep + 15) / 16) * 16;
+    if (B.dep_rows < 16) B.dep_rows = 16;
+    B.scale = p.scale; B.scale_log2 = p.scale_log2;
+    B.LSE = LSE; B.Drow = Dws;
+    B.dQ = static_cast<__nv_bfloat16*>(dQ);
+    B.dKd = static_cast<__nv_bfloat16*>(dKd);
+    B.dVd = static_cast<__nv_bfloat16*>(dVd);
+    B.status = device_status_word();
+    if ((e = make_tma_3d_bf16(&B.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&B.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
+    B.tk = A.tk;
+    B.tv = A.tv;
+    if (p.L > 0) {
+        const uint64_t rows = (uint64_t)p.T * p.L;
+        if ((e = make_tma_3d_bf16(&B.tkd, Kd, D, rows, (uint64_t)p.B * p.Hk, B.dep_rows, 1)) != cudaSuccess) return e;
+        if ((e = make_tma_3d_bf16(&B.tvd, Vd, D, rows, (uint64_t)p.B * p.Hk, B.dep_rows, 1)) != cudaSuccess) return e;
+    } else {
+        B.tkd = A.tk;
+        B.tvd = A.tv;
+    }
+    {
+        const uint32_t smem = DqLayout<D>::kDynSmem;
+        if ((e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        const long long grid = (long long)p.B * p.Hk * B.n_qt;
+        dq_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(B);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
 
 cudaError_t launch_bwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, const void* O, const float* LSE,
                              const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
                              float* Dws, cudaStream_t stream) {
-    return launch_bwd_simt(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, stream);
+    if (p.d == 128)
+        return launch_d<128>(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, stream);
+    if (p.d == 64)
+        return launch_d<64>(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace moda
