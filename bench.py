@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoDA operator on B200: fwd+bwd TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic input
+already resident in HBM: depth repack of K_depth and V_depth (layer-major to
+token-major), forward, backward.  The workload is the 1.5B-scale attention
+layer at T = 4096 (B=2, Hq=16, Hk=4, d=128, L=16).  FLOPs are algorithmic:
+forward 4*B*Hq*d*(T(T+1)/2 + T*L), backward 2.5x that.
+
+Printed (rank 0, one JSON line): the whole-job value, the same workload at
+L = 0 (the FlashAttention-style reference point), the forward at T = 65536
+(L = 32 and L = 0), an end-to-end figure through host buffers, the roofline of
+the dominant launch, the oracle timed on the host as a CPU baseline, and the
+SM clocks sampled during the timed region.
+
+Under torchrun (N > 1) every rank runs its own batch (data parallel, weak
+scaling, no collective in the operator); times are the max over ranks.
+`--impl reference` times the CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+sys.path.insert(0, os.path.join(ROOT, "tests"))
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from sequence_depth_attention_moda_b200 import inputs as I  # noqa: E402
+
+WORKLOAD = I.LAYER_1P5B
+LONG = I.LONG_64K
+BWD_FACTOR = 2.5
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the L=0 twin and T=64K lines")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers --
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.05)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def traffic_from_profile(kernel_src: str):
+    """Per-launch DRAM bytes of the dominant launch from the committed ncu
+    summary, or None when the kernel source has changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "moda_bwd_layer_T4k_traffic.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"source sha256: ([0-9a-f]{16})", text)
+    m_bytes = re.search(r"bytes per call: (\d+)", text)
+    if not m_hash or not m_bytes:
+        return None
+    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    return int(m_bytes.group(1)) if cur == m_hash.group(1) else None
+
+
+# --------------------------------------------------------------- our arm ----
+class Runner:
+    """Device buffers and the four C-ABI calls of one step."""
+
+    def __init__(self, w: I.Workload, x, backward=True):
+        import sequence_depth_attention_moda_b200 as moda
+        self.moda = moda
+        self.w = w
+        self.x = x
+        self.backward = backward
+        dev = x["Q"].device
+        self.sh = moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C)
+        bf = torch.bfloat16
+        self.Kd = torch.empty(w.B, w.Hk, w.T * w.L, w.d, device=dev, dtype=bf) if w.L else None
+        self.Vd = torch.empty_like(self.Kd) if w.L else None
+        self.O = torch.empty_like(x["Q"])
+        self.LSE = torch.empty(w.B, w.Hq, w.T, device=dev, dtype=torch.float32)
+        if backward:
+            self.nws = moda.moda_workspace_size(self.sh, True)
+            self.ws = torch.empty(max(self.nws, 16), device=dev, dtype=torch.uint8)
+            self.dQ = torch.empty_like(x["Q"])
+            self.dK = torch.empty_like(x["K"])
+            self.dV = torch.empty_like(x["V"])
+            self.dKd = torch.empty_like(self.Kd) if w.L else None
+            self.dVd = torch.empty_like(self.Vd) if w.L else None
+
+    def launches_per_step(self):
+        return (2 if self.w.L else 0) + 1 + (3 if self.backward else 0)
+
+    def step(self, ev=None):
+        m, x = self.moda, self.x
+        if ev is not None:
+            ev[0].record()
+        if self.w.L:
+            m.moda_repack_depth(self.sh, x["Kd_layer"], self.Kd)
+            m.moda_repack_depth(self.sh, x["Vd_layer"], self.Vd)
+        if ev is not None:
+            ev[1].record()
+        m.moda_fwd(self.sh, x["Q"], x["K"], x["V"], self.Kd, self.Vd, self.O, self.LSE)
+        if ev is not None:
+            ev[2].record()
+        if self.backward:
+            m.moda_bwd(self.sh, x["Q"], x["K"], x["V"], self.Kd, self.Vd, self.O, self.LSE, x["dO"],
+                       self.dQ, self.dK, self.dV, self.dKd, self.dVd, self.ws, self.nws)
+        if ev is not None:
+            ev[3].record()
+
+    def outputs(self):
+        outs = [self.O, self.LSE]
+        if self.backward:
+            outs += [self.dQ, self.dK, self.dV] + ([self.dKd, self.dVd] if self.w.L else [])
+        return outs
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(r: Runner, steps: int, warmup: int, world: int, per_call=False, clocks=None):
+    """Warm up, then time exactly `steps` steps between barriers + syncs.
+    Returns (ms per step, per-call mean ms or None)."""
+    for _ in range(warmup):
+        r.step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)] if per_call else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ctx = clocks if clocks is not None else _Null()
+    with ctx:
+        start.record()
+        for i in range(steps):
+            r.step(evs[i] if per_call else None)
+        end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(end) / steps
+    calls = None
+    if per_call:
+        calls = {"repack": np.mean([e[0].elapsed_time(e[1]) for e in evs]),
+                 "fwd": np.mean([e[1].elapsed_time(e[2]) for e in evs]),
+                 "bwd": np.mean([e[2].elapsed_time(e[3]) for e in evs])}
+    return max_over_ranks(ms, world), calls
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def e2e_measure(w: I.Workload, x, steps: int, world: int):
+    """Same step through the C ABI with host buffers: pinned host -> device
+    copies of every input and device -> host copies of every output inside
+    the timed region."""
+    host_in = {k: v.cpu().pin_memory() for k, v in x.items()}
+    r = Runner(w, x)
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in r.outputs()]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def one():
+        for k, v in host_in.items():
+            x[k].copy_(v, non_blocking=True)
+        r.step()
+        for dst, src in zip(host_out, r.outputs()):
+            dst.copy_(src, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        one()
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world)
+    return ms, h2d, d2h
+
+
+def cpu_baseline_sample(w: I.Workload, x):
+    """The oracle, as it stands, on one (b, hk) slice of the workload
+    (forward + backward of G heads over all T tokens and L depth rows)."""
+    import oracle
+    from moda_cases import slice_workload, token_major, f64
+    ws, xs = slice_workload(w, x, 0, 0)
+    Kd, Vd = token_major(xs, ws)
+    args = [f64(xs["Q"]), f64(xs["K"]), f64(xs["V"]), f64(Kd), f64(Vd)]
+    dO = f64(xs["dO"])
+    lib = oracle.load_library()
+    t0 = time.perf_counter()
+    oracle.fwd(*args, lib=lib)
+    oracle.bwd(*args, dO, lib=lib)
+    dt = time.perf_counter() - t0
+    flops = ws.fwd_flops() * (1 + BWD_FACTOR)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(lib),
+            "kind": "oracle",
+            "sample": f"one (b,hk) slice of the workload: B=1, Hq=G={ws.Hq}, Hk=1, T={ws.T}, "
+                      f"L={ws.L}, d={ws.d}, fwd+bwd in fp64 ({1.0 / (w.B * w.Hk):.4f} of a step), "
+                      f"{dt:.1f} s"}
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    import sequence_depth_attention_moda_b200 as moda
+    moda.load()
+    peaks = load_peaks()
+    w = WORKLOAD
+    x = I.make_inputs(w, device="cuda", seed=w.seed + 1000 * rank)
+    r = Runner(w, x)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    ms, calls = time_steps(r, args.steps, args.warmup, world, per_call=True, clocks=clocks)
+    moda.moda_check_status()
+    flops_step = w.fwd_flops() * (1 + BWD_FACTOR)
+    value = world * flops_step / (ms * 1e-3) / 1e12
+    per_gpu = value / world
+
+    # roofline of the dominant launch group: the backward call (rowdot + dkdv + dq)
+    bwd_flops = w.fwd_flops() * BWD_FACTOR
+    kernel_src = os.path.join(ROOT, "sequence_depth_attention_moda_b200", "csrc", "moda_bwd_sm100.cu")
+    achieved = bwd_flops / (calls["bwd"] * 1e-3) / 1e12
+    roofline = {"kernel": "moda_bwd (rowdot + dkdv + dq launches of one call)", "bound": "tensor",
+                "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                "traffic": traffic_from_profile(kernel_src),
+                "per_call_ms": {k: round(v, 4) for k, v in calls.items()}}
+    fwd_ach = w.fwd_flops() / (calls["fwd"] * 1e-3) / 1e12
+    roofline_fwd = {"kernel": "moda_fwd_sm100_kernel", "bound": "tensor", "achieved": round(fwd_ach, 1),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": round(fwd_ach / peaks["bf16_tflops"], 4)}
+    rep_bytes = 2 * 2 * w.B * w.Hk * w.T * w.L * w.d * 2
+    rep_ach = rep_bytes / (calls["repack"] * 1e-3) / 1e9
+    roofline_repack = {"kernel": "repack_vec16_kernel (x2)", "bound": "hbm", "achieved": round(rep_ach, 1),
+                       "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(rep_ach / peaks["hbm_gbs"], 4)}
+
+    extra = {}
+    if not args.no_extra:
+        w0 = w.with_(L=0)
+        x0 = dict(x)
+        r0 = Runner(w0, x0)
+        ms0, _ = time_steps(r0, args.steps, args.warmup, world)
+        v0 = world * w0.fwd_flops() * (1 + BWD_FACTOR) / (ms0 * 1e-3) / 1e12
+        extra["l0_twin"] = {"value": round(v0, 2), "ms_per_step": round(ms0, 4),
+                            "ratio": round(value / v0, 4)}
+        del r0
+        xl = I.make_inputs(LONG, device="cuda", seed=LONG.seed + 1000 * rank, grad_out=False)
+        long_res = {}
+        for L in (LONG.L, 0):
+            wl = LONG.with_(L=L)
+            rl = Runner(wl, xl, backward=False)
+            msl, callsl = time_steps(rl, max(3, args.steps // 4), 2, world, per_call=True)
+            tf = wl.fwd_flops() / (callsl["fwd"] * 1e-3) / 1e12
+            long_res[f"L{L}"] = {"fwd_tflops": round(tf, 1),
+                                 "fwd_frac_of_peak": round(tf / peaks["bf16_tflops"], 4),
+                                 "fwd_ms": round(callsl["fwd"], 3)}
+            del rl
+        long_res["fwd_vs_L0"] = round(long_res[f"L{LONG.L}"]["fwd_tflops"] / long_res["L0"]["fwd_tflops"], 4)
+        extra["long_context_T64k_fwd"] = long_res
+        del xl
+        torch.cuda.empty_cache()
+
+    e2e = None
+    if not args.no_e2e:
+        ms_e, h2d, d2h = e2e_measure(w, x, max(2, min(args.steps, 5)), world)
+        e2e = {"value": round(world * flops_step / (ms_e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e, 3)}
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu:
+        cpu = cpu_baseline_sample(w, x)
+
+    if rank == 0:
+        line = {
+            "metric": "MoDA fwd+bwd TFLOP/s (depth repack + forward + backward per step)",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "pct_of_peak_per_gpu": round(100 * per_gpu / peaks["bf16_tflops"], 2),
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hk": w.Hk, "d": w.d, "T": w.T,
+                       "L": w.L, "C": w.C, "global_batch": w.B * world, "seq_len": w.T,
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (%.0f MB read per step)" %
+                             (sum(t.numel() * t.element_size() for t in x.values()) / 1e6)},
+            "roofline": roofline, "roofline_fwd": roofline_fwd, "roofline_repack": roofline_repack,
+            "gpu_launches": r.launches_per_step() * args.steps,
+            "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu, **extra,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# --------------------------------------------------------- reference arm ----
+def run_reference(args):
+    """The CPU oracle as the reference arm: bounded sample of the workload
+    per step (one (b, hk) slice), on the host cores, rank 0 only."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from moda_cases import slice_workload, token_major, f64
+    w = WORKLOAD
+    x = I.make_inputs(w, device="cpu")
+    ws, xs = slice_workload(w, x, 0, 0)
+    Kd, Vd = token_major(xs, ws)
+    a = [f64(xs["Q"]), f64(xs["K"]), f64(xs["V"]), f64(Kd), f64(Vd)]
+    dO = f64(xs["dO"])
+    lib = oracle.load_library()
+
+    def step():
+        oracle.fwd(*a, lib=lib)
+        oracle.bwd(*a, dO, lib=lib)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = ws.fwd_flops() * (1 + BWD_FACTOR)
+    value = flops / dt / 1e12
+    sample = (f"one (b,hk) slice per step: B=1, Hq=G={ws.Hq}, Hk=1, T={ws.T}, L={ws.L}, "
+              f"d={ws.d}, fwd+bwd in fp64")
+    line = {"impl": "reference", "metric": "MoDA fwd+bwd TFLOP/s (depth repack + forward + backward per step)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hk": w.Hk, "d": w.d, "T": w.T,
+                       "L": w.L, "C": w.C, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.threads(lib),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
