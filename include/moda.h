@@ -148,6 +148,32 @@ moda_status moda_bwd(const moda_shape* shape,
                      void* ws, size_t ws_bytes, moda_stream_t stream);
 
 /*
+ * moda_bwd_noalloc: moda_bwd without a workspace argument.  The pages have no
+ * counterpart; it exists for callers that cannot allocate device memory where
+ * they run the backward -- for example a plugin whose host framework owns all
+ * device memory and forbids allocation while it executes, or code replaying a
+ * fixed memory plan -- and so cannot hand moda_bwd its workspace.
+ *
+ * Same arguments, layouts, results and errors as moda_bwd, minus ws/ws_bytes;
+ * it allocates nothing and calls no allocating routine.  Its scratch (one fp32
+ * per query row) is a fixed 16 MiB array inside the library, so it accepts at
+ * most B*Hq*T = 4,194,304 query rows; larger problems get MODA_ERR_WORKSPACE.
+ * Every device that loads the library holds that array until the process
+ * exits.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array, and each call
+ * writes every row it reads before reading it, so nothing needs clearing
+ * between calls -- but calls that overlap on the GPU (concurrent streams,
+ * threads) race on it: serialise them.
+ */
+moda_status moda_bwd_noalloc(const moda_shape* shape,
+                             const void* Q, const void* K, const void* V,
+                             const void* Kd, const void* Vd,
+                             const void* O, const float* LSE, const void* dO,
+                             void* dQ, void* dK, void* dV, void* dKd, void* dVd,
+                             moda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's kernel
  * status word.  MODA_ERR_TIMEOUT if a kernel's bounded wait ran out since the
  * last check, MODA_ERR_CUDA if the stream reports an error, else MODA_OK.

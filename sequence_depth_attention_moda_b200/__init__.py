@@ -5,11 +5,11 @@ the C ABI of ``include/moda.h``); ``_binding`` marshals torch tensors into it
 and ``ops`` offers tensor-allocating conveniences over the same entry points.
 """
 from ._binding import (EXPORTED, LIB_PATH, MODA_BF16, MODA_DEPTH_CHUNKED, MODA_DEPTH_FLAT,
-                       MODA_FP32, MoDAError, load, make_shape, moda_bwd, moda_check_status,
-                       moda_fwd, moda_last_error_message, moda_repack_depth, moda_shape,
+                       MODA_FP32, MoDAError, load, make_shape, moda_bwd, moda_bwd_noalloc,
+                       moda_check_status, moda_fwd, moda_last_error_message, moda_repack_depth, moda_shape,
                        moda_status_string, moda_version, moda_workspace_size)
 
 __all__ = ["EXPORTED", "LIB_PATH", "MODA_BF16", "MODA_DEPTH_CHUNKED", "MODA_DEPTH_FLAT",
-           "MODA_FP32", "MoDAError", "load", "make_shape", "moda_bwd", "moda_check_status",
+           "MODA_FP32", "MoDAError", "load", "make_shape", "moda_bwd", "moda_bwd_noalloc", "moda_check_status",
            "moda_fwd", "moda_last_error_message", "moda_repack_depth", "moda_shape",
            "moda_status_string", "moda_version", "moda_workspace_size"]

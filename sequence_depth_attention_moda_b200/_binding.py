@@ -30,7 +30,7 @@ MODA_DEPTH_CHUNKED = 1
 
 # Every symbol include/moda.h declares.
 EXPORTED = ("moda_workspace_size", "moda_repack_depth", "moda_fwd", "moda_bwd",
-            "moda_check_status", "moda_status_string", "moda_last_error_message", "moda_version")
+            "moda_bwd_noalloc", "moda_check_status", "moda_status_string", "moda_last_error_message", "moda_version")
 
 
 class moda_shape(ctypes.Structure):
@@ -73,6 +73,8 @@ def load(path: Optional[str] = None):
         lib.moda_fwd.restype = i
         lib.moda_bwd.argtypes = [sp] + [vp] * 13 + [vp, sz, vp]
         lib.moda_bwd.restype = i
+        lib.moda_bwd_noalloc.argtypes = [sp] + [vp] * 13 + [vp]
+        lib.moda_bwd_noalloc.restype = i
         lib.moda_check_status.argtypes = [vp]
         lib.moda_check_status.restype = i
         lib.moda_status_string.argtypes = [i]
@@ -144,6 +146,17 @@ def moda_bwd(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dV
     _check(load().moda_bwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd),
                            _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dKd),
                            _ptr(dVd), _ptr(ws), int(ws_bytes), _stream(stream)), "moda_bwd")
+
+
+def moda_bwd_noalloc(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd,
+                     stream=None):
+    """moda_bwd for callers that cannot allocate: no workspace argument; the
+    library's built-in scratch holds at most B*Hq*T = 4,194,304 query rows,
+    and overlapping calls on the GPU share (and race on) that scratch."""
+    _check(load().moda_bwd_noalloc(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd),
+                                   _ptr(Vd), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK),
+                                   _ptr(dV), _ptr(dKd), _ptr(dVd), _stream(stream)),
+           "moda_bwd_noalloc")
 
 
 def moda_check_status(stream=None):

@@ -124,6 +124,10 @@ int device_sm_count() {
     return g_sm_count[dev];
 }
 
+// Hooks for entry points that live in other files of the library.
+moda_status api_validate(const moda_shape* shape, Problem* p) { return validate(shape, p); }
+moda_status api_fail(moda_status s, const char* msg) { return fail(s, "%s", msg); }
+
 }  // namespace moda
 
 using namespace moda;
