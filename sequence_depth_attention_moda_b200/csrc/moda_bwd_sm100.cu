@@ -78,6 +78,9 @@ __global__ void __launch_bounds__(256) rowdot_kernel(long long nrows,
 }
 
 // -------------------------------------------------------------- 2. dkdv ----
+// Query blocks are 64 rows, so S^T and dP^T are double-buffered in TMEM:
+//   S^T0 [0,64) S^T1 [64,128) | dP^T0 [128,192) dP^T1 [192,256) |
+//   dV [256, 256+D) | dK [384, 384+D)
 struct DkdvArgs {
     TmaMap tk, tv, tq, tdo;
     const float* LSE;
@@ -85,26 +88,31 @@ struct DkdvArgs {
     __nv_bfloat16* dK;
     __nv_bfloat16* dV;
     unsigned int* status;
-    int B, Hq, Hk, T, G, n_kt, n_qb;
+    int B, Hq, Hk, T, G, n_kt, n_qb;     // n_qb counts 64-row query blocks
     float scale, scale_log2;
 };
+
+constexpr int kKvBQ = 64;               // query rows per iteration
+constexpr int kKvStages = 4;            // Q/dO ring depth
+constexpr uint32_t kKvSlab = 64 * 128;
 
 template <int D>
 struct DkdvLayout {
     static constexpr int kSlabs = D / 64;
-    static constexpr uint32_t kTile = kSlabs * kSlabBytes;
+    static constexpr uint32_t kKTile = kSlabs * kSlabBytes;     // 128 key rows
+    static constexpr uint32_t kQTile = kSlabs * kKvSlab;        // 64 query rows
     static constexpr uint32_t kK = 0;
-    static constexpr uint32_t kV = kTile;
-    static constexpr uint32_t kQ = 2 * kTile;            // 2 stages
-    static constexpr uint32_t kDO = 4 * kTile;           // 2 stages
-    static constexpr uint32_t kStat = 6 * kTile;         // 2 x (lse2[128], D[128]) floats
-    static constexpr uint32_t kBar = kStat + 2048;
+    static constexpr uint32_t kV = kKTile;
+    static constexpr uint32_t kQ = 2 * kKTile;                  // kKvStages stages
+    static constexpr uint32_t kDO = kQ + kKvStages * kQTile;    // kKvStages stages
+    static constexpr uint32_t kStat = kDO + kKvStages * kQTile; // 2 x (lse2[64], D[64]) floats
+    static constexpr uint32_t kBar = kStat + 1024;
     static constexpr uint32_t kBytes = kBar + 256;
     static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
 };
 
-enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 3, kA_SFull = 5, kA_PReady = 6, kA_Final = 7,
-       kA_NumBars = 8 };
+enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 1 + kKvStages, kA_SFull = 1 + 2 * kKvStages,
+       kA_PReady = 3 + 2 * kKvStages, kA_Final = 5 + 2 * kKvStages, kA_NumBars = 6 + 2 * kKvStages };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant__ DkdvArgs a) {
@@ -124,17 +132,20 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     const int bh = static_cast<int>(blockIdx.x) % nbh;
     const int b = bh / a.Hk;
     const int hk = bh - b * a.Hk;
-    const int nqb = a.n_qb - kt;                            // query blocks qb = kt .. n_qb-1
+    const int qb0 = kt * (BN / kKvBQ);                      // first query block that sees the keys
+    const int nqb = a.n_qb - qb0;
     const int n_it = a.G * nqb;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kA_KVFull], 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kKvStages; ++s) {
             mbar_init(&bars[kA_QFull + s], 1);
             mbar_init(&bars[kA_QEmpty + s], 1);
         }
-        mbar_init(&bars[kA_SFull], 1);
-        mbar_init(&bars[kA_PReady], kMathThreads);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kA_SFull + s], 1);
+            mbar_init(&bars[kA_PReady + s], kMathThreads);
+        }
         mbar_init(&bars[kA_Final], 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -151,67 +162,80 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     if (warp == 0) {
         if (lane == 0) {
             prefetch_tmap(&a.tk); prefetch_tmap(&a.tv); prefetch_tmap(&a.tq); prefetch_tmap(&a.tdo);
-            mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * Lay::kTile);
+            mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * Lay::kKTile);
             for (int s = 0; s < Lay::kSlabs; ++s) {
                 tma_load_3d(smem + Lay::kK + s * kSlabBytes, &a.tk, &bars[kA_KVFull], s * 64, kt * BN, bh);
                 tma_load_3d(smem + Lay::kV + s * kSlabBytes, &a.tv, &bars[kA_KVFull], s * 64, kt * BN, bh);
             }
             int issued = 0;
             for (int it = 0; it < n_it; ++it) {
-                const int st = it & 1;
-                if (it >= 2 && !mbar_wait(&bars[kA_QEmpty + st], ((it >> 1) - 1) & 1, a.status, abort_flag))
+                const int st = it % kKvStages;
+                if (it >= kKvStages &&
+                    !mbar_wait(&bars[kA_QEmpty + st], ((it / kKvStages) - 1) & 1, a.status, abort_flag))
                     break;
                 const int g = it / nqb;
-                const int qb = kt + (it - g * nqb);
+                const int qb = qb0 + (it - g * nqb);
                 const int qh = b * a.Hq + hk * a.G + g;
-                mbar_arrive_expect_tx(&bars[kA_QFull + st], 2 * Lay::kTile);
+                mbar_arrive_expect_tx(&bars[kA_QFull + st], 2 * Lay::kQTile);
                 for (int s = 0; s < Lay::kSlabs; ++s) {
-                    tma_load_3d(smem + Lay::kQ + st * Lay::kTile + s * kSlabBytes, &a.tq,
-                                &bars[kA_QFull + st], s * 64, qb * BM, qh);
-                    tma_load_3d(smem + Lay::kDO + st * Lay::kTile + s * kSlabBytes, &a.tdo,
-                                &bars[kA_QFull + st], s * 64, qb * BM, qh);
+                    tma_load_3d(smem + Lay::kQ + st * Lay::kQTile + s * kKvSlab, &a.tq,
+                                &bars[kA_QFull + st], s * 64, qb * kKvBQ, qh);
+                    tma_load_3d(smem + Lay::kDO + st * Lay::kQTile + s * kKvSlab, &a.tdo,
+                                &bars[kA_QFull + st], s * 64, qb * kKvBQ, qh);
                 }
                 issued = it + 1;
             }
             mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
-            for (int it = max(0, issued - 2); it < issued; ++it)
-                mbar_wait(&bars[kA_QFull + (it & 1)], (it >> 1) & 1, a.status, abort_flag);
+            for (int it = max(0, issued - kKvStages); it < issued; ++it)
+                mbar_wait(&bars[kA_QFull + it % kKvStages], (it / kKvStages) & 1, a.status, abort_flag);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(128, BM, false, false);
+            const uint32_t id_s = idesc_bf16(128, kKvBQ, false, false);
             const uint32_t id_g = idesc_bf16(128, D, false, true);
             const uint32_t k_addr = smem_u32(smem + Lay::kK);
             const uint32_t v_addr = smem_u32(smem + Lay::kV);
-            bool ok = mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
+            // S^T(j) = K Q_j^T and dP^T(j) = V dO_j^T into buffer j & 1.
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % kKvStages;
+                const int buf = j & 1;
+                if (!mbar_wait(&bars[kA_QFull + st], (j / kKvStages) & 1, a.status, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kQTile);
+                const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kQTile);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t offk = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    const uint32_t offq = (kk >> 2) * kKvSlab + (kk & 3) * 32;
+                    umma_ss(tmem + buf * 64, desc_kmajor_sw128(k_addr + offk),
+                            desc_kmajor_sw128(q_addr + offq), id_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t offk = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    const uint32_t offq = (kk >> 2) * kKvSlab + (kk & 3) * 32;
+                    umma_ss(tmem + 128 + buf * 64, desc_kmajor_sw128(v_addr + offk),
+                            desc_kmajor_sw128(do_addr + offq), id_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[kA_SFull + buf]);
+                return true;
+            };
+            bool ok = mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag) && (n_it == 0 || issue_s(0));
             for (int it = 0; ok && it < n_it; ++it) {
-                const int st = it & 1;
-                if (!mbar_wait(&bars[kA_QFull + st], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
+                const int st = it % kKvStages;
+                const int buf = it & 1;
+                if (!mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kTile);
-                const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kTile);
+                const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kQTile);
+                const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kQTile);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    umma_ss(tmem + 0, desc_kmajor_sw128(k_addr + off), desc_kmajor_sw128(q_addr + off),
-                            id_s, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    umma_ss(tmem + 128, desc_kmajor_sw128(v_addr + off), desc_kmajor_sw128(do_addr + off),
-                            id_s, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&bars[kA_SFull]);
-                if (!mbar_wait(&bars[kA_PReady], it & 1, a.status, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < BM / 16; ++kk) {
+                for (int kk = 0; kk < kKvBQ / 16; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts(tmem + 256, tmem + 0 + kk * 8,
-                            desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes), id_g, acc);
-                    umma_ts(tmem + 384, tmem + 128 + kk * 8,
-                            desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes), id_g, acc);
+                    umma_ts(tmem + 256, tmem + buf * 64 + kk * 8,
+                            desc_mnmajor_sw128(do_addr + kk * 2048, kKvSlab), id_g, acc);
+                    umma_ts(tmem + 384, tmem + 128 + buf * 64 + kk * 8,
+                            desc_mnmajor_sw128(q_addr + kk * 2048, kKvSlab), id_g, acc);
                 }
                 umma_commit(&bars[kA_QEmpty + st]);
             }
@@ -227,44 +251,45 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int g = it / nqb;
-            const int qb = kt + (it - g * nqb);
+            const int qb = qb0 + (it - g * nqb);
+            const int buf = it & 1;
             const size_t qrow0 = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T;
-            float* sbuf = stat + (it & 1) * 256;
-            {
-                const int t = qb * BM + mt;
+            float* sbuf = stat + buf * 128;
+            if (mt < kKvBQ) {
+                const int t = qb * kKvBQ + mt;
                 sbuf[mt] = t < a.T ? a.LSE[qrow0 + t] * kLog2e : INFINITY;
-                sbuf[128 + mt] = t < a.T ? a.Drow[qrow0 + t] : 0.0f;
+                sbuf[64 + mt] = t < a.T ? a.Drow[qrow0 + t] : 0.0f;
             }
             named_bar_sync(1, kMathThreads);
-            if (!mbar_wait(&bars[kA_SFull], it & 1, a.status, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const bool diag = qb == kt;
+            const int tq0 = qb * kKvBQ;
+            const bool diag = tq0 < kt * BN + BN;         // some key of the tile is after some query
+            uint32_t s[64], dp[64], pk[32], dk[32];
+            tmem_ld32(lane_base + buf * 64, s);
+            tmem_ld32(lane_base + buf * 64 + 32, s + 32);
+            tmem_ld32(lane_base + 128 + buf * 64, dp);
+            tmem_ld32(lane_base + 128 + buf * 64 + 32, dp + 32);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t s[32], dp[32], pk[16], dk[16];
-                tmem_ld32(lane_base + 32 * c4, s);
-                tmem_ld32(lane_base + 128 + 32 * c4, dp);
-                tmem_wait_ld();
+            for (int e = 0; e < 64; e += 2) {
+                float p2[2], d2[2];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float p2[2], d2[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int c = 32 * c4 + e + u;
-                        const bool vis = !diag || k <= qb * BM + c;
-                        const float p = vis ? ex2(fmaf(__uint_as_float(s[e + u]), sl2, -sbuf[c])) : 0.0f;
-                        p2[u] = p;
-                        d2[u] = vis ? p * (__uint_as_float(dp[e + u]) - sbuf[128 + c]) : 0.0f;
-                    }
-                    pk[e / 2] = pack_bf16(p2[0], p2[1]);
-                    dk[e / 2] = pack_bf16(d2[0], d2[1]);
+                for (int u = 0; u < 2; ++u) {
+                    const int c = e + u;
+                    const bool vis = !diag || k <= tq0 + c;
+                    const float p = vis ? ex2(fmaf(__uint_as_float(s[c]), sl2, -sbuf[c])) : 0.0f;
+                    p2[u] = p;
+                    d2[u] = vis ? p * (__uint_as_float(dp[c]) - sbuf[64 + c]) : 0.0f;
                 }
-                tmem_st16(lane_base + 16 * c4, pk);
-                tmem_st16(lane_base + 128 + 16 * c4, dk);
+                pk[e / 2] = pack_bf16(p2[0], p2[1]);
+                dk[e / 2] = pack_bf16(d2[0], d2[1]);
             }
+            tmem_st32(lane_base + buf * 64, pk);
+            tmem_st32(lane_base + 128 + buf * 64, dk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[kA_PReady]);
+            mbar_arrive(&bars[kA_PReady + buf]);
         }
         if (ok) ok = mbar_wait(&bars[kA_Final], 0, a.status, abort_flag);
         if (ok) {
@@ -302,6 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------- 3. dq ----
+// Key and depth blocks are 64 rows, so S and dP are double-buffered in TMEM:
+// the MMAs of block i+1 run while the math warps work on block i.
+//   TMEM columns: S0 [0,64) S1 [64,128) | dP0 [128,192) dP1 [192,256) |
+//                 dQ [256, 256+D) | dKd^T [384,448) | dVd^T [448,512)
 struct DqArgs {
     TmaMap tq, tdo, tk, tv, tkd, tvd;
     const float* LSE;
@@ -314,25 +343,31 @@ struct DqArgs {
     float scale, scale_log2;
 };
 
+constexpr int kDqBN = 64;            // rows per key / depth block
+constexpr int kDqStages = 3;         // K/V ring depth
+constexpr uint32_t kDqSlab = 64 * 128;   // 64 rows x 64 bf16
+
 template <int D>
 struct DqLayout {
     static constexpr int kSlabs = D / 64;
-    static constexpr uint32_t kTile = kSlabs * kSlabBytes;
+    static constexpr uint32_t kQTile = kSlabs * kSlabBytes;      // 128 rows
+    static constexpr uint32_t kKTile = kSlabs * kDqSlab;         // 64 rows
     static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kDO = kTile;
-    static constexpr uint32_t kK = 2 * kTile;        // 2 stages
-    static constexpr uint32_t kV = 4 * kTile;        // 2 stages
-    static constexpr uint32_t kDS = 6 * kTile;       // [128 q rows][64 depth] bf16, 128-B swizzle
+    static constexpr uint32_t kDO = kQTile;
+    static constexpr uint32_t kK = 2 * kQTile;                   // kDqStages stages
+    static constexpr uint32_t kV = kK + kDqStages * kKTile;      // kDqStages stages
+    static constexpr uint32_t kDS = kV + kDqStages * kKTile;     // [128 q][64 depth] bf16, 128-B swizzle
     static constexpr uint32_t kP = kDS + kSlabBytes;
-    static constexpr uint32_t kBar = kP + kSlabBytes;
+    static constexpr uint32_t kStage = kP + kSlabBytes;          // [64 rows][D] bf16 x 2 (dKd, dVd)
+    static constexpr uint32_t kBar = kStage + 2 * 64 * D * 2;
     static constexpr uint32_t kBytes = kBar + 256;
     static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
 };
 
-enum { kB_QFull = 0, kB_KFull = 1, kB_VFull = 3, kB_KVEmpty = 5, kB_SFull = 7, kB_PReady = 8,
-       kB_DDFull = 9, kB_Final = 10, kB_NumBars = 11 };
+enum { kB_QFull = 0, kB_KVFull = 1, kB_KVEmpty = 1 + kDqStages, kB_SFull = 1 + 2 * kDqStages,
+       kB_PReady = 3 + 2 * kDqStages, kB_DDFull = 5 + 2 * kDqStages, kB_Final = 6 + 2 * kDqStages,
+       kB_NumBars = 7 + 2 * kDqStages };
 
-// TMEM columns of the dq kernel.
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDKd = 384, kColDVd = 448;
 
 template <int D>
@@ -355,28 +390,29 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const int t0 = qt * a.Tq;
     const int R = a.G * a.Tq;
     const int t_end = min(t0 + a.Tq, a.T);
-    const int n_seq = (t_end - 1) / BN + 1;
+    const int n_seq = (t_end - 1) / kDqBN + 1;
     const int dep_total = a.L > 0 ? (t_end - t0) * a.L : 0;
     const int n_dep = (dep_total + a.dep_rows - 1) / a.dep_rows;
     const int nb = n_seq + n_dep;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kB_QFull], 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[kB_KFull + s], 1);
-            mbar_init(&bars[kB_VFull + s], 1);
+        for (int s = 0; s < kDqStages; ++s) {
+            mbar_init(&bars[kB_KVFull + s], 1);
             mbar_init(&bars[kB_KVEmpty + s], 1);
         }
-        mbar_init(&bars[kB_SFull], 1);
-        mbar_init(&bars[kB_PReady], kMathThreads);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[kB_SFull + s], 1);
+            mbar_init(&bars[kB_PReady + s], kMathThreads);
+        }
         mbar_init(&bars[kB_DDFull], 1);
         mbar_init(&bars[kB_Final], 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
     if (R < BM) {  // rows the Q / dO boxes do not cover: zeros
-        for (int i = threadIdx.x; i < 2 * Lay::kSlabs * (BM - R) * 8; i += kThreads) {
-            const int per = (BM - R) * 8;
+        const int per = (BM - R) * 8;
+        for (int i = threadIdx.x; i < 2 * Lay::kSlabs * per; i += kThreads) {
             const int which = i / (Lay::kSlabs * per);       // 0: Q, 1: dO
             const int rem0 = i - which * Lay::kSlabs * per;
             const int slab = rem0 / per;
@@ -397,6 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const uint32_t tmem = *tmem_holder;
 
     if (warp == 0) {
+        // ------------------------------------------------------ producer ----
         if (lane == 0) {
             prefetch_tmap(&a.tq); prefetch_tmap(&a.tdo); prefetch_tmap(&a.tk); prefetch_tmap(&a.tv);
             if (a.L > 0) { prefetch_tmap(&a.tkd); prefetch_tmap(&a.tvd); }
@@ -408,33 +445,32 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             }
             int issued = 0;
             for (int i = 0; i < nb; ++i) {
-                const int st = i & 1;
-                if (i >= 2 && !mbar_wait(&bars[kB_KVEmpty + st], ((i >> 1) - 1) & 1, a.status, abort_flag))
+                const int st = i % kDqStages;
+                if (i >= kDqStages &&
+                    !mbar_wait(&bars[kB_KVEmpty + st], ((i / kDqStages) - 1) & 1, a.status, abort_flag))
                     break;
-                unsigned char* dk = smem + Lay::kK + st * Lay::kTile;
-                unsigned char* dv = smem + Lay::kV + st * Lay::kTile;
+                unsigned char* dk = smem + Lay::kK + st * Lay::kKTile;
+                unsigned char* dv = smem + Lay::kV + st * Lay::kKTile;
                 const bool seq = i < n_seq;
-                const int row0 = seq ? i * BN : t0 * a.L + (i - n_seq) * a.dep_rows;
-                const uint32_t bytes = Lay::kSlabs * 128u * (seq ? BN : a.dep_rows);
+                const int row0 = seq ? i * kDqBN : t0 * a.L + (i - n_seq) * a.dep_rows;
+                const uint32_t bytes = Lay::kSlabs * 128u * (seq ? kDqBN : a.dep_rows);
                 const void* mk = seq ? static_cast<const void*>(&a.tk) : static_cast<const void*>(&a.tkd);
                 const void* mv = seq ? static_cast<const void*>(&a.tv) : static_cast<const void*>(&a.tvd);
-                mbar_arrive_expect_tx(&bars[kB_KFull + st], bytes);
-                for (int s = 0; s < Lay::kSlabs; ++s)
-                    tma_load_3d(dk + s * kSlabBytes, mk, &bars[kB_KFull + st], s * 64, row0, bh);
-                mbar_arrive_expect_tx(&bars[kB_VFull + st], bytes);
-                for (int s = 0; s < Lay::kSlabs; ++s)
-                    tma_load_3d(dv + s * kSlabBytes, mv, &bars[kB_VFull + st], s * 64, row0, bh);
+                mbar_arrive_expect_tx(&bars[kB_KVFull + st], 2 * bytes);
+                for (int s = 0; s < Lay::kSlabs; ++s) {
+                    tma_load_3d(dk + s * kDqSlab, mk, &bars[kB_KVFull + st], s * 64, row0, bh);
+                    tma_load_3d(dv + s * kDqSlab, mv, &bars[kB_KVFull + st], s * 64, row0, bh);
+                }
                 issued = i + 1;
             }
             mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag);
-            for (int i = max(0, issued - 2); i < issued; ++i) {
-                mbar_wait(&bars[kB_KFull + (i & 1)], (i >> 1) & 1, a.status, abort_flag);
-                mbar_wait(&bars[kB_VFull + (i & 1)], (i >> 1) & 1, a.status, abort_flag);
-            }
+            for (int i = max(0, issued - kDqStages); i < issued; ++i)
+                mbar_wait(&bars[kB_KVFull + i % kDqStages], (i / kDqStages) & 1, a.status, abort_flag);
         }
     } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer --
         if (lane == 0) {
-            const uint32_t id_seq = idesc_bf16(128, BN, false, false);
+            const uint32_t id_seq = idesc_bf16(128, kDqBN, false, false);
             const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
             const uint32_t id_dq = idesc_bf16(128, D, false, true);
             const uint32_t id_dd = idesc_bf16(128, a.dep_rows, true, true);
@@ -442,36 +478,47 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             const uint32_t do_addr = smem_u32(smem + Lay::kDO);
             const uint32_t ds_addr = smem_u32(smem + Lay::kDS);
             const uint32_t p_addr = smem_u32(smem + Lay::kP);
-            bool ok = mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag);
+            // S(j) = Q K_j^T and dP(j) = dO V_j^T into buffer j & 1.
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % kDqStages;
+                const int buf = j & 1;
+                if (!mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t id = j < n_seq ? id_seq : id_dep;
+                const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kKTile);
+                const uint32_t v_addr = smem_u32(smem + Lay::kV + st * Lay::kKTile);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t offq = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    const uint32_t offk = (kk >> 2) * kDqSlab + (kk & 3) * 32;
+                    umma_ss(tmem + kColS + buf * 64, desc_kmajor_sw128(q_addr + offq),
+                            desc_kmajor_sw128(k_addr + offk), id, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t offq = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    const uint32_t offk = (kk >> 2) * kDqSlab + (kk & 3) * 32;
+                    umma_ss(tmem + kColDP + buf * 64, desc_kmajor_sw128(do_addr + offq),
+                            desc_kmajor_sw128(v_addr + offk), id, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[kB_SFull + buf]);
+                return true;
+            };
+            bool ok = mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag) && issue_s(0);
             for (int i = 0; ok && i < nb; ++i) {
-                const int st = i & 1;
+                // the next block's scores first: its buffer was released when
+                // the math warps finished block i-1 (waited below last round)
+                if (i + 1 < nb && !issue_s(i + 1)) { ok = false; break; }
+                const int st = i % kDqStages;
+                const int buf = i & 1;
                 const bool seq = i < n_seq;
-                const uint32_t id = seq ? id_seq : id_dep;
-                const int n = seq ? BN : a.dep_rows;
-                const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kTile);
-                const uint32_t v_addr = smem_u32(smem + Lay::kV + st * Lay::kTile);
-                if (!mbar_wait(&bars[kB_KFull + st], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                const int n = seq ? kDqBN : a.dep_rows;
+                if (!mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    umma_ss(tmem + kColS, desc_kmajor_sw128(q_addr + off), desc_kmajor_sw128(k_addr + off),
-                            id, kk > 0 ? 1u : 0u);
-                }
-                if (!mbar_wait(&bars[kB_VFull + st], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    umma_ss(tmem + kColDP, desc_kmajor_sw128(do_addr + off), desc_kmajor_sw128(v_addr + off),
-                            id, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&bars[kB_SFull]);
-                if (!mbar_wait(&bars[kB_PReady], i & 1, a.status, abort_flag)) { ok = false; break; }
-                tc_fence_after();
+                const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kKTile);
                 for (int kk = 0; kk < n / 16; ++kk)
-                    umma_ts(tmem + kColDQ, tmem + kColS + kk * 8,
-                            desc_mnmajor_sw128(k_addr + kk * 2048, kSlabBytes), id_dq,
+                    umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8,
+                            desc_mnmajor_sw128(k_addr + kk * 2048, kDqSlab), id_dq,
                             (i > 0 || kk > 0) ? 1u : 0u);
                 if (!seq) {
 #pragma unroll
@@ -488,8 +535,10 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             umma_commit(&bars[kB_Final]);
         }
     } else {
+        // ------------------------------------------------------ math --------
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
+        const int mt = threadIdx.x - 64;                  // 0..127
         const bool row_real = r < R;
         const int g = row_real ? r / a.Tq : 0;
         const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
@@ -501,9 +550,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const float sl2 = a.scale_log2;
         unsigned char* sDS = smem + Lay::kDS;
         unsigned char* sP = smem + Lay::kP;
-        const size_t dep_base = static_cast<size_t>(bh) * a.T * a.L;   // first depth row of (b, hk)
+        __nv_bfloat16* stK = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kStage);
+        __nv_bfloat16* stV = stK + 64 * D;
+        const size_t dep_base = (static_cast<size_t>(bh) * a.T + t0) * a.L;  // first depth row of the tile
 
-        // Depth epilogue: TMEM lane = d index, columns = depth rows of block jd.
+        // dKd / dVd of depth block jd: TMEM lane = d index, column = depth row.
+        // Transposed through shared memory, then 16-byte row stores.
         auto depth_epilogue = [&](int jd) {
             uint32_t xk[64], xv[64];
             tmem_ld32(lane_base + kColDKd, xk);
@@ -511,81 +563,87 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             tmem_ld32(lane_base + kColDVd, xv);
             tmem_ld32(lane_base + kColDVd + 32, xv + 32);
             tmem_wait_ld();
-            const int dd = r;                      // d index of this lane
-            const int row0 = jd * a.dep_rows;      // relative to t0*L
-            const int nvalid = min(a.dep_rows, dep_total - row0);
-            if (dd < D) {
-                __nv_bfloat16* pk = a.dKd + (dep_base + static_cast<size_t>(t0) * a.L + row0) * D + dd;
-                __nv_bfloat16* pv = a.dVd + (dep_base + static_cast<size_t>(t0) * a.L + row0) * D + dd;
+            named_bar_sync(1, kMathThreads);             // staging free (previous readers done)
+            if (r < D) {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
-                    if (c < nvalid) {
-                        pk[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
-                        pv[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xv[c]));
-                    }
+                    stK[c * D + r] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
+                    stV[c * D + r] = __float2bfloat16_rn(__uint_as_float(xv[c]));
                 }
+            }
+            named_bar_sync(1, kMathThreads);
+            const int row0 = jd * a.dep_rows;
+            const int nvalid = min(a.dep_rows, dep_total - row0);
+            constexpr int kVecPerRow = D / 8;
+            const uint4* sk4 = reinterpret_cast<const uint4*>(stK);
+            const uint4* sv4 = reinterpret_cast<const uint4*>(stV);
+            uint4* gk = reinterpret_cast<uint4*>(a.dKd + (dep_base + row0) * D);
+            uint4* gv = reinterpret_cast<uint4*>(a.dVd + (dep_base + row0) * D);
+            for (int u = mt; u < nvalid * kVecPerRow; u += kMathThreads) {
+                gk[u] = sk4[u];
+                gv[u] = sv4[u];
             }
         };
 
         bool ok = true;
         int jd = 0;
         for (int i = 0; i < nb; ++i) {
+            const int buf = i & 1;
             const bool seq = i < n_seq;
-            if (!seq && jd >= 1) {
-                if (!mbar_wait(&bars[kB_DDFull], (jd - 1) & 1, a.status, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                depth_epilogue(jd - 1);
-            }
-            if (!mbar_wait(&bars[kB_SFull], i & 1, a.status, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&bars[kB_SFull + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const int nchunk = seq ? 4 : 2;
-            int lo = 0, hi = BN, kb = 0;
+            uint32_t s[64], dp[64], dsk[32], pk[32];
+            tmem_ld32(lane_base + kColS + buf * 64, s);
+            tmem_ld32(lane_base + kColS + buf * 64 + 32, s + 32);
+            tmem_ld32(lane_base + kColDP + buf * 64, dp);
+            tmem_ld32(lane_base + kColDP + buf * 64 + 32, dp + 32);
+            tmem_wait_ld();
+            int lo = 0, hi = kDqBN, kb = 0;
             if (seq) {
-                kb = i * BN;
+                kb = i * kDqBN;
             } else {
                 lo = t_row * a.L - (t0 * a.L + jd * a.dep_rows);
                 hi = min(lo + a.L, a.dep_rows);
             }
-            for (int c4 = 0; c4 < nchunk; ++c4) {
-                uint32_t s[32], dp[32], dsk[16], pk[16];
-                tmem_ld32(lane_base + kColS + 32 * c4, s);
-                tmem_ld32(lane_base + kColDP + 32 * c4, dp);
-                tmem_wait_ld();
+            const bool all_visible = seq && kb + kDqBN - 1 <= t_row;
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float p2[2], d2[2];
+            for (int e = 0; e < 64; e += 2) {
+                float p2[2], d2[2];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int c = 32 * c4 + e + u;
-                        const bool vis = seq ? (kb + c <= t_row) : (c >= lo && c < hi);
-                        const float p = vis ? ex2(fmaf(__uint_as_float(s[e + u]), sl2, -lse2)) : 0.0f;
-                        p2[u] = p;
-                        d2[u] = vis ? p * (__uint_as_float(dp[e + u]) - Dr) : 0.0f;
-                    }
-                    dsk[e / 2] = pack_bf16(d2[0], d2[1]);
-                    pk[e / 2] = pack_bf16(p2[0], p2[1]);
+                for (int u = 0; u < 2; ++u) {
+                    const int c = e + u;
+                    const bool vis = all_visible || (seq ? (kb + c <= t_row) : (c >= lo && c < hi));
+                    const float p = vis ? ex2(fmaf(__uint_as_float(s[c]), sl2, -lse2)) : 0.0f;
+                    p2[u] = p;
+                    d2[u] = vis ? p * (__uint_as_float(dp[c]) - Dr) : 0.0f;
                 }
-                tmem_st16(lane_base + kColS + 16 * c4, dsk);
-                if (!seq) {
-                    // row r of the [q][depth] staging tiles, 128-byte swizzle
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int ch = 4 * c4 + e;
-                        const uint32_t off = r * 128 + ((ch ^ (r & 7)) << 4);
-                        *reinterpret_cast<uint4*>(sDS + off) =
-                            make_uint4(dsk[4 * e], dsk[4 * e + 1], dsk[4 * e + 2], dsk[4 * e + 3]);
-                        *reinterpret_cast<uint4*>(sP + off) =
-                            make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                    }
-                }
+                dsk[e / 2] = pack_bf16(d2[0], d2[1]);
+                pk[e / 2] = pack_bf16(p2[0], p2[1]);
             }
-            tmem_wait_st();
+            tmem_st32(lane_base + kColS + buf * 64, dsk);
             if (!seq) {
+                // the previous depth block's MMAs are done before its staging
+                // tiles and TMEM columns are reused
+                if (jd >= 1) {
+                    if (!mbar_wait(&bars[kB_DDFull], (jd - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    depth_epilogue(jd - 1);
+                }
+                // row r of the [q][depth] staging tiles, 128-byte swizzle
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint32_t off = r * 128 + ((ch ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4*>(sDS + off) =
+                        make_uint4(dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
+                    *reinterpret_cast<uint4*>(sP + off) =
+                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                }
                 fence_proxy_async_smem();
                 ++jd;
             }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[kB_PReady]);
+            mbar_arrive(&bars[kB_PReady + buf]);
         }
         if (ok && n_dep > 0) {
             if (mbar_wait(&bars[kB_DDFull], (n_dep - 1) & 1, a.status, abort_flag)) {
@@ -642,7 +700,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     DkdvArgs A;
     A.B = p.B; A.Hq = p.Hq; A.Hk = p.Hk; A.T = p.T; A.G = p.G;
     A.n_kt = (p.T + BN - 1) / BN;
-    A.n_qb = (p.T + BM - 1) / BM;
+    A.n_qb = (p.T + kKvBQ - 1) / kKvBQ;
     A.scale = p.scale; A.scale_log2 = p.scale_log2;
     A.LSE = LSE; A.Drow = Dws;
     A.dK = static_cast<__nv_bfloat16*>(dK);
@@ -650,8 +708,8 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     A.status = device_status_word();
     if ((e = make_tma_3d_bf16(&A.tk, K, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&A.tv, V, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
-    if ((e = make_tma_3d_bf16(&A.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, BM, 1)) != cudaSuccess) return e;
-    if ((e = make_tma_3d_bf16(&A.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, BM, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&A.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&A.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
     {
         const uint32_t smem = DkdvLayout<D>::kDynSmem;
         if ((e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -678,15 +736,15 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     B.status = device_status_word();
     if ((e = make_tma_3d_bf16(&B.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&B.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
-    B.tk = A.tk;
-    B.tv = A.tv;
+    if ((e = make_tma_3d_bf16(&B.tk, K, D, p.T, (uint64_t)p.B * p.Hk, kDqBN, 1)) != cudaSuccess) return e;
+    if ((e = make_tma_3d_bf16(&B.tv, V, D, p.T, (uint64_t)p.B * p.Hk, kDqBN, 1)) != cudaSuccess) return e;
     if (p.L > 0) {
         const uint64_t rows = (uint64_t)p.T * p.L;
         if ((e = make_tma_3d_bf16(&B.tkd, Kd, D, rows, (uint64_t)p.B * p.Hk, B.dep_rows, 1)) != cudaSuccess) return e;
         if ((e = make_tma_3d_bf16(&B.tvd, Vd, D, rows, (uint64_t)p.B * p.Hk, B.dep_rows, 1)) != cudaSuccess) return e;
     } else {
-        B.tkd = A.tk;
-        B.tvd = A.tv;
+        B.tkd = B.tk;
+        B.tvd = B.tv;
     }
     {
         const uint32_t smem = DqLayout<D>::kDynSmem;

@@ -13,9 +13,12 @@
 // group, and the depth rows of the tile's Tq tokens are one contiguous range
 // [t0*L, (t0+Tq)*L) of the token-major depth tensor.
 //
-// CTA roles (192 threads):
-//   warp 0      TMA producer: Q once, then K/V (or K_depth/V_depth) tiles
-//               through a 2-stage ring of mbarriers.
+// CTA roles (224 threads):
+//   warp 0      TMA producer of Q (once) and of the K (or K_depth) tiles;
+//   warp 6      TMA producer of the V (or V_depth) tiles.  K and V have rings
+//               of their own: a K stage frees as soon as S_i = Q K_i^T is
+//               done, a V stage only when O += P_i V_i is, so the next K
+//               tiles stream in while PV still holds older V tiles.
 //   warp 1      TMEM allocator and MMA issuer (one thread):
 //               S_i = Q K_i^T into one of two TMEM S buffers, then
 //               O += P_{i-1} V_{i-1} with P read from TMEM.
@@ -38,8 +41,15 @@ using namespace ptx;
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = 128;          // sequence keys per block
-constexpr int kStages = 2;       // K/V shared-memory stages
-constexpr int kThreads = 192;
+#ifndef MODA_FWD_KSTAGES
+#define MODA_FWD_KSTAGES 3
+#endif
+#ifndef MODA_FWD_VSTAGES
+#define MODA_FWD_VSTAGES 3
+#endif
+constexpr int kKStages = MODA_FWD_KSTAGES;   // K ring: a stage frees when S_i is done
+constexpr int kVStages = MODA_FWD_VSTAGES;   // V ring: a stage frees when PV_i is done
+constexpr int kThreads = 224;
 constexpr int kSoftmaxThreads = 128;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kSlabBytes = 128 * 128;   // 128 rows x 64 bf16
@@ -61,8 +71,8 @@ struct Layout {
     static constexpr uint32_t kTile = kSlabs * kSlabBytes;
     static constexpr uint32_t kQ = 0;
     static constexpr uint32_t kK = kTile;
-    static constexpr uint32_t kV = kK + kStages * kTile;
-    static constexpr uint32_t kBar = kV + kStages * kTile;
+    static constexpr uint32_t kV = kK + kKStages * kTile;
+    static constexpr uint32_t kBar = kV + kVStages * kTile;
     static constexpr uint32_t kBytes = kBar + 256;
     // + alignment slack; never below 120 KB so that one CTA (and one 512-column
     // TMEM allocation) is resident per SM.
@@ -70,8 +80,9 @@ struct Layout {
 };
 
 // Barrier slots.
-enum { kQFull = 0, kKFull = 1, kVFull = 3, kKVEmpty = 5, kSFull = 7, kPReady = 9, kOReady = 11,
-       kOFinal = 12, kNumBars = 13 };
+enum { kQFull = 0, kKFull = 1, kKEmpty = kKFull + kKStages, kVFull = kKEmpty + kKStages,
+       kVEmpty = kVFull + kVStages, kSFull = kVEmpty + kVStages, kPReady = kSFull + 2,
+       kOReady = kPReady + 2, kOFinal = kOReady + 1, kNumBars = kOFinal + 1 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __grid_constant__ FwdArgs a) {
@@ -104,10 +115,13 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kQFull], 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(&bars[kKFull + s], 1);
+            mbar_init(&bars[kKEmpty + s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(&bars[kVFull + s], 1);
-            mbar_init(&bars[kKVEmpty + s], 1);
+            mbar_init(&bars[kVEmpty + s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[kSFull + s], 1);
@@ -137,51 +151,44 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == 0) {
-        // ------------------------------------------------------ producer ----
+    if (warp == 0 || warp == 6) {
+        // ------------------------------------------------------ producers ---
+        // warp 0: Q, then K_i (sequence) / K_depth tiles; warp 6: V tiles.
         if (lane == 0) {
-            prefetch_tmap(&a.tq);
-            prefetch_tmap(&a.tk);
-            prefetch_tmap(&a.tv);
-            if (a.L > 0) { prefetch_tmap(&a.tkd); prefetch_tmap(&a.tvd); }
-            const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
-            mbar_arrive_expect_tx(&bars[kQFull], q_bytes);
-            for (int s = 0; s < Lay::kSlabs; ++s)
-                tma_load_3d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, t0, b * a.Hq + hk * a.G);
+            const bool is_k = warp == 0;
+            const int nst = is_k ? kKStages : kVStages;
+            uint64_t* full = &bars[is_k ? kKFull : kVFull];
+            uint64_t* empty = &bars[is_k ? kKEmpty : kVEmpty];
+            unsigned char* ring = is_k ? sK : sV;
+            const void* m_seq = is_k ? static_cast<const void*>(&a.tk) : static_cast<const void*>(&a.tv);
+            const void* m_dep = is_k ? static_cast<const void*>(&a.tkd) : static_cast<const void*>(&a.tvd);
+            prefetch_tmap(m_seq);
+            if (a.L > 0) prefetch_tmap(m_dep);
+            if (is_k) {
+                prefetch_tmap(&a.tq);
+                const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
+                mbar_arrive_expect_tx(&bars[kQFull], q_bytes);
+                for (int s = 0; s < Lay::kSlabs; ++s)
+                    tma_load_3d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, t0, b * a.Hq + hk * a.G);
+            }
             int issued = 0;
             for (int i = 0; i < nb; ++i) {
-                const int st = i % kStages;
-                if (i >= kStages &&
-                    !mbar_wait(&bars[kKVEmpty + st], ((i / kStages) - 1) & 1, a.status, abort_flag))
+                const int st = i % nst;
+                if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1, a.status, abort_flag))
                     break;
-                unsigned char* dk = sK + st * Lay::kTile;
-                unsigned char* dv = sV + st * Lay::kTile;
-                if (i < n_seq) {
-                    const uint32_t bytes = Lay::kTile;
-                    mbar_arrive_expect_tx(&bars[kKFull + st], bytes);
-                    for (int s = 0; s < Lay::kSlabs; ++s)
-                        tma_load_3d(dk + s * kSlabBytes, &a.tk, &bars[kKFull + st], s * 64, i * BN, bh);
-                    mbar_arrive_expect_tx(&bars[kVFull + st], bytes);
-                    for (int s = 0; s < Lay::kSlabs; ++s)
-                        tma_load_3d(dv + s * kSlabBytes, &a.tv, &bars[kVFull + st], s * 64, i * BN, bh);
-                } else {
-                    const int row0 = t0 * a.L + (i - n_seq) * a.dep_rows;
-                    const uint32_t bytes = Lay::kSlabs * 128u * a.dep_rows;
-                    mbar_arrive_expect_tx(&bars[kKFull + st], bytes);
-                    for (int s = 0; s < Lay::kSlabs; ++s)
-                        tma_load_3d(dk + s * kSlabBytes, &a.tkd, &bars[kKFull + st], s * 64, row0, bh);
-                    mbar_arrive_expect_tx(&bars[kVFull + st], bytes);
-                    for (int s = 0; s < Lay::kSlabs; ++s)
-                        tma_load_3d(dv + s * kSlabBytes, &a.tvd, &bars[kVFull + st], s * 64, row0, bh);
-                }
+                unsigned char* dst = ring + st * Lay::kTile;
+                const bool seq = i < n_seq;
+                const int row0 = seq ? i * BN : t0 * a.L + (i - n_seq) * a.dep_rows;
+                const uint32_t bytes = Lay::kSlabs * 128u * (seq ? BN : a.dep_rows);
+                mbar_arrive_expect_tx(&full[st], bytes);
+                for (int s = 0; s < Lay::kSlabs; ++s)
+                    tma_load_3d(dst + s * kSlabBytes, seq ? m_seq : m_dep, &full[st], s * 64, row0, bh);
                 issued = i + 1;
             }
             // Let every load this thread started land before the CTA retires.
-            mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
-            for (int i = max(0, issued - kStages); i < issued; ++i) {
-                mbar_wait(&bars[kKFull + i % kStages], (i / kStages) & 1, a.status, abort_flag);
-                mbar_wait(&bars[kVFull + i % kStages], (i / kStages) & 1, a.status, abort_flag);
-            }
+            if (is_k) mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
+            for (int i = max(0, issued - nst); i < issued; ++i)
+                mbar_wait(&full[i % nst], (i / nst) & 1, a.status, abort_flag);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer --
@@ -192,10 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             const uint32_t q_addr = smem_u32(sQ);
             bool ok = mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
             auto issue_pv = [&](int j) -> bool {
-                const int st = j % kStages;
+                const int st = j % kVStages;
                 const int sb = j & 1;
                 if (!mbar_wait(&bars[kPReady + sb], (j >> 1) & 1, a.status, abort_flag)) return false;
-                if (!mbar_wait(&bars[kVFull + st], (j / kStages) & 1, a.status, abort_flag)) return false;
+                if (!mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status, abort_flag)) return false;
                 tc_fence_after();
                 const int krows = j < n_seq ? BN : a.dep_rows;
                 const uint32_t v_addr = smem_u32(sV + st * Lay::kTile);
@@ -203,14 +210,14 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     const uint64_t bdesc = desc_mnmajor_sw128(v_addr + kk * 2048, kSlabBytes);
                     umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, bdesc, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bars[kKVEmpty + st]);
+                umma_commit(&bars[kVEmpty + st]);
                 umma_commit(&bars[kOReady]);
                 return true;
             };
             for (int i = 0; ok && i < nb; ++i) {
-                const int st = i % kStages;
+                const int st = i % kKStages;
                 const int sb = i & 1;
-                if (!mbar_wait(&bars[kKFull + st], (i / kStages) & 1, a.status, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&bars[kKFull + st], (i / kKStages) & 1, a.status, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t k_addr = smem_u32(sK + st * Lay::kTile);
                 const uint32_t id = i < n_seq ? id_seq : id_dep;
@@ -221,12 +228,13 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                             desc_kmajor_sw128(k_addr + off), id, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[kSFull + sb]);
+                umma_commit(&bars[kKEmpty + st]);
                 if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
             }
             if (ok) ok = issue_pv(nb - 1);
             umma_commit(&bars[kOFinal]);
         }
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ------------------------------------------------------ softmax -----
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
         const int r = quarter * 32 + lane;            // tile row
