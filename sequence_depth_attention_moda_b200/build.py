@@ -44,8 +44,8 @@ def _deps_mtime():
     return max(os.path.getmtime(h) for h in hdrs)
 
 
-def _compile(src: str, force: bool, verbose: bool, extra=()):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, force: bool, verbose: bool, extra=(), build_dir: str = BUILD):
+    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
     if (not force and os.path.exists(obj)
             and os.path.getmtime(obj) >= max(os.path.getmtime(src), _deps_mtime())):
         return obj, None
@@ -56,28 +56,34 @@ def _compile(src: str, force: bool, verbose: bool, extra=()):
     return obj, (res.stdout + res.stderr) if verbose else None
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compile every .cu under csrc/ for sm_100a and link lib/libmoda.so."""
-    os.makedirs(BUILD, exist_ok=True)
-    os.makedirs(LIB_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          defines=(), out: str | None = None) -> str:
+    """Compile every .cu under csrc/ for sm_100a and link lib/libmoda.so
+    (or `out`, with extra -D `defines`, into a separate object directory)."""
+    lib_path = out or LIB
+    build_dir = BUILD if not defines else os.path.join(BUILD, "v_" + "_".join(d.replace("=", "") for d in defines))
+    os.makedirs(build_dir, exist_ok=True)
+    os.makedirs(os.path.dirname(lib_path), exist_ok=True)
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    extra += [f"-D{d}" for d in defines]
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, force or ptxas_info, verbose or ptxas_info, extra), srcs))
+        results = list(ex.map(lambda s: _compile(s, force or ptxas_info, verbose or ptxas_info, extra,
+                                                 build_dir), srcs))
     objs = [o for o, _ in results]
     for _, log in results:
         if log:
             print(log, file=sys.stderr)
-    if (force or not os.path.exists(LIB)
-            or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs)):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if (force or not os.path.exists(lib_path)
+            or os.path.getmtime(lib_path) < max(os.path.getmtime(o) for o in objs)):
+        tmp = lib_path + f".tmp{os.getpid()}"
         cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt",
                "-lpthread"]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"link failed:\n{res.stdout}{res.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":

@@ -47,6 +47,31 @@ constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Optional hand-off timeline of CTA 0 (clock64 per event and iteration), only
+// in builds with -DMODA_TRACE; read back with moda_trace_copy_bwd().
+#ifdef MODA_TRACE
+constexpr int kTraceSlots = 16, kTraceIters = 96;
+__device__ long long g_trace_bwd[kTraceSlots * kTraceIters];
+__device__ long long g_trace_dq[kTraceSlots * kTraceIters];
+#define MODA_TR(slot, it)                                                   \
+    do {                                                                    \
+        if (blockIdx.x == 0 && (it) >= 0 && (it) < kTraceIters)             \
+            g_trace_bwd[(slot) * kTraceIters + (it)] = clock64();           \
+    } while (0)
+#define MODA_TRQ(slot, it)                                                  \
+    do {                                                                    \
+        if (blockIdx.x == 0 && (it) >= 0 && (it) < kTraceIters)             \
+            g_trace_dq[(slot) * kTraceIters + (it)] = clock64();            \
+    } while (0)
+#else
+#define MODA_TR(slot, it) \
+    do {                  \
+    } while (0)
+#define MODA_TRQ(slot, it) \
+    do {                   \
+    } while (0)
+#endif
+
 // ------------------------------------------------------------ 1. rowdot ----
 template <int D>
 __global__ void __launch_bounds__(256) rowdot_kernel(long long nrows,
@@ -93,7 +118,10 @@ struct DkdvArgs {
 };
 
 constexpr int kKvBQ = 64;               // query rows per iteration
-constexpr int kKvStages = 4;            // Q/dO ring depth
+#ifndef MODA_DKDV_STAGES
+#define MODA_DKDV_STAGES 4
+#endif
+constexpr int kKvStages = MODA_DKDV_STAGES;   // Q/dO ring depth
 constexpr uint32_t kKvSlab = 64 * 128;
 
 template <int D>
@@ -173,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 if (it >= kKvStages &&
                     !mbar_wait(&bars[kA_QEmpty + st], ((it / kKvStages) - 1) & 1, a.status, abort_flag))
                     break;
+                MODA_TR(9, it);
                 const int g = it / nqb;
                 const int qb = qb0 + (it - g * nqb);
                 const int qh = b * a.Hq + hk * a.G + g;
@@ -200,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 const int st = j % kKvStages;
                 const int buf = j & 1;
                 if (!mbar_wait(&bars[kA_QFull + st], (j / kKvStages) & 1, a.status, abort_flag)) return false;
+                MODA_TR(10, j);
                 tc_fence_after();
                 const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kQTile);
                 const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kQTile);
@@ -222,10 +252,13 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             };
             bool ok = mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag) && (n_it == 0 || issue_s(0));
             for (int it = 0; ok && it < n_it; ++it) {
+                MODA_TR(0, it);
                 if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
+                MODA_TR(1, it);
                 const int st = it % kKvStages;
                 const int buf = it & 1;
                 if (!mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                MODA_TR(2, it);
                 tc_fence_after();
                 const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kQTile);
                 const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kQTile);
@@ -238,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                             desc_mnmajor_sw128(q_addr + kk * 2048, kKvSlab), id_g, acc);
                 }
                 umma_commit(&bars[kA_QEmpty + st]);
+                MODA_TR(3, it);
             }
             umma_commit(&bars[kA_Final]);
         }
@@ -261,7 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 sbuf[64 + mt] = t < a.T ? a.Drow[qrow0 + t] : 0.0f;
             }
             named_bar_sync(1, kMathThreads);
+            if (mt == 0) MODA_TR(4, it);
             if (!mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+            if (mt == 0) MODA_TR(5, it);
             tc_fence_after();
             const int tq0 = qb * kKvBQ;
             const bool diag = tq0 < kt * BN + BN;         // some key of the tile is after some query
@@ -271,23 +307,38 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             tmem_ld32(lane_base + 128 + buf * 64, dp);
             tmem_ld32(lane_base + 128 + buf * 64 + 32, dp + 32);
             tmem_wait_ld();
+            if (mt == 0) MODA_TR(6, it);
+            // visible columns c >= k - tq0 on the diagonal blocks; selects, no
+            // branch per element (masked: score -inf, dP = D, so P = dS = 0)
+            const int vlo = diag ? k - tq0 : 0;
+            const float4* sl4 = reinterpret_cast<const float4*>(sbuf);
+            const float4* sd4 = reinterpret_cast<const float4*>(sbuf + 64);
 #pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-                float p2[2], d2[2];
+            for (int e = 0; e < 64; e += 4) {
+                const float4 l4 = sl4[e / 4];
+                const float4 d4 = sd4[e / 4];
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+                float p4[4], g4[4];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     const int c = e + u;
-                    const bool vis = !diag || k <= tq0 + c;
-                    const float p = vis ? ex2(fmaf(__uint_as_float(s[c]), sl2, -sbuf[c])) : 0.0f;
-                    p2[u] = p;
-                    d2[u] = vis ? p * (__uint_as_float(dp[c]) - sbuf[64 + c]) : 0.0f;
+                    const bool vis = c >= vlo;
+                    const float sv = vis ? __uint_as_float(s[c]) : -INFINITY;
+                    const float dv = vis ? __uint_as_float(dp[c]) : dvv[u];
+                    p4[u] = ex2(fmaf(sv, sl2, -lv[u]));
+                    g4[u] = p4[u] * (dv - dvv[u]);
                 }
-                pk[e / 2] = pack_bf16(p2[0], p2[1]);
-                dk[e / 2] = pack_bf16(d2[0], d2[1]);
+                pk[e / 2] = pack_bf16(p4[0], p4[1]);
+                pk[e / 2 + 1] = pack_bf16(p4[2], p4[3]);
+                dk[e / 2] = pack_bf16(g4[0], g4[1]);
+                dk[e / 2 + 1] = pack_bf16(g4[2], g4[3]);
             }
+            if (mt == 0) MODA_TR(7, it);
             tmem_st32(lane_base + buf * 64, pk);
             tmem_st32(lane_base + 128 + buf * 64, dk);
             tmem_wait_st();
+            if (mt == 0) MODA_TR(8, it);
             tc_fence_before();
             mbar_arrive(&bars[kA_PReady + buf]);
         }
@@ -344,7 +395,10 @@ struct DqArgs {
 };
 
 constexpr int kDqBN = 64;            // rows per key / depth block
-constexpr int kDqStages = 3;         // K/V ring depth
+#ifndef MODA_DQ_STAGES
+#define MODA_DQ_STAGES 3
+#endif
+constexpr int kDqStages = MODA_DQ_STAGES;   // K/V ring depth
 constexpr uint32_t kDqSlab = 64 * 128;   // 64 rows x 64 bf16
 
 template <int D>
@@ -483,6 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 const int st = j % kDqStages;
                 const int buf = j & 1;
                 if (!mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag)) return false;
+                MODA_TRQ(8, j);
                 tc_fence_after();
                 const uint32_t id = j < n_seq ? id_seq : id_dep;
                 const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kKTile);
@@ -508,12 +563,15 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             for (int i = 0; ok && i < nb; ++i) {
                 // the next block's scores first: its buffer was released when
                 // the math warps finished block i-1 (waited below last round)
+                MODA_TRQ(0, i);
                 if (i + 1 < nb && !issue_s(i + 1)) { ok = false; break; }
+                MODA_TRQ(1, i);
                 const int st = i % kDqStages;
                 const int buf = i & 1;
                 const bool seq = i < n_seq;
                 const int n = seq ? kDqBN : a.dep_rows;
                 if (!mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                MODA_TRQ(2, i);
                 tc_fence_after();
                 const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kKTile);
                 for (int kk = 0; kk < n / 16; ++kk)
@@ -531,6 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     umma_commit(&bars[kB_DDFull]);
                 }
                 umma_commit(&bars[kB_KVEmpty + st]);
+                MODA_TRQ(3, i);
             }
             umma_commit(&bars[kB_Final]);
         }
@@ -590,7 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         for (int i = 0; i < nb; ++i) {
             const int buf = i & 1;
             const bool seq = i < n_seq;
+            if (mt == 0) MODA_TRQ(4, i);
             if (!mbar_wait(&bars[kB_SFull + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+            if (mt == 0) MODA_TRQ(5, i);
             tc_fence_after();
             uint32_t s[64], dp[64], dsk[32], pk[32];
             tmem_ld32(lane_base + kColS + buf * 64, s);
@@ -606,20 +667,38 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 hi = min(lo + a.L, a.dep_rows);
             }
             const bool all_visible = seq && kb + kDqBN - 1 <= t_row;
+            // Masked entries get score -inf and dP 0 by selects (no branch per
+            // element), so exp2 runs unconditionally and yields exactly 0.
+            if (all_visible) {
 #pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-                float p2[2], d2[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int c = e + u;
-                    const bool vis = all_visible || (seq ? (kb + c <= t_row) : (c >= lo && c < hi));
-                    const float p = vis ? ex2(fmaf(__uint_as_float(s[c]), sl2, -lse2)) : 0.0f;
-                    p2[u] = p;
-                    d2[u] = vis ? p * (__uint_as_float(dp[c]) - Dr) : 0.0f;
+                for (int e = 0; e < 64; e += 2) {
+                    const float p0 = ex2(fmaf(__uint_as_float(s[e]), sl2, -lse2));
+                    const float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), sl2, -lse2));
+                    dsk[e / 2] = pack_bf16(p0 * (__uint_as_float(dp[e]) - Dr),
+                                           p1 * (__uint_as_float(dp[e + 1]) - Dr));
+                    pk[e / 2] = pack_bf16(p0, p1);
                 }
-                dsk[e / 2] = pack_bf16(d2[0], d2[1]);
-                pk[e / 2] = pack_bf16(p2[0], p2[1]);
+            } else {
+                // visible columns: seq c <= t_row - kb; depth lo <= c < hi
+                const int vlo = seq ? 0 : lo;
+                const int vhi = seq ? t_row - kb + 1 : hi;
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    float p2[2], d2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int c = e + u;
+                        const bool vis = c >= vlo && c < vhi;
+                        const float sv = vis ? __uint_as_float(s[c]) : -INFINITY;
+                        const float dv = vis ? __uint_as_float(dp[c]) : Dr;
+                        p2[u] = ex2(fmaf(sv, sl2, -lse2));
+                        d2[u] = p2[u] * (dv - Dr);
+                    }
+                    dsk[e / 2] = pack_bf16(d2[0], d2[1]);
+                    pk[e / 2] = pack_bf16(p2[0], p2[1]);
+                }
             }
+            if (mt == 0) MODA_TRQ(6, i);
             tmem_st32(lane_base + kColS + buf * 64, dsk);
             if (!seq) {
                 // the previous depth block's MMAs are done before its staging
@@ -642,6 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 ++jd;
             }
             tmem_wait_st();
+            if (mt == 0) MODA_TRQ(7, i);
             tc_fence_before();
             mbar_arrive(&bars[kB_PReady + buf]);
         }
@@ -759,6 +839,17 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
 }
 
 }  // namespace
+
+#ifdef MODA_TRACE
+extern "C" int moda_trace_copy_bwd(long long* host, int n) {
+    const int cnt = n < kTraceSlots * kTraceIters ? n : kTraceSlots * kTraceIters;
+    return cudaMemcpyFromSymbol(host, g_trace_bwd, cnt * sizeof(long long)) == cudaSuccess ? cnt : -1;
+}
+extern "C" int moda_trace_copy_dq(long long* host, int n) {
+    const int cnt = n < kTraceSlots * kTraceIters ? n : kTraceSlots * kTraceIters;
+    return cudaMemcpyFromSymbol(host, g_trace_dq, cnt * sizeof(long long)) == cudaSuccess ? cnt : -1;
+}
+#endif
 
 cudaError_t launch_bwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, const void* O, const float* LSE,
