@@ -47,7 +47,7 @@ BWD_FACTOR = 2.5
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the L=0 twin and T=64K lines")
@@ -70,68 +70,68 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+    """SM clock and throttle reasons sampled (NVML, every 10 ms, from a thread)
+    while the timed region runs; nvidia-smi is the fallback."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, index: int):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []       # (sm_mhz, reasons bitmask)
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((float(mhz), int(rs)))
+                except Exception:
+                    pass
+                self._stop.wait(0.01)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            time.sleep(0.05)
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+        return False
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml"}
+        reasons = sorted({nm for _, rs in self.samples for nm, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": float(np.median([m for m, _ in self.samples])), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
-def traffic_from_profile(kernel_src: str):
-    """Per-launch DRAM bytes of the dominant launch from the committed ncu
-    summary, or None when the kernel source has changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", "moda_bwd_layer_T4k_traffic.md")
+def traffic_from_profile(kernel: str, kernel_src: str):
+    """Per-launch DRAM bytes (read + write) of `kernel` from the committed ncu
+    summary, or None when its source has changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic_layer_T4k.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_hash = re.search(r"source sha256: ([0-9a-f]{16})", text)
-    m_bytes = re.search(r"bytes per call: (\d+)", text)
+    m_bytes = re.search(r"^\| %s \| (\d+) \|" % re.escape(kernel), text, re.M)
     if not m_hash or not m_bytes:
         return None
     cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
@@ -168,6 +168,9 @@ class Runner:
         return (2 if self.w.L else 0) + 1 + (3 if self.backward else 0)
 
     def step(self, ev=None):
+        """One step.  With `ev` (8 CUDA events) the repack is bracketed by
+        ev[0:2] and the library records ev[2:4] around the forward kernel and
+        ev[4:8] around the backward's three kernels (moda_set_phase_events)."""
         m, x = self.moda, self.x
         if ev is not None:
             ev[0].record()
@@ -176,14 +179,15 @@ class Runner:
             m.moda_repack_depth(self.sh, x["Vd_layer"], self.Vd)
         if ev is not None:
             ev[1].record()
+            m.moda_set_phase_events(ev[2:4])
         m.moda_fwd(self.sh, x["Q"], x["K"], x["V"], self.Kd, self.Vd, self.O, self.LSE)
-        if ev is not None:
-            ev[2].record()
         if self.backward:
+            if ev is not None:
+                m.moda_set_phase_events(ev[4:8])
             m.moda_bwd(self.sh, x["Q"], x["K"], x["V"], self.Kd, self.Vd, self.O, self.LSE, x["dO"],
                        self.dQ, self.dK, self.dV, self.dKd, self.dVd, self.ws, self.nws)
         if ev is not None:
-            ev[3].record()
+            m.moda_set_phase_events([])
 
     def outputs(self):
         outs = [self.O, self.LSE]
@@ -198,11 +202,24 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """Max of a per-rank time over all ranks (NCCL on GPUs, gloo on CPUs)."""
     if world == 1:
         return v
-    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    dev = (torch.device("cuda", torch.cuda.current_device())
+           if torch.distributed.get_backend() == "nccl" else torch.device("cpu"))
+    t = torch.tensor([v], device=dev, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w: I.Workload, rank: int) -> int:
+    """Each rank draws its own batch (data parallel)."""
+    return w.seed + 1000 * rank
+
+
+def job_value(flops_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
 
 
 def time_steps(r: Runner, steps: int, warmup: int, world: int, per_call=False, clocks=None):
@@ -211,7 +228,12 @@ def time_steps(r: Runner, steps: int, warmup: int, world: int, per_call=False, c
     for _ in range(warmup):
         r.step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)] if per_call else None
+    evs = None
+    if per_call:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(steps)]
+        for e in (e for row in evs for e in row):
+            e.record()           # creates the event so its handle can be passed on
+        torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -227,8 +249,12 @@ def time_steps(r: Runner, steps: int, warmup: int, world: int, per_call=False, c
     calls = None
     if per_call:
         calls = {"repack": np.mean([e[0].elapsed_time(e[1]) for e in evs]),
-                 "fwd": np.mean([e[1].elapsed_time(e[2]) for e in evs]),
-                 "bwd": np.mean([e[2].elapsed_time(e[3]) for e in evs])}
+                 "fwd": np.mean([e[2].elapsed_time(e[3]) for e in evs])}
+        if r.backward:
+            calls.update(rowdot=np.mean([e[4].elapsed_time(e[5]) for e in evs]),
+                         dkdv=np.mean([e[5].elapsed_time(e[6]) for e in evs]),
+                         dq=np.mean([e[6].elapsed_time(e[7]) for e in evs]),
+                         bwd=np.mean([e[4].elapsed_time(e[7]) for e in evs]))
     return max_over_ranks(ms, world), calls
 
 
@@ -309,30 +335,41 @@ def run_ours(args):
     moda.load()
     peaks = load_peaks()
     w = WORKLOAD
-    x = I.make_inputs(w, device="cuda", seed=w.seed + 1000 * rank)
+    x = I.make_inputs(w, device="cuda", seed=rank_seed(w, rank))
     r = Runner(w, x)
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(int(vis.split(",")[local]) if vis else torch.cuda.current_device())
     ms, calls = time_steps(r, args.steps, args.warmup, world, per_call=True, clocks=clocks)
     moda.moda_check_status()
     flops_step = w.fwd_flops() * (1 + BWD_FACTOR)
-    value = world * flops_step / (ms * 1e-3) / 1e12
+    value = job_value(flops_step, ms, world)
     per_gpu = value / world
 
-    # roofline of the dominant launch group: the backward call (rowdot + dkdv + dq)
-    bwd_flops = w.fwd_flops() * BWD_FACTOR
-    kernel_src = os.path.join(ROOT, "sequence_depth_attention_moda_b200", "csrc", "moda_bwd_sm100.cu")
-    achieved = bwd_flops / (calls["bwd"] * 1e-3) / 1e12
-    roofline = {"kernel": "moda_bwd (rowdot + dkdv + dq launches of one call)", "bound": "tensor",
-                "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4),
+    # Roofline of the dominant kernel (largest mean duration).  Algorithmic
+    # FLOPs per kernel: the backward's five matmuls over [seq | depth] keys
+    # (2.5x the forward) split as dkdv = S^T, dP^T, dV, dK over the sequence
+    # keys and dq = dQ over all keys plus S, dP, dK, dV over the depth keys;
+    # dq's recomputation of the sequence S and dP is not counted.
+    mm_seq = 2.0 * w.B * w.Hq * w.d * (w.T * (w.T + 1) / 2)
+    mm_dep = 2.0 * w.B * w.Hq * w.d * (w.T * w.L)
+    algo = {"fwd": w.fwd_flops(), "dkdv": 4 * mm_seq, "dq": (mm_seq + mm_dep) + 4 * mm_dep}
+    names = {"fwd": "moda_fwd_sm100_kernel", "dkdv": "dkdv_kernel", "dq": "dq_kernel"}
+    srcs = {"fwd": "moda_fwd_sm100.cu", "dkdv": "moda_bwd_sm100.cu", "dq": "moda_bwd_sm100.cu"}
+    dom = max(algo, key=lambda k: calls[k])
+
+    def roof(k):
+        ach = algo[k] / (calls[k] * 1e-3) / 1e12
+        src = os.path.join(ROOT, "sequence_depth_attention_moda_b200", "csrc", srcs[k])
+        return {"kernel": names[k], "bound": "tensor", "achieved": round(ach, 1),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(ach / peaks["bf16_tflops"], 4),
                 "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                "traffic": traffic_from_profile(kernel_src),
-                "per_call_ms": {k: round(v, 4) for k, v in calls.items()}}
-    fwd_ach = w.fwd_flops() / (calls["fwd"] * 1e-3) / 1e12
-    roofline_fwd = {"kernel": "moda_fwd_sm100_kernel", "bound": "tensor", "achieved": round(fwd_ach, 1),
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": round(fwd_ach / peaks["bf16_tflops"], 4)}
+                "traffic": traffic_from_profile(names[k], src),
+                "mean_ms": round(calls[k], 4), "algorithmic_flops": algo[k]}
+
+    roofline = roof(dom)
+    roofline["per_kernel_ms"] = {k: round(v, 4) for k, v in calls.items()}
+    roofline_others = {k: roof(k) for k in algo if k != dom}
     rep_bytes = 2 * 2 * w.B * w.Hk * w.T * w.L * w.d * 2
     rep_ach = rep_bytes / (calls["repack"] * 1e-3) / 1e9
     roofline_repack = {"kernel": "repack_vec16_kernel (x2)", "bound": "hbm", "achieved": round(rep_ach, 1),
@@ -386,7 +423,8 @@ def run_ours(args):
                        "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (%.0f MB read per step)" %
                              (sum(t.numel() * t.element_size() for t in x.values()) / 1e6)},
-            "roofline": roofline, "roofline_fwd": roofline_fwd, "roofline_repack": roofline_repack,
+            "roofline": roofline, "roofline_other_kernels": roofline_others,
+            "roofline_repack": roofline_repack,
             "gpu_launches": r.launches_per_step() * args.steps,
             "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu, **extra,
         }

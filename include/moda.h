@@ -174,6 +174,19 @@ moda_status moda_bwd_noalloc(const moda_shape* shape,
                              moda_stream_t stream);
 
 /*
+ * Optional timing markers (observability; the pages have no counterpart).
+ * After this call, every moda_fwd and moda_bwd call made by the calling
+ * thread records events[0] on its stream before its first kernel launch and
+ * events[k] right after its k-th launch: moda_fwd has one launch; moda_bwd
+ * has three (row dots D = rowsum(dO*O), the dK/dV kernel, the dQ + depth-
+ * gradient kernel), so it uses events[0..3].  Markers beyond n are skipped.
+ *   events   array of n cudaEvent_t handles, created and owned by the caller
+ *   n        0..8; 0 turns the markers off
+ * Nothing is allocated; the library keeps only the handles (thread-local).
+ */
+moda_status moda_set_phase_events(void* const* events, int n);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's kernel
  * status word.  MODA_ERR_TIMEOUT if a kernel's bounded wait ran out since the
  * last check, MODA_ERR_CUDA if the stream reports an error, else MODA_OK.

@@ -6,10 +6,10 @@ and ``ops`` offers tensor-allocating conveniences over the same entry points.
 """
 from ._binding import (EXPORTED, LIB_PATH, MODA_BF16, MODA_DEPTH_CHUNKED, MODA_DEPTH_FLAT,
                        MODA_FP32, MoDAError, load, make_shape, moda_bwd, moda_bwd_noalloc,
-                       moda_check_status, moda_fwd, moda_last_error_message, moda_repack_depth, moda_shape,
-                       moda_status_string, moda_version, moda_workspace_size)
+                       moda_check_status, moda_fwd, moda_last_error_message, moda_repack_depth, moda_set_phase_events,
+                       moda_shape, moda_status_string, moda_version, moda_workspace_size)
 
 __all__ = ["EXPORTED", "LIB_PATH", "MODA_BF16", "MODA_DEPTH_CHUNKED", "MODA_DEPTH_FLAT",
            "MODA_FP32", "MoDAError", "load", "make_shape", "moda_bwd", "moda_bwd_noalloc", "moda_check_status",
-           "moda_fwd", "moda_last_error_message", "moda_repack_depth", "moda_shape",
+           "moda_fwd", "moda_last_error_message", "moda_repack_depth", "moda_set_phase_events", "moda_shape",
            "moda_status_string", "moda_version", "moda_workspace_size"]

@@ -30,7 +30,7 @@ MODA_DEPTH_CHUNKED = 1
 
 # Every symbol include/moda.h declares.
 EXPORTED = ("moda_workspace_size", "moda_repack_depth", "moda_fwd", "moda_bwd",
-            "moda_bwd_noalloc", "moda_check_status", "moda_status_string", "moda_last_error_message", "moda_version")
+            "moda_bwd_noalloc", "moda_set_phase_events", "moda_check_status", "moda_status_string", "moda_last_error_message", "moda_version")
 
 
 class moda_shape(ctypes.Structure):
@@ -75,6 +75,8 @@ def load(path: Optional[str] = None):
         lib.moda_bwd.restype = i
         lib.moda_bwd_noalloc.argtypes = [sp] + [vp] * 13 + [vp]
         lib.moda_bwd_noalloc.restype = i
+        lib.moda_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
+        lib.moda_set_phase_events.restype = i
         lib.moda_check_status.argtypes = [vp]
         lib.moda_check_status.restype = i
         lib.moda_status_string.argtypes = [i]
@@ -157,6 +159,15 @@ def moda_bwd_noalloc(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV,
                                    _ptr(Vd), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK),
                                    _ptr(dV), _ptr(dKd), _ptr(dVd), _stream(stream)),
            "moda_bwd_noalloc")
+
+
+def moda_set_phase_events(events) -> None:
+    """Timing markers: `events` is a list of torch.cuda.Event (or raw
+    cudaEvent_t ints) the following moda_fwd / moda_bwd calls of this thread
+    record between their kernel launches; [] turns them off."""
+    handles = [e if isinstance(e, int) else e.cuda_event for e in events]
+    arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
+    _check(load().moda_set_phase_events(arr, len(handles)), "moda_set_phase_events")
 
 
 def moda_check_status(stream=None):

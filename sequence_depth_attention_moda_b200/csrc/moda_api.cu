@@ -23,6 +23,10 @@ int g_sm_count[kMaxDevices] = {};
 
 thread_local std::string g_last_error;
 
+constexpr int kMaxPhaseEvents = 8;
+thread_local cudaEvent_t g_phase_events[kMaxPhaseEvents] = {};
+thread_local int g_n_phase_events = 0;
+
 moda_status fail(moda_status s, const char* fmt, ...) {
     char buf[512];
     va_list ap;
@@ -124,6 +128,10 @@ int device_sm_count() {
     return g_sm_count[dev];
 }
 
+void phase_mark(int k, cudaStream_t stream) {
+    if (k >= 0 && k < g_n_phase_events && g_phase_events[k]) cudaEventRecord(g_phase_events[k], stream);
+}
+
 // Hooks for entry points that live in other files of the library.
 moda_status api_validate(const moda_shape* shape, Problem* p) { return validate(shape, p); }
 moda_status api_fail(moda_status s, const char* msg) { return fail(s, "%s", msg); }
@@ -167,9 +175,11 @@ moda_status moda_fwd(const moda_shape* shape, const void* Q, const void* K, cons
     if (p.L > 0 && (st = check_ptrs({{Kd, "Kd"}, {Vd, "Vd"}})) != MODA_OK) return st;
     if (!device_status_word()) return fail(MODA_ERR_CUDA, "no usable CUDA device");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    phase_mark(0, s);
     cudaError_t e = p.elem_bytes == 2
                         ? launch_fwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, s)
                         : launch_fwd_simt(p, Q, K, V, Kd, Vd, O, LSE, s);
+    if (e == cudaSuccess) phase_mark(1, s);
     return e == cudaSuccess ? MODA_OK : cuda_fail(e, "forward launch");
 }
 
@@ -195,6 +205,7 @@ moda_status moda_bwd(const moda_shape* shape, const void* Q, const void* K, cons
     if (!device_status_word()) return fail(MODA_ERR_CUDA, "no usable CUDA device");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* Dws = static_cast<float*>(ws);
+    phase_mark(0, s);
     cudaError_t e =
         p.elem_bytes == 2
             ? launch_bwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, s)
@@ -233,6 +244,15 @@ const char* moda_status_string(moda_status status) {
 }
 
 const char* moda_last_error_message(void) { return g_last_error.c_str(); }
+
+moda_status moda_set_phase_events(void* const* events, int n) {
+    if (n < 0 || n > kMaxPhaseEvents) return fail(MODA_ERR_INVALID_ARG, "n=%d must be 0..%d", n, kMaxPhaseEvents);
+    if (n > 0 && !events) return fail(MODA_ERR_INVALID_ARG, "events is NULL");
+    for (int i = 0; i < kMaxPhaseEvents; ++i)
+        g_phase_events[i] = i < n ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+    g_n_phase_events = n;
+    return MODA_OK;
+}
 
 int moda_version(void) { return 100; }
 

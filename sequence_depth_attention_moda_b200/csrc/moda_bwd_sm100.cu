@@ -775,6 +775,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     rowdot_kernel<D><<<(unsigned)((nrows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(
         nrows, static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), Dws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    phase_mark(1, stream);
 
     // 2. dK, dV
     DkdvArgs A;
@@ -798,6 +799,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
         const long long grid = (long long)p.B * p.Hk * A.n_kt;
         dkdv_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(A);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        phase_mark(2, stream);
     }
 
     // 3. dQ, dKd, dVd
@@ -834,6 +836,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
         const long long grid = (long long)p.B * p.Hk * B.n_qt;
         dq_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(B);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        phase_mark(3, stream);
     }
     return cudaSuccess;
 }

@@ -27,6 +27,10 @@ unsigned int* device_status_word();
 // SM count of the current device (cached).
 int device_sm_count();
 
+// Records the calling thread's k-th phase marker on `stream`, if one is set
+// (see moda_set_phase_events); a no-op otherwise.
+void phase_mark(int k, cudaStream_t stream);
+
 // ---- depth repack (moda_repack.cu) -----------------------------------------
 cudaError_t launch_repack(int B, int Hk, int T, int d, int L, int elem_bytes,
                           const void* src, void* dst, cudaStream_t stream);

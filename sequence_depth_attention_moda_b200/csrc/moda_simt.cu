@@ -275,17 +275,20 @@ cudaError_t bwd_impl(const Problem& p, const void* Q, const void* K, const void*
     const long long rows = (long long)p.B * p.Hq * p.T;
     bwd_rowdot_kernel<T><<<blocks_for(rows), kWarps * 32, 0, s>>>(rows, p.d, (const T*)O,
                                                                   (const T*)dO, D);
+    phase_mark(1, s);
     bwd_dq_simt_kernel<T><<<blocks_for(rows), kWarps * 32, 0, s>>>(
         p, (const T*)Q, (const T*)K, (const T*)V, (const T*)Kd, (const T*)Vd, LSE, (const T*)dO,
         D, (T*)dQ);
     const long long krows = (long long)p.B * p.Hk * p.T;
     bwd_dkdv_simt_kernel<T><<<blocks_for(krows), kWarps * 32, 0, s>>>(
         p, (const T*)Q, (const T*)K, (const T*)V, LSE, (const T*)dO, D, (T*)dK, (T*)dV);
+    phase_mark(2, s);
     if (p.L > 0) {
         const long long drows = krows * p.L;
         bwd_ddepth_simt_kernel<T><<<blocks_for(drows), kWarps * 32, 0, s>>>(
             p, (const T*)Q, (const T*)Kd, (const T*)Vd, LSE, (const T*)dO, D, (T*)dKd, (T*)dVd);
     }
+    phase_mark(3, s);
     return cudaGetLastError();
 }
 

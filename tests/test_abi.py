@@ -108,3 +108,12 @@ def test_empty_problems_are_noops(lib):
         sh = moda.make_shape(**base)
         assert call_fwd(lib, sh, [None] * 7) == 0
         assert lib.moda_repack_depth(ctypes.byref(sh), None, None, None) == 0
+
+
+def test_phase_events_validation(lib):
+    # n outside 0..8 or a NULL array with n > 0 is rejected; n = 0 turns them off
+    assert lib.moda_set_phase_events(None, 0) == 0
+    assert lib.moda_set_phase_events(None, 2) == 1
+    arr = (ctypes.c_void_p * 9)()
+    assert lib.moda_set_phase_events(arr, 9) == 1
+    assert lib.moda_set_phase_events(arr, 0) == 0
