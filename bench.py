@@ -129,13 +129,12 @@ def traffic_from_profile(kernel: str, kernel_src: str):
     path = os.path.join(ROOT, "profiles", "dram_traffic_layer_T4k.md")
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    m_hash = re.search(r"source sha256: ([0-9a-f]{16})", text)
-    m_bytes = re.search(r"^\| %s \| (\d+) \|" % re.escape(kernel), text, re.M)
-    if not m_hash or not m_bytes:
+    m = re.search(r"^\| %s \| (\d+) \| [^|]+ \| ([0-9a-f]{16}) \|" % re.escape(kernel),
+                  open(path).read(), re.M)
+    if not m:
         return None
     cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
-    return int(m_bytes.group(1)) if cur == m_hash.group(1) else None
+    return int(m.group(1)) if cur == m.group(2) else None
 
 
 # --------------------------------------------------------------- our arm ----
