@@ -20,13 +20,19 @@
 //               done, a V stage only when O += P_i V_i is, so the next K
 //               tiles stream in while PV still holds older V tiles.
 //   warp 1      TMEM allocator and MMA issuer (one thread):
-//               S_i = Q K_i^T into one of two TMEM S buffers, then
-//               O += P_{i-1} V_{i-1} with P read from TMEM.
+//               S_i = Q K_i^T into one of three TMEM S buffers, and
+//               O += P_i V_i with P read from TMEM; S_{i+2} is issued
+//               before PV_i, so two score tiles are always ahead of the
+//               softmax and the tensor pipe's issue-to-completion latency
+//               (hundreds of cycles) is off the softmax's critical path.
 //   warps 2..5  softmax, one thread per tile row: tcgen05.ld of S, masks,
 //               running max, exp2, row sum, P (bf16) written back over S with
 //               tcgen05.st; O in TMEM is rescaled only when the running max
 //               grew by more than 2^8 (exact: the final o / acc cancels it).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d).
+// TMEM columns: S0 [0,128), S1 [128,256), S2 [256,384), O [384, 384+d).
+// Softmax: row max as four partial maxima; exp2 on the MUFU unit (a build
+// knob moves a share of column pairs to ex2_fma on the FMA pipe; measured
+// slower here, so off).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -54,7 +60,27 @@ constexpr int kSoftmaxThreads = 128;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kSlabBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
+constexpr int kSBufs = 3;            // S / P buffers in TMEM
+constexpr uint32_t kColO = 384;      // O accumulator after the three S buffers
+#ifndef MODA_FWD_SWEXP
+#define MODA_FWD_SWEXP 0             // of every 4 column pairs, this many use ex2_fma
+#endif
+
+// Optional hand-off timeline of CTA 0 (clock64 per event and block), only in
+// builds with -DMODA_TRACE; read back with moda_trace_copy_fwd().
+#ifdef MODA_TRACE
+constexpr int kTraceSlots = 16, kTraceIters = 96;
+__device__ long long g_trace_fwd[kTraceSlots * kTraceIters];
+#define MODA_TRF(slot, it)                                                  \
+    do {                                                                    \
+        if (blockIdx.x == 0 && (it) >= 0 && (it) < kTraceIters)             \
+            g_trace_fwd[(slot) * kTraceIters + (it)] = clock64();           \
+    } while (0)
+#else
+#define MODA_TRF(slot, it) \
+    do {                   \
+    } while (0)
+#endif
 
 struct FwdArgs {
     TmaMap tq, tk, tv, tkd, tvd;
@@ -80,9 +106,10 @@ struct Layout {
 };
 
 // Barrier slots.
-enum { kQFull = 0, kKFull = 1, kKEmpty = kKFull + kKStages, kVFull = kKEmpty + kKStages,
-       kVEmpty = kVFull + kVStages, kSFull = kVEmpty + kVStages, kPReady = kSFull + 2,
-       kOReady = kPReady + 2, kOFinal = kOReady + 1, kNumBars = kOFinal + 1 };
+enum { kQFull = 0, kKFull = 1, kVFull = kKFull + kKStages, kVEmpty = kVFull + kVStages,
+       kSFull = kVEmpty + kVStages, kPReady = kSFull + kSBufs, kOFinal = kPReady + kSBufs,
+       kNumBars = kOFinal + 1 };
+static_assert(kKStages == kSBufs, "a K stage is released by the score barrier of its S buffer");
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __grid_constant__ FwdArgs a) {
@@ -115,19 +142,15 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kQFull], 1);
-        for (int s = 0; s < kKStages; ++s) {
-            mbar_init(&bars[kKFull + s], 1);
-            mbar_init(&bars[kKEmpty + s], 1);
-        }
+        for (int s = 0; s < kKStages; ++s) mbar_init(&bars[kKFull + s], 1);
         for (int s = 0; s < kVStages; ++s) {
             mbar_init(&bars[kVFull + s], 1);
             mbar_init(&bars[kVEmpty + s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kSBufs; ++s) {
             mbar_init(&bars[kSFull + s], 1);
             mbar_init(&bars[kPReady + s], kSoftmaxThreads);
         }
-        mbar_init(&bars[kOReady], 1);
         mbar_init(&bars[kOFinal], 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -158,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             const bool is_k = warp == 0;
             const int nst = is_k ? kKStages : kVStages;
             uint64_t* full = &bars[is_k ? kKFull : kVFull];
-            uint64_t* empty = &bars[is_k ? kKEmpty : kVEmpty];
+            uint64_t* empty = &bars[is_k ? kSFull : kVEmpty];
             unsigned char* ring = is_k ? sK : sV;
             const void* m_seq = is_k ? static_cast<const void*>(&a.tk) : static_cast<const void*>(&a.tv);
             const void* m_dep = is_k ? static_cast<const void*>(&a.tkd) : static_cast<const void*>(&a.tvd);
@@ -174,6 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             int issued = 0;
             for (int i = 0; i < nb; ++i) {
                 const int st = i % nst;
+                // K stage of block i-nst is free once S(i-nst) is done: that is
+                // the score barrier of its buffer (three K stages, three S
+                // buffers), so no separate commit is needed for K.
                 if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1, a.status, abort_flag))
                     break;
                 unsigned char* dst = ring + st * Lay::kTile;
@@ -198,10 +224,33 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             const uint32_t id_pv = idesc_bf16(128, D, false, true);
             const uint32_t q_addr = smem_u32(sQ);
             bool ok = mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
+            // S(j) = Q K_j^T into buffer j % 3.  The buffer last held P(j-3),
+            // read by PV(j-3), which is issued before S(j) (in-order pipe).
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % kKStages;
+                const int sb = j % kSBufs;
+                MODA_TRF(0, j);
+                if (!mbar_wait(&bars[kKFull + st], (j / kKStages) & 1, a.status, abort_flag)) return false;
+                MODA_TRF(1, j);
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(sK + st * Lay::kTile);
+                const uint32_t id = j < n_seq ? id_seq : id_dep;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+                    umma_ss(tmem + sb * 128, desc_kmajor_sw128(q_addr + off),
+                            desc_kmajor_sw128(k_addr + off), id, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[kSFull + sb]);
+                MODA_TRF(2, j);
+                return true;
+            };
+            // O += P(j) V_j with P read from TMEM buffer j % 3.
             auto issue_pv = [&](int j) -> bool {
                 const int st = j % kVStages;
-                const int sb = j & 1;
-                if (!mbar_wait(&bars[kPReady + sb], (j >> 1) & 1, a.status, abort_flag)) return false;
+                const int sb = j % kSBufs;
+                if (!mbar_wait(&bars[kPReady + sb], (j / kSBufs) & 1, a.status, abort_flag)) return false;
+                MODA_TRF(4, j);
                 if (!mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status, abort_flag)) return false;
                 tc_fence_after();
                 const int krows = j < n_seq ? BN : a.dep_rows;
@@ -211,27 +260,20 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, bdesc, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&bars[kVEmpty + st]);
-                umma_commit(&bars[kOReady]);
+                MODA_TRF(3, j);
                 return true;
             };
+            // Two score tiles run ahead of the softmax.  S(i+2) goes in
+            // before PV(i): its buffer held P(i-1), whose PV(i-1) is already
+            // in the (in-order) pipe, so it never waits for P(i); each issue
+            // blocks until the shallow MMA queue has room, so this order is
+            // what keeps the next scores ready when the softmax needs them.
+            if (ok) ok = issue_s(0);
+            if (ok && nb > 1) ok = issue_s(1);
             for (int i = 0; ok && i < nb; ++i) {
-                const int st = i % kKStages;
-                const int sb = i & 1;
-                if (!mbar_wait(&bars[kKFull + st], (i / kKStages) & 1, a.status, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(sK + st * Lay::kTile);
-                const uint32_t id = i < n_seq ? id_seq : id_dep;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    umma_ss(tmem + sb * 128, desc_kmajor_sw128(q_addr + off),
-                            desc_kmajor_sw128(k_addr + off), id, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&bars[kSFull + sb]);
-                umma_commit(&bars[kKEmpty + st]);
-                if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
+                if (i + 2 < nb && !issue_s(i + 2)) { ok = false; break; }
+                if (!issue_pv(i)) { ok = false; break; }
             }
-            if (ok) ok = issue_pv(nb - 1);
             umma_commit(&bars[kOFinal]);
         }
     } else if (warp >= 2 && warp <= 5) {
@@ -246,8 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         float m = -INFINITY, l = 0.0f;
         bool ok = true;
         for (int i = 0; i < nb; ++i) {
-            const int sb = i & 1;
-            if (!mbar_wait(&bars[kSFull + sb], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+            const int sb = i % kSBufs;
+            if (r == 0) MODA_TRF(5, i);
+            if (!mbar_wait(&bars[kSFull + sb], (i / kSBufs) & 1, a.status, abort_flag)) { ok = false; break; }
+            if (r == 0) MODA_TRF(6, i);
             tc_fence_after();
             uint32_t sr[128];
             const uint32_t s_addr = lane_base + sb * 128;
@@ -256,35 +300,40 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             tmem_ld32(s_addr + 64, sr + 64);
             tmem_ld32(s_addr + 96, sr + 96);
             tmem_wait_ld();
-            float mx = -INFINITY;
+            if (r == 0) MODA_TRF(7, i);
+            // masks, then the row max as four independent partial maxima
             if (i < n_seq) {
                 const int kb = i * BN;
-                if (kb + BN - 1 <= t_row) {
+                if (kb + BN - 1 > t_row) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c) {
+                    for (int c = 0; c < 128; ++c)
                         if (kb + c > t_row) sr[c] = __float_as_uint(-INFINITY);
-                        mx = fmaxf(mx, __uint_as_float(sr[c]));
-                    }
                 }
             } else {
                 const int lo = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows);
                 const int hi = min(lo + a.L, a.dep_rows);
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
+                for (int c = 0; c < 128; ++c)
                     if (c < lo || c >= hi) sr[c] = __float_as_uint(-INFINITY);
-                    mx = fmaxf(mx, __uint_as_float(sr[c]));
-                }
             }
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], __uint_as_float(sr[c + u]));
+            }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             const float m_new = fmaxf(m, mx * sl2);
+            if (r == 0) MODA_TRF(8, i);
             if (i == 0) {
                 m = m_new;
             } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
-                // O must hold P_{i-1} V_{i-1} before it is rescaled.  S_i was
-                // issued after PV_{i-2}, so at most PV_{i-1} is in flight.
-                if (!mbar_wait(&bars[kOReady], (i - 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                // O must hold P_{i-1} V_{i-1} before it is rescaled: wait for
+                // the V-stage release PV_{i-1} commits.  S_i was issued after
+                // PV_{i-2}, so at most PV_{i-1} is in flight, and PV_{i+2}
+                // (the stage's next use) needs P_{i+2}: the parity is exact.
+                if (!mbar_wait(&bars[kVEmpty + (i - 1) % kVStages], ((i - 1) / kVStages) & 1, a.status,
+                               abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const float alpha = ex2(m - m_new);
                 l *= alpha;
@@ -300,19 +349,31 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 }
                 tmem_wait_st();
             }
-            float rs = 0.0f;
+            if (r == 0) MODA_TRF(9, i);
+            float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             uint32_t pk[64];
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-                const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -m));
-                const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m));
-                rs += p0 + p1;
+                const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -m);
+                const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m);
+                float p0, p1;
+                if ((c & 3) < 4 - MODA_FWD_SWEXP) {     // MUFU
+                    p0 = ex2(x0);
+                    p1 = ex2(x1);
+                } else {                                 // FMA pipe
+                    p0 = ex2_fma(x0);
+                    p1 = ex2_fma(x1);
+                }
+                rs4[c & 3] += p0 + p1;
                 pk[c] = pack_bf16(p0, p1);
             }
+            const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
             l += rs;
+            if (r == 0) MODA_TRF(10, i);
             tmem_st32(s_addr, pk);
             tmem_st32(s_addr + 32, pk + 32);
             tmem_wait_st();
+            if (r == 0) MODA_TRF(11, i);
             tc_fence_before();
             mbar_arrive(&bars[kPReady + sb]);
         }
@@ -385,6 +446,13 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
 }
 
 }  // namespace
+
+#ifdef MODA_TRACE
+extern "C" int moda_trace_copy_fwd(long long* host, int n) {
+    const int cnt = n < kTraceSlots * kTraceIters ? n : kTraceSlots * kTraceIters;
+    return cudaMemcpyFromSymbol(host, g_trace_fwd, cnt * sizeof(long long)) == cudaSuccess ? cnt : -1;
+}
+#endif
 
 cudaError_t launch_fwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, void* O, float* LSE,
