@@ -222,8 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, kKvBQ, false, false);
             const uint32_t id_g = idesc_bf16(128, D, false, true);
-            const uint32_t k_addr = smem_u32(smem + Lay::kK);
-            const uint32_t v_addr = smem_u32(smem + Lay::kV);
+            const uint64_t kd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kK));
+            const uint64_t vd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kV));
             // S^T(j) = K Q_j^T and dP^T(j) = V dO_j^T into buffer j & 1.
             auto issue_s = [&](int j) -> bool {
                 const int st = j % kKvStages;
@@ -231,21 +231,19 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 if (!mbar_wait(&bars[kA_QFull + st], (j / kKvStages) & 1, a.status, abort_flag)) return false;
                 MODA_TR(10, j);
                 tc_fence_after();
-                const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kQTile);
-                const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kQTile);
+                const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
+                const uint64_t dd = desc_kmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t offk = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    const uint32_t offq = (kk >> 2) * kKvSlab + (kk & 3) * 32;
-                    umma_ss(tmem + buf * 64, desc_kmajor_sw128(k_addr + offk),
-                            desc_kmajor_sw128(q_addr + offq), id_s, kk > 0 ? 1u : 0u);
+                    const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                    const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t offk = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    const uint32_t offq = (kk >> 2) * kKvSlab + (kk & 3) * 32;
-                    umma_ss(tmem + 128 + buf * 64, desc_kmajor_sw128(v_addr + offk),
-                            desc_kmajor_sw128(do_addr + offq), id_s, kk > 0 ? 1u : 0u);
+                    const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                    const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[kA_SFull + buf]);
                 return true;
@@ -260,15 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 if (!mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
                 MODA_TR(2, it);
                 tc_fence_after();
-                const uint32_t q_addr = smem_u32(smem + Lay::kQ + st * Lay::kQTile);
-                const uint32_t do_addr = smem_u32(smem + Lay::kDO + st * Lay::kQTile);
+                const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
+                const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
 #pragma unroll
                 for (int kk = 0; kk < kKvBQ / 16; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts(tmem + 256, tmem + buf * 64 + kk * 8,
-                            desc_mnmajor_sw128(do_addr + kk * 2048, kKvSlab), id_g, acc);
-                    umma_ts(tmem + 384, tmem + 128 + buf * 64 + kk * 8,
-                            desc_mnmajor_sw128(q_addr + kk * 2048, kKvSlab), id_g, acc);
+                    umma_ts(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, acc);
+                    umma_ts(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g, acc);
                 }
                 umma_commit(&bars[kA_QEmpty + st]);
                 MODA_TR(3, it);
@@ -532,6 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             const uint32_t do_addr = smem_u32(smem + Lay::kDO);
             const uint32_t ds_addr = smem_u32(smem + Lay::kDS);
             const uint32_t p_addr = smem_u32(smem + Lay::kP);
+            const uint64_t qd0 = desc_kmajor_sw128(q_addr);
+            const uint64_t dod0 = desc_kmajor_sw128(do_addr);
             // S(j) = Q K_j^T and dP(j) = dO V_j^T into buffer j & 1.
             auto issue_s = [&](int j) -> bool {
                 const int st = j % kDqStages;
@@ -540,21 +538,19 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 MODA_TRQ(8, j);
                 tc_fence_after();
                 const uint32_t id = j < n_seq ? id_seq : id_dep;
-                const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kKTile);
-                const uint32_t v_addr = smem_u32(smem + Lay::kV + st * Lay::kKTile);
+                const uint64_t kd = desc_kmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile));
+                const uint64_t vd = desc_kmajor_sw128(smem_u32(smem + Lay::kV + st * Lay::kKTile));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t offq = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    const uint32_t offk = (kk >> 2) * kDqSlab + (kk & 3) * 32;
-                    umma_ss(tmem + kColS + buf * 64, desc_kmajor_sw128(q_addr + offq),
-                            desc_kmajor_sw128(k_addr + offk), id, kk > 0 ? 1u : 0u);
+                    const uint64_t offq = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                    const uint64_t offk = ((kk >> 2) * kDqSlab + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + kColS + buf * 64, qd0 + offq, kd + offk, id, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t offq = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    const uint32_t offk = (kk >> 2) * kDqSlab + (kk & 3) * 32;
-                    umma_ss(tmem + kColDP + buf * 64, desc_kmajor_sw128(do_addr + offq),
-                            desc_kmajor_sw128(v_addr + offk), id, kk > 0 ? 1u : 0u);
+                    const uint64_t offq = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                    const uint64_t offk = ((kk >> 2) * kDqSlab + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + kColDP + buf * 64, dod0 + offq, vd + offk, id, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[kB_SFull + buf]);
                 return true;
@@ -573,11 +569,17 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 if (!mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
                 MODA_TRQ(2, i);
                 tc_fence_after();
-                const uint32_t k_addr = smem_u32(smem + Lay::kK + st * Lay::kKTile);
-                for (int kk = 0; kk < n / 16; ++kk)
-                    umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8,
-                            desc_mnmajor_sw128(k_addr + kk * 2048, kDqSlab), id_dq,
-                            (i > 0 || kk > 0) ? 1u : 0u);
+                const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
+                if (n == kDqBN) {
+#pragma unroll
+                    for (int kk = 0; kk < kDqBN / 16; ++kk)
+                        umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
+                                (i > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    for (int kk = 0; kk < n / 16; ++kk)
+                        umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
+                                (i > 0 || kk > 0) ? 1u : 0u);
+                }
                 if (!seq) {
 #pragma unroll
                     for (int kk = 0; kk < BM / 16; ++kk) {

@@ -30,7 +30,7 @@
 //               tcgen05.st; O in TMEM is rescaled only when the running max
 //               grew by more than 2^8 (exact: the final o / acc cancels it).
 // TMEM columns: S0 [0,128), S1 [128,256), S2 [256,384), O [384, 384+d).
-// Softmax: row max as four partial maxima; exp2 on the MUFU unit (a build
+// Softmax: row max as four partial maxima of three-input max; exp2 on the MUFU unit (a build
 // knob moves a share of column pairs to ex2_fma on the FMA pipe; measured
 // slower here, so off).
 #include <cuda_bf16.h>
@@ -222,7 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             const uint32_t id_seq = idesc_bf16(128, BN, false, false);
             const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
             const uint32_t id_pv = idesc_bf16(128, D, false, true);
-            const uint32_t q_addr = smem_u32(sQ);
+            // Descriptors are built once; a K step adds its byte offset / 16
+            // to the 14-bit address field (shared addresses stay < 256 KB).
+            const uint64_t qd0 = desc_kmajor_sw128(smem_u32(sQ));
             bool ok = mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
             // S(j) = Q K_j^T into buffer j % 3.  The buffer last held P(j-3),
             // read by PV(j-3), which is issued before S(j) (in-order pipe).
@@ -233,13 +235,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 if (!mbar_wait(&bars[kKFull + st], (j / kKStages) & 1, a.status, abort_flag)) return false;
                 MODA_TRF(1, j);
                 tc_fence_after();
-                const uint32_t k_addr = smem_u32(sK + st * Lay::kTile);
+                const uint64_t kd0 = desc_kmajor_sw128(smem_u32(sK + st * Lay::kTile));
                 const uint32_t id = j < n_seq ? id_seq : id_dep;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-                    umma_ss(tmem + sb * 128, desc_kmajor_sw128(q_addr + off),
-                            desc_kmajor_sw128(k_addr + off), id, kk > 0 ? 1u : 0u);
+                    const uint64_t off = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + sb * 128, qd0 + off, kd0 + off, id, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[kSFull + sb]);
                 MODA_TRF(2, j);
@@ -254,10 +255,16 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 if (!mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status, abort_flag)) return false;
                 tc_fence_after();
                 const int krows = j < n_seq ? BN : a.dep_rows;
-                const uint32_t v_addr = smem_u32(sV + st * Lay::kTile);
-                for (int kk = 0; kk < krows / 16; ++kk) {
-                    const uint64_t bdesc = desc_mnmajor_sw128(v_addr + kk * 2048, kSlabBytes);
-                    umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, bdesc, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                const uint64_t vd0 = desc_mnmajor_sw128(smem_u32(sV + st * Lay::kTile), kSlabBytes);
+                if (krows == BN) {
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    for (int kk = 0; kk < krows / 16; ++kk)
+                        umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
+                                (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&bars[kVEmpty + st]);
                 MODA_TRF(3, j);
@@ -318,9 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             }
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 128; c += 4) {
+            for (int c = 0; c < 128; c += 8) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], __uint_as_float(sr[c + u]));
+                for (int u = 0; u < 4; ++u)
+                    mx4[u] = fmax3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
             }
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             const float m_new = fmaxf(m, mx * sl2);
