@@ -64,8 +64,12 @@ def load_library(path: str | None = None):
         i, d = ctypes.c_int, ctypes.c_double
         lib.moda_oracle_fwd.argtypes = [i, i, i, i, i, i, d] + [_dp] * 7
         lib.moda_oracle_fwd.restype = i
+        lib.moda_oracle_fwd_ex.argtypes = [i, i, i, i, i, i, d, i, i] + [_dp] * 7
+        lib.moda_oracle_fwd_ex.restype = i
         lib.moda_oracle_bwd.argtypes = [i, i, i, i, i, i, d] + [_dp] * 11
         lib.moda_oracle_bwd.restype = i
+        lib.moda_oracle_bwd_ex.argtypes = [i, i, i, i, i, i, d, i, i] + [_dp] * 11
+        lib.moda_oracle_bwd_ex.restype = i
         lib.moda_oracle_row.argtypes = [i, i, i, d] + [_dp] * 8
         lib.moda_oracle_row.restype = None
         lib.moda_oracle_repack.argtypes = [i, i, i, i, i, i, ctypes.c_void_p, ctypes.c_void_p]
@@ -104,11 +108,14 @@ def threads(lib=None) -> int:
     return int((lib or load_library()).moda_oracle_threads())
 
 
-def fwd(Q, K, V, Kd=None, Vd=None, scale: float = 0.0, lib=None):
+def fwd(Q, K, V, Kd=None, Vd=None, scale: float = 0.0, lib=None, causal: bool = True,
+        window: int = 0):
     """Forward: returns (O [B,Hq,T,d], LSE [B,Hq,T]) in float64.
 
     Kd/Vd are the token-major depth tensors [B,Hk,T*L,d]; pass None (or
-    empty arrays) for L = 0.  scale <= 0 selects 1/sqrt(d).
+    empty arrays) for L = 0.  scale <= 0 selects 1/sqrt(d).  causal=False
+    drops the sequence mask; window > 0 keeps each token's last `window`
+    depth rows only.
     """
     lib = lib or load_library()
     Q, K, V = _f64(Q), _f64(K), _f64(V)
@@ -117,15 +124,15 @@ def fwd(Q, K, V, Kd=None, Vd=None, scale: float = 0.0, lib=None):
     B, Hq, Hk, T, d, L = _shape(Q, K, Kd)
     O = np.zeros((B, Hq, T, d))
     LSE = np.zeros((B, Hq, T))
-    rc = lib.moda_oracle_fwd(B, Hq, Hk, T, d, L, float(scale), _ptr(Q), _ptr(K), _ptr(V),
-                             _ptr(Kd), _ptr(Vd), _ptr(O), _ptr(LSE))
+    rc = lib.moda_oracle_fwd_ex(B, Hq, Hk, T, d, L, float(scale), int(bool(causal)), int(window),
+                                _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd), _ptr(O), _ptr(LSE))
     if rc != 0:
         raise ValueError("oracle rejected the shape")
     return O, LSE
 
 
-def bwd(Q, K, V, Kd, Vd, dO, scale: float = 0.0, lib=None):
-    """Backward: returns (dQ, dK, dV, dKd, dVd) in float64."""
+def bwd(Q, K, V, Kd, Vd, dO, scale: float = 0.0, lib=None, causal: bool = True, window: int = 0):
+    """Backward: returns (dQ, dK, dV, dKd, dVd) in float64 (same options as fwd)."""
     lib = lib or load_library()
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
     Kd = None if Kd is None or np.size(Kd) == 0 else _f64(Kd)
@@ -136,33 +143,35 @@ def bwd(Q, K, V, Kd, Vd, dO, scale: float = 0.0, lib=None):
     dV = np.zeros_like(V)
     dKd = np.zeros((B, Hk, T * L, d))
     dVd = np.zeros((B, Hk, T * L, d))
-    rc = lib.moda_oracle_bwd(B, Hq, Hk, T, d, L, float(scale), _ptr(Q), _ptr(K), _ptr(V),
-                             _ptr(Kd), _ptr(Vd), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV),
-                             _ptr(dKd if L else None), _ptr(dVd if L else None))
+    rc = lib.moda_oracle_bwd_ex(B, Hq, Hk, T, d, L, float(scale), int(bool(causal)), int(window),
+                                _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd), _ptr(dO), _ptr(dQ),
+                                _ptr(dK), _ptr(dV), _ptr(dKd if L else None),
+                                _ptr(dVd if L else None))
     if rc != 0:
         raise ValueError("oracle rejected the shape")
     return dQ, dK, dV, dKd, dVd
 
 
 def row(q, Kseq, Vseq, Kdep, Vdep, scale: float = 0.0, lib=None, return_p: bool = False):
-    """One query row at token t = len(Kseq) - 1.
+    """One query row: one softmax over exactly the given visible rows.
 
-    q [d]; Kseq/Vseq [t+1, d] (the KV head's rows 0..t); Kdep/Vdep [L, d]
-    (token t's depth rows).  Returns (o [d], lse) or (o, lse, p) where p is
-    the normalised [seq | depth] weight row.
+    q [d]; Kseq/Vseq [n_seq, d] (for the causal operator at token t, the KV
+    head's rows 0..t); Kdep/Vdep [n_dep, d] (token t's visible depth rows).
+    Returns (o [d], lse) or (o, lse, p) where p is the normalised
+    [seq | depth] weight row.
     """
     lib = lib or load_library()
     q, Kseq, Vseq = _f64(q), _f64(Kseq), _f64(Vseq)
     Kdep, Vdep = _f64(Kdep), _f64(Vdep)
     d = q.shape[-1]
-    t = Kseq.shape[0] - 1
+    n_seq = Kseq.shape[0]
     L = Kdep.shape[0]
     if scale <= 0:
         scale = 1.0 / np.sqrt(d)
     o = np.zeros(d)
     lse = np.zeros(1)
-    p = np.zeros(t + 1 + L) if return_p else None
-    lib.moda_oracle_row(t, d, L, float(scale), _ptr(q), _ptr(Kseq), _ptr(Vseq),
+    p = np.zeros(n_seq + L) if return_p else None
+    lib.moda_oracle_row(n_seq, L, d, float(scale), _ptr(q), _ptr(Kseq), _ptr(Vseq),
                         _ptr(Kdep if L else None), _ptr(Vdep if L else None),
                         _ptr(o), _ptr(lse), _ptr(p))
     return (o, float(lse[0]), p) if return_p else (o, float(lse[0]))

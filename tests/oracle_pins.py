@@ -19,7 +19,12 @@ Sources (page title, section):
 * "moda-attention 0.1.0" PyPI page, "Key Design Choices" -- GQA expansion by
   repeat_interleave; "Using the Kernel Directly" -- tensor layouts;
 * paper summary, "Hardware-Efficient Implementation" -- token t's L depth rows
-  sit at [t*L, (t+1)*L) of the flattened depth tensor.
+  sit at [t*L, (t+1)*L) of the flattened depth tensor;
+* ByteDance-Seed/MoDA README, "TODO" (non-causal MoDA kernel) and paper
+  summary, "7. Implications and Future Directions" (vision use) -- the
+  non-causal operator drops the sequence mask and keeps the depth mask;
+* paper summary, "6. Limitations and Trade-offs" (bounded depth-KV slots,
+  sliding-window recency) -- a depth window keeps each token's last S layers.
 """
 from __future__ import annotations
 
@@ -47,9 +52,11 @@ def rand_case(B, Hq, Hk, T, d, L, seed, dtype=torch.float64):
 
 
 # ------------------------------------------ independent dense formulation ----
-def dense_moda(Q, K, V, Kd, Vd, scale=None):
+def dense_moda(Q, K, V, Kd, Vd, scale=None, causal=True, window=0):
     """The 'naive' dense form: concatenate [K | K_depth], build the full mask
     matrix M in the flattened row index i_q = t*G + g, one softmax per row.
+    causal=False drops the sequence mask; window > 0 keeps depth column j_d
+    only if its layer j_d mod L is among the token's last `window` layers.
     Pure torch library ops (differentiable), fp64."""
     B, Hq, T, d = Q.shape
     Hk = K.shape[1]
@@ -61,7 +68,12 @@ def dense_moda(Q, K, V, Kd, Vd, scale=None):
     i_q = torch.arange(T * G)
     t_base = i_q // G
     seq_mask = t_base[:, None] >= torch.arange(T)[None, :]
-    dep_mask = t_base[:, None] == (torch.arange(T * L) // max(L, 1))[None, :]
+    if not causal:
+        seq_mask = torch.ones_like(seq_mask)
+    j_d = torch.arange(T * L)
+    dep_mask = t_base[:, None] == (j_d // max(L, 1))[None, :]
+    if window:
+        dep_mask &= ((j_d % max(L, 1)) >= L - window)[None, :]
     M = torch.cat([seq_mask, dep_mask], dim=1)
     Kc = torch.cat([K, Kd], dim=2)
     Vc = torch.cat([V, Vd], dim=2)
@@ -328,7 +340,64 @@ def pin_repack_definition(lib):
     assert out.dtype == src.dtype and np.array_equal(out, ref), "repack permutation"
 
 
+def pin_noncausal_l0_is_sdpa(lib):
+    """Non-causal with L = 0 is plain softmax attention over all T keys
+    (library SDPA without the causal mask, repeat_interleaved K/V)."""
+    for (B, Hq, Hk, T, d, seed) in ((1, 4, 2, 11, 16, 101), (2, 3, 3, 6, 8, 102)):
+        Q, K, V, _, _, _ = rand_case(B, Hq, Hk, T, d, 0, seed)
+        O, LSE = oracle.fwd(Q, K, V, None, None, lib=lib, causal=False)
+        G = Hq // Hk
+        Ke, Ve = K.repeat_interleave(G, dim=1), V.repeat_interleave(G, dim=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, Ke, Ve)
+        lse = torch.logsumexp((Q @ Ke.transpose(-1, -2)) / math.sqrt(d), -1)
+        _close(O, ref.numpy(), 1e-12, "non-causal O vs SDPA")
+        _close(LSE, lse.numpy(), 1e-12, "non-causal LSE")
+
+
+def pin_modes_dense_bruteforce(lib):
+    """Non-causal and depth-window forward against the dense formulation."""
+    for (causal, window, seed) in ((False, 0, 111), (True, 2, 112), (False, 3, 113), (True, 4, 114)):
+        Q, K, V, Kd, Vd, _ = rand_case(1, 4, 2, 9, 8, 4, seed)
+        O, LSE = oracle.fwd(Q, K, V, Kd, Vd, lib=lib, causal=causal, window=window)
+        Or, LSEr = dense_moda(Q, K, V, Kd, Vd, causal=causal, window=window)
+        _close(O, Or.numpy(), 1e-12, f"O causal={causal} window={window}")
+        _close(LSE, LSEr.numpy(), 1e-12, f"LSE causal={causal} window={window}")
+
+
+def pin_window_is_truncated_depth(lib):
+    """A depth window of S equals the full-depth operator on depth tensors
+    cut to each token's last S layers (L' = S)."""
+    B, Hq, Hk, T, d, L, S = 2, 4, 2, 7, 8, 5, 2
+    Q, K, V, Kd, Vd, _ = rand_case(B, Hq, Hk, T, d, L, 121)
+    cut = lambda x: x.reshape(B, Hk, T, L, d)[:, :, :, L - S:].reshape(B, Hk, T * S, d)
+    O, LSE = oracle.fwd(Q, K, V, Kd, Vd, lib=lib, window=S)
+    O2, LSE2 = oracle.fwd(Q, K, V, cut(Kd), cut(Vd), lib=lib)
+    _close(O, O2, 1e-12, "window O vs truncated depth")
+    _close(LSE, LSE2, 1e-12, "window LSE vs truncated depth")
+    g = oracle.bwd(Q, K, V, Kd, Vd, rand_case(B, Hq, Hk, T, d, L, 122)[5], lib=lib, window=S)
+    g2 = oracle.bwd(Q, K, V, cut(Kd), cut(Vd), rand_case(B, Hq, Hk, T, d, L, 122)[5], lib=lib)
+    for i, nm in ((0, "dQ"), (1, "dK"), (2, "dV")):
+        _close(g[i], g2[i], 1e-11, f"window {nm}")
+    full = g[3].reshape(B, Hk, T, L, d)
+    _close(full[:, :, :, L - S:].reshape(B, Hk, T * S, d), g2[3], 1e-11, "window dKd")
+    assert np.all(full[:, :, :, :L - S] == 0.0), "rows outside the window get zero gradient"
+
+
+def pin_modes_bwd_autograd(lib):
+    """Backward of the non-causal and windowed operator equals autograd
+    through the dense formulation."""
+    for (causal, window, seed) in ((False, 0, 131), (True, 2, 132), (False, 1, 133)):
+        Q, K, V, Kd, Vd, dO = rand_case(1, 4, 2, 7, 8, 3, seed)
+        xs = [x.clone().requires_grad_(True) for x in (Q, K, V, Kd, Vd)]
+        O, _ = dense_moda(*xs, causal=causal, window=window)
+        grads = torch.autograd.grad((O * dO).sum(), xs)
+        mine = oracle.bwd(Q, K, V, Kd, Vd, dO, lib=lib, causal=causal, window=window)
+        for nm, a, g in zip(("dQ", "dK", "dV", "dKd", "dVd"), mine, grads):
+            _close(a, g.numpy(), 1e-11, f"{nm} causal={causal} window={window}")
+
+
 ALL_PINS = [pin_l0_is_causal_sdpa, pin_t1_self_plus_depth, pin_dense_bruteforce,
             pin_algorithm1, pin_zero_query_closed_form, pin_depth_permutation,
             pin_gqa_is_repeat_interleave, pin_convexity, pin_bwd_autograd,
-            pin_bwd_finite_differences, pin_repack_definition]
+            pin_bwd_finite_differences, pin_repack_definition, pin_noncausal_l0_is_sdpa,
+            pin_modes_dense_bruteforce, pin_window_is_truncated_depth, pin_modes_bwd_autograd]

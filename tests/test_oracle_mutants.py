@@ -15,9 +15,9 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "moda_oracle.c")
 # (name, text in the oracle, planted replacement)
 MUTANTS = [
     ("seq_scale_dropped", "row[j] = scale * dot(", "row[j] = dot("),
-    ("depth_scale_dropped", "row[t + 1 + l] = scale * dot(", "row[t + 1 + l] = dot("),
-    ("depth_of_previous_token", "kd_off(b, hk, t, 0, Hk, T, L, d) : NULL;\n                const double* vd",
-     "kd_off(b, hk, t > 0 ? t - 1 : 0, 0, Hk, T, L, d) : NULL;\n                const double* vd"),
+    ("depth_scale_dropped", "row[n_seq + l] = scale * dot(", "row[n_seq + l] = dot("),
+    ("depth_of_previous_token", "kd_off(b, hk, t, l0, Hk, T, L, d) : NULL;\n                const double* vd",
+     "kd_off(b, hk, t > 0 ? t - 1 : 0, l0, Hk, T, L, d) : NULL;\n                const double* vd"),
     ("gqa_head_tiled", "const int hk = h / G;   /* [GQA] */", "const int hk = h % Hk;"),
     ("depth_value_dropped", "o[c] += w * Vdep[", "o[c] += 0.0 * Vdep["),
     ("lse_without_max", "*lse = m + log(Z);", "*lse = log(Z);"),
@@ -25,8 +25,11 @@ MUTANTS = [
      "const double ds = p * (dot(go, v, d) + Dr[r]);\n                        for (int c = 0; c < d; ++c) dq"),
     ("bwd_dkd_unscaled", "dKd[o + c] += scale * ds * q[c];", "dKd[o + c] += ds * q[c];"),
     ("bwd_dv_uses_ds", "dv[c] += p * go[c];", "dv[c] += ds * go[c];"),
-    ("bwd_dk_diagonal_dropped", "for (int t = j; t < T; ++t)", "for (int t = j + 1; t < T; ++t)"),
+    ("bwd_dk_diagonal_dropped", "for (int t = causal ? j : 0; t < T; ++t)",
+     "for (int t = causal ? j + 1 : 0; t < T; ++t)"),
     ("bwd_dq_transposed_operand", "dq[c] += scale * ds * k[c];", "dq[c] += scale * ds * q[c];"),
+    ("noncausal_ignored", "{ return causal ? t + 1 : T; }", "{ return t + 1; }"),
+    ("depth_window_ignored", "{ return (window > 0 && window < L) ? L - window : 0; }", "{ return 0; }"),
     ("repack_layer_major_kept", "const size_t o = (((size_t)b * Hk + hk) * T + t) * L + l;",
      "const size_t o = (((size_t)b * Hk + hk) * L + l) * T + t;"),
 ]
