@@ -79,6 +79,13 @@ typedef enum moda_depth_layout {
     MODA_DEPTH_CHUNKED = 1
 } moda_depth_layout;
 
+/* moda_shape.flags bits. */
+#define MODA_FLAG_NONCAUSAL 1  /* drop the sequence causal mask: every row sees
+                                  keys 0..T-1 (ByteDance-Seed/MoDA README,
+                                  "TODO": the non-causal MoDA kernel; vision use,
+                                  paper summary, "7. Implications and Future
+                                  Directions").  The depth matching mask stays. */
+
 typedef struct moda_shape {
     int B;            /* batch, >= 0 (0 = nothing to do)                   */
     int Hq;           /* query heads, >= 1                                  */
@@ -90,6 +97,12 @@ typedef struct moda_shape {
     moda_dtype dtype;
     moda_depth_layout depth_layout;
     float softmax_scale;  /* <= 0 selects 1/sqrt(d) */
+    int flags;        /* MODA_FLAG_* bits; 0 = the causal operator           */
+    int depth_window; /* 0 = all L depth rows; S in 1..L = each token attends
+                         only to its last S depth rows t*L+L-S .. t*L+L-1
+                         (bounded depth slots with a sliding-window policy,
+                         paper summary, "6. Limitations and Trade-offs");
+                         gradients of the other depth rows are zero          */
 } moda_shape;
 
 /*
@@ -193,6 +206,18 @@ moda_status moda_set_phase_events(void* const* events, int n);
  */
 moda_status moda_check_status(moda_stream_t stream);
 
+/*
+ * Failure-path self-test (the pages have no counterpart).  Queues on `stream`
+ * one small kernel whose warps wait, through the same bounded mbarrier wait
+ * the forward and backward kernels use, on a barrier that nothing arrives on.
+ * The wait gives up after its time limit (2 s), the kernel records the
+ * timeout in the device status word and returns normally; the next
+ * moda_check_status(stream) then returns MODA_ERR_TIMEOUT (and clears the
+ * word), and the device stays usable.  No memory is allocated or faulted.
+ * Returns MODA_ERR_CUDA if the launch fails, else MODA_OK.
+ */
+moda_status moda_selftest_wait_timeout(moda_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char* moda_status_string(moda_status status);
 
@@ -200,7 +225,7 @@ const char* moda_status_string(moda_status status);
 const char* moda_last_error_message(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
-int moda_version(void);
+int moda_version(void);   /* 10100: adds flags and depth_window to moda_shape */
 
 #ifdef __cplusplus
 }  /* extern "C" */

@@ -27,17 +27,21 @@ MODA_BF16 = 0
 MODA_FP32 = 1
 MODA_DEPTH_FLAT = 0
 MODA_DEPTH_CHUNKED = 1
+MODA_FLAG_NONCAUSAL = 1
 
 # Every symbol include/moda.h declares.
 EXPORTED = ("moda_workspace_size", "moda_repack_depth", "moda_fwd", "moda_bwd",
-            "moda_bwd_noalloc", "moda_set_phase_events", "moda_check_status", "moda_status_string", "moda_last_error_message", "moda_version")
+            "moda_bwd_noalloc", "moda_set_phase_events", "moda_check_status",
+            "moda_selftest_wait_timeout", "moda_status_string", "moda_last_error_message",
+            "moda_version")
 
 
 class moda_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hk", ctypes.c_int),
                 ("T", ctypes.c_int), ("d", ctypes.c_int), ("L", ctypes.c_int),
                 ("C", ctypes.c_int), ("dtype", ctypes.c_int), ("depth_layout", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_int),
+                ("depth_window", ctypes.c_int)]
 
 
 class MoDAError(RuntimeError):
@@ -79,6 +83,8 @@ def load(path: Optional[str] = None):
         lib.moda_set_phase_events.restype = i
         lib.moda_check_status.argtypes = [vp]
         lib.moda_check_status.restype = i
+        lib.moda_selftest_wait_timeout.argtypes = [vp]
+        lib.moda_selftest_wait_timeout.restype = i
         lib.moda_status_string.argtypes = [i]
         lib.moda_status_string.restype = ctypes.c_char_p
         lib.moda_last_error_message.argtypes = []
@@ -98,9 +104,9 @@ def status_name(status: int) -> str:
 
 
 def make_shape(B, Hq, Hk, T, d, L, C=0, dtype=MODA_BF16, depth_layout=MODA_DEPTH_FLAT,
-               softmax_scale=0.0) -> moda_shape:
+               softmax_scale=0.0, flags=0, depth_window=0) -> moda_shape:
     return moda_shape(int(B), int(Hq), int(Hk), int(T), int(d), int(L), int(C), int(dtype),
-                      int(depth_layout), float(softmax_scale))
+                      int(depth_layout), float(softmax_scale), int(flags), int(depth_window))
 
 
 def _ptr(x) -> Optional[int]:
@@ -172,6 +178,12 @@ def moda_set_phase_events(events) -> None:
 
 def moda_check_status(stream=None):
     _check(load().moda_check_status(_stream(stream)), "moda_check_status")
+
+
+def moda_selftest_wait_timeout(stream=None):
+    """Queue the bounded-wait self-test; the next moda_check_status raises
+    MoDAError with MODA_ERR_TIMEOUT."""
+    _check(load().moda_selftest_wait_timeout(_stream(stream)), "moda_selftest_wait_timeout")
 
 
 def moda_status_string(status: int) -> str:

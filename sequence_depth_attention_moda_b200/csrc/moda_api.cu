@@ -66,6 +66,11 @@ moda_status validate(const moda_shape* s, Problem* p) {
     } else if (s->C < 0) {
         return fail(MODA_ERR_INVALID_ARG, "C=%d must be >= 0", s->C);
     }
+    if (s->flags & ~MODA_FLAG_NONCAUSAL)
+        return fail(MODA_ERR_INVALID_ARG, "unknown flags 0x%x", (unsigned)s->flags);
+    if (s->depth_window < 0 || s->depth_window > s->L)
+        return fail(MODA_ERR_INVALID_ARG, "depth_window=%d must be in 0..L (L=%d)", s->depth_window,
+                    s->L);
     const int G = s->Hq / s->Hk;
     if (s->dtype == MODA_BF16) {
         if (s->d != 64 && s->d != 128)
@@ -84,6 +89,8 @@ moda_status validate(const moda_shape* s, Problem* p) {
     p->scale = s->softmax_scale > 0.0f ? s->softmax_scale : 1.0f / std::sqrt(float(s->d));
     p->scale_log2 = p->scale * 1.4426950408889634f;
     p->elem_bytes = s->dtype == MODA_BF16 ? 2 : 4;
+    p->causal = (s->flags & MODA_FLAG_NONCAUSAL) ? 0 : 1;
+    p->win_lo = s->depth_window > 0 ? s->L - s->depth_window : 0;
     return MODA_OK;
 }
 
@@ -254,6 +261,6 @@ moda_status moda_set_phase_events(void* const* events, int n) {
     return MODA_OK;
 }
 
-int moda_version(void) { return 100; }
+int moda_version(void) { return 10100; }
 
 }  // extern "C"

@@ -11,6 +11,8 @@
 //     dV_j = sum over the same rows of P dO
 //     dKd[t*L+l] = scale * sum over the group's heads of dS'_l q[h,t]
 //     dVd[t*L+l] = sum over the group's heads of P'_l dO[h,t]
+// Non-causal: "rows t >= j" becomes all rows.  Depth window S: only the last S
+// depth rows of a token take part; the gradients of the others are zero.
 //
 // Three launches, no floating-point atomics (bitwise repeatable):
 //  1. rowdot:  D[b,h,t] = sum_c dO * O                      (CUDA cores, HBM)
@@ -114,6 +116,7 @@ struct DkdvArgs {
     __nv_bfloat16* dV;
     unsigned int* status;
     int B, Hq, Hk, T, G, n_kt, n_qb;     // n_qb counts 64-row query blocks
+    int causal;
     float scale, scale_log2;
 };
 
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     const int bh = static_cast<int>(blockIdx.x) % nbh;
     const int b = bh / a.Hk;
     const int hk = bh - b * a.Hk;
-    const int qb0 = kt * (BN / kKvBQ);                      // first query block that sees the keys
+    const int qb0 = a.causal ? kt * (BN / kKvBQ) : 0;      // first query block that sees the keys
     const int nqb = a.n_qb - qb0;
     const int n_it = a.G * nqb;
 
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             if (mt == 0) MODA_TR(5, it);
             tc_fence_after();
             const int tq0 = qb * kKvBQ;
-            const bool diag = tq0 < kt * BN + BN;         // some key of the tile is after some query
+            const bool diag = a.causal && tq0 < kt * BN + BN;   // some key after some query
             uint32_t s[64], dp[64], pk[32], dk[32];
             tmem_ld32(lane_base + buf * 64, s);
             tmem_ld32(lane_base + buf * 64 + 32, s + 32);
@@ -387,6 +390,7 @@ struct DqArgs {
     __nv_bfloat16* dVd;
     unsigned int* status;
     int B, Hq, Hk, T, L, G, Tq, n_qt, dep_rows;
+    int causal, win_lo;
     float scale, scale_log2;
 };
 
@@ -440,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const int t0 = qt * a.Tq;
     const int R = a.G * a.Tq;
     const int t_end = min(t0 + a.Tq, a.T);
-    const int n_seq = (t_end - 1) / kDqBN + 1;
+    const int n_seq = ((a.causal ? t_end : a.T) - 1) / kDqBN + 1;
     const int dep_total = a.L > 0 ? (t_end - t0) * a.L : 0;
     const int n_dep = (dep_total + a.dep_rows - 1) / a.dep_rows;
     const int nb = n_seq + n_dep;
@@ -662,13 +666,15 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             tmem_ld32(lane_base + kColDP + buf * 64 + 32, dp + 32);
             tmem_wait_ld();
             int lo = 0, hi = kDqBN, kb = 0;
+            const int lim = a.causal ? t_row : a.T - 1;   // last visible sequence key
             if (seq) {
                 kb = i * kDqBN;
             } else {
-                lo = t_row * a.L - (t0 * a.L + jd * a.dep_rows);
-                hi = min(lo + a.L, a.dep_rows);
+                const int base = t_row * a.L - (t0 * a.L + jd * a.dep_rows);
+                lo = base + a.win_lo;
+                hi = min(base + a.L, a.dep_rows);
             }
-            const bool all_visible = seq && kb + kDqBN - 1 <= t_row;
+            const bool all_visible = seq && kb + kDqBN - 1 <= lim;
             // Masked entries get score -inf and dP 0 by selects (no branch per
             // element), so exp2 runs unconditionally and yields exactly 0.
             if (all_visible) {
@@ -683,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             } else {
                 // visible columns: seq c <= t_row - kb; depth lo <= c < hi
                 const int vlo = seq ? 0 : lo;
-                const int vhi = seq ? t_row - kb + 1 : hi;
+                const int vhi = seq ? lim - kb + 1 : hi;
 #pragma unroll
                 for (int e = 0; e < 64; e += 2) {
                     float p2[2], d2[2];
@@ -785,6 +791,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     A.n_kt = (p.T + BN - 1) / BN;
     A.n_qb = (p.T + kKvBQ - 1) / kKvBQ;
     A.scale = p.scale; A.scale_log2 = p.scale_log2;
+    A.causal = p.causal;
     A.LSE = LSE; A.Drow = Dws;
     A.dK = static_cast<__nv_bfloat16*>(dK);
     A.dV = static_cast<__nv_bfloat16*>(dV);
@@ -813,6 +820,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     B.dep_rows = dep >= 64 ? 64 : ((dep + 15) / 16) * 16;
     if (B.dep_rows < 16) B.dep_rows = 16;
     B.scale = p.scale; B.scale_log2 = p.scale_log2;
+    B.causal = p.causal; B.win_lo = p.win_lo;
     B.LSE = LSE; B.Drow = Dws;
     B.dQ = static_cast<__nv_bfloat16*>(dQ);
     B.dKd = static_cast<__nv_bfloat16*>(dKd);

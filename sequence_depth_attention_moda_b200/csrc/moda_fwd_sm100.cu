@@ -4,7 +4,10 @@
 // (MoDA): The Unified Operator" -- one softmax over the causal sequence keys
 // (j <= t) and the token's own L depth rows, scaled by 1/sqrt(d); the online
 // form is "Fused online-softmax (Algorithm 1)" (running max / sum / output in
-// base 2, sequence blocks then depth blocks, o / acc at the end).
+// base 2, sequence blocks then depth blocks, o / acc at the end).  Two options
+// change only the visible sets: non-causal (every row sees keys 0..T-1; the
+// README's "TODO" non-causal kernel) and a depth window (the last S of the L
+// depth rows; bounded depth slots, summary "6. Limitations and Trade-offs").
 //
 // Work unit: one query tile of 128 rows = the G heads of one KV head times
 // Tq = 128/G consecutive tokens (row r -> head g = r / Tq, token t0 + r % Tq).
@@ -88,6 +91,8 @@ struct FwdArgs {
     float* LSE;
     unsigned int* status;
     int B, Hq, Hk, T, L, G, Tq, n_qt, dep_rows;
+    int causal;       // 0: every row sees keys 0..T-1
+    int win_lo;       // first visible depth row of a token
     float scale_log2;
 };
 
@@ -136,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
     const int t0 = qt * a.Tq;
     const int R = a.G * a.Tq;
     const int t_end = min(t0 + a.Tq, a.T);           // one past the last real token
-    const int n_seq = (t_end - 1) / BN + 1;
+    const int n_seq = ((a.causal ? t_end : a.T) - 1) / BN + 1;
     const int n_dep = a.L > 0 ? ((t_end - t0) * a.L + a.dep_rows - 1) / a.dep_rows : 0;
     const int nb = n_seq + n_dep;
 
@@ -311,14 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             // masks, then the row max as four independent partial maxima
             if (i < n_seq) {
                 const int kb = i * BN;
-                if (kb + BN - 1 > t_row) {
+                const int lim = a.causal ? t_row : a.T - 1;   // last visible key
+                if (kb + BN - 1 > lim) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if (kb + c > t_row) sr[c] = __float_as_uint(-INFINITY);
+                        if (kb + c > lim) sr[c] = __float_as_uint(-INFINITY);
                 }
             } else {
-                const int lo = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows);
-                const int hi = min(lo + a.L, a.dep_rows);
+                const int base = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows);
+                const int lo = base + a.win_lo;
+                const int hi = min(base + a.L, a.dep_rows);
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c < lo || c >= hi) sr[c] = __float_as_uint(-INFINITY);
@@ -429,6 +436,8 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     a.dep_rows = dep >= 128 ? 128 : ((dep + 15) / 16) * 16;
     if (a.dep_rows < 16) a.dep_rows = 16;
     a.scale_log2 = p.scale_log2;
+    a.causal = p.causal;
+    a.win_lo = p.win_lo;
     a.O = static_cast<__nv_bfloat16*>(O);
     a.LSE = LSE;
     a.status = device_status_word();

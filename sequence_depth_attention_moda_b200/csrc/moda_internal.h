@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "moda.h"
+
 namespace moda {
 
 // A validated problem.  Index conventions follow the C ABI (include/moda.h).
@@ -14,6 +16,8 @@ struct Problem {
     float scale;        // softmax scale on the natural-log scale
     float scale_log2;   // scale * log2(e): scores go straight into exp2
     int elem_bytes;     // 2 (bf16) or 4 (fp32)
+    int causal;         // 1: key j visible to row t iff j <= t; 0: all keys
+    int win_lo;         // first visible depth row of a token (L - window, or 0)
 };
 
 // Kernel-side status bits written into the per-device status word.
@@ -23,6 +27,10 @@ enum : unsigned int {
 
 // Address of the calling device's status word (device memory), or nullptr.
 unsigned int* device_status_word();
+// Shape validation and error recording of the API layer, for entry points
+// defined outside moda_api.cu.
+moda_status api_validate(const moda_shape* shape, Problem* p);
+moda_status api_fail(moda_status s, const char* msg);
 
 // SM count of the current device (cached).
 int device_sm_count();

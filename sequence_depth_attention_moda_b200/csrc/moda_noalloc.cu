@@ -9,10 +9,6 @@
 #include "moda_internal.h"
 
 namespace moda {
-
-moda_status api_validate(const moda_shape* shape, Problem* p);
-moda_status api_fail(moda_status s, const char* msg);
-
 namespace {
 
 // Capacity in query rows (B * Hq * T): 4 Mi rows = 16 MiB of fp32.  Every

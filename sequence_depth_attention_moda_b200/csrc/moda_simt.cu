@@ -92,8 +92,9 @@ fwd_simt_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K,
         }
         m = m_new;
     };
-    for (int j = 0; j <= t; ++j) visit(K + (kv0 + j) * d, V + (kv0 + j) * d);
-    for (int l2 = 0; l2 < p.L; ++l2) {
+    const int jmax = p.causal ? t : p.T - 1;   // last visible sequence key
+    for (int j = 0; j <= jmax; ++j) visit(K + (kv0 + j) * d, V + (kv0 + j) * d);
+    for (int l2 = p.win_lo; l2 < p.L; ++l2) {
         const long long r = (kv0 + t) * p.L + l2;
         visit(Kd + r * d, Vd + r * d);
     }
@@ -152,8 +153,9 @@ bwd_dq_simt_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K,
             if (c < d) dq[i] += ds * to_f(krow[c]);
         }
     };
-    for (int j = 0; j <= t; ++j) visit(K + (kv0 + j) * d, V + (kv0 + j) * d);
-    for (int l2 = 0; l2 < p.L; ++l2) {
+    const int jmax = p.causal ? t : p.T - 1;   // last visible sequence key
+    for (int j = 0; j <= jmax; ++j) visit(K + (kv0 + j) * d, V + (kv0 + j) * d);
+    for (int l2 = p.win_lo; l2 < p.L; ++l2) {
         const long long r = (kv0 + t) * p.L + l2;
         visit(Kd + r * d, Vd + r * d);
     }
@@ -176,6 +178,7 @@ bwd_ddepth_simt_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__
     const long long nrows = (long long)p.B * p.Hk * p.T * p.L;
     if (r >= nrows) return;
     const long long tok = r / p.L;               // (b*Hk + hk)*T + t
+    const bool in_window = (int)(r - tok * p.L) >= p.win_lo;
     const int t = (int)(tok % p.T);
     const long long bh = tok / p.T;
     const int hk = (int)(bh % p.Hk);
@@ -185,7 +188,7 @@ bwd_ddepth_simt_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__
     float dk[kMaxPerLane] = {0.f, 0.f, 0.f, 0.f}, dv[kMaxPerLane] = {0.f, 0.f, 0.f, 0.f};
     load_row(Kd + r * d, d, lane, kd);
     load_row(Vd + r * d, d, lane, vd);
-    for (int g = 0; g < p.G; ++g) {
+    for (int g = 0; g < (in_window ? p.G : 0); ++g) {
         const long long qrow = ((long long)b * p.Hq + hk * p.G + g) * p.T + t;
         const float pr =
             exp2f(dot_row(kd, Q + qrow * d, d, lane) * p.scale_log2 - LSE[qrow] * 1.4426950408889634f);
@@ -231,7 +234,7 @@ bwd_dkdv_simt_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K
     load_row(V + r * d, d, lane, v);
     for (int g = 0; g < p.G; ++g) {
         const long long q0 = ((long long)b * p.Hq + hk * p.G + g) * p.T;
-        for (int t = j; t < p.T; ++t) {
+        for (int t = p.causal ? j : 0; t < p.T; ++t) {
             const long long qrow = q0 + t;
             const float pr = exp2f(dot_row(k, Q + qrow * d, d, lane) * p.scale_log2 -
                                    LSE[qrow] * 1.4426950408889634f);

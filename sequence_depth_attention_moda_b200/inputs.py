@@ -34,6 +34,8 @@ class Workload:
     qk_scaled: bool = False      # Q and K drawn as N(0,1)/sqrt(d)
     backward: bool = False       # the workload includes the backward pass
     seed: int = 1000
+    causal: bool = True          # False: every row sees all T sequence keys
+    window: int = 0              # > 0: each token's last `window` depth rows only
 
     @property
     def G(self) -> int:

@@ -32,7 +32,9 @@ GRAD_MAX_REL, GRAD_MEAN_REL = 2e-2, 5e-3
 
 def shape_of(w: Workload, layout=moda.MODA_DEPTH_FLAT, C=None):
     return moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C if C is None else C,
-                           moda.MODA_BF16 if w.dtype == "bf16" else moda.MODA_FP32, layout)
+                           moda.MODA_BF16 if w.dtype == "bf16" else moda.MODA_FP32, layout,
+                           flags=0 if w.causal else moda.MODA_FLAG_NONCAUSAL,
+                           depth_window=w.window)
 
 
 def run_gpu(w: Workload, x: Dict[str, torch.Tensor], backward=None, layout=moda.MODA_DEPTH_FLAT,
@@ -92,12 +94,13 @@ def f64(t: torch.Tensor) -> np.ndarray:
 def oracle_fwd_full(w, x):
     Kd, Vd = token_major(x, w)
     return oracle.fwd(f64(x["Q"]), f64(x["K"]), f64(x["V"]), f64(Kd) if w.L else None,
-                      f64(Vd) if w.L else None)
+                      f64(Vd) if w.L else None, causal=w.causal, window=w.window)
 
 
 def oracle_bwd_full(w, x):
     Kd, Vd = token_major(x, w)
-    return oracle.bwd(f64(x["Q"]), f64(x["K"]), f64(x["V"]), f64(Kd), f64(Vd), f64(x["dO"]))
+    return oracle.bwd(f64(x["Q"]), f64(x["K"]), f64(x["V"]), f64(Kd), f64(Vd), f64(x["dO"]),
+                      causal=w.causal, window=w.window)
 
 
 def sample_rows(w: Workload, n_random: int, seed: int = 7) -> List[Tuple[int, int, int]]:
@@ -115,19 +118,22 @@ def sample_rows(w: Workload, n_random: int, seed: int = 7) -> List[Tuple[int, in
 
 
 def oracle_rows(w: Workload, x, Kd_dev, Vd_dev, rows: Sequence[Tuple[int, int, int]]):
-    """Oracle O and LSE for sampled rows; depth rows are read from the
-    token-major tensors gathered through the oracle's index definition."""
+    """Oracle O and LSE for sampled rows, each computed from its visible rows
+    alone (sequence keys and depth rows taken straight from the inputs)."""
     O = np.zeros((len(rows), w.d))
     LSE = np.zeros(len(rows))
     for i, (b, h, t) in enumerate(rows):
         hk = h // w.G
         q = f64(x["Q"][b, h, t])
-        Ks = f64(x["K"][b, hk, :t + 1])
-        Vs = f64(x["V"][b, hk, :t + 1])
+        n_seq = t + 1 if w.causal else w.T
+        Ks = f64(x["K"][b, hk, :n_seq])
+        Vs = f64(x["V"][b, hk, :n_seq])
         if w.L:
-            # layer-major source: depth row l of token t is Kd_layer[l, b, hk, t]
-            Kdep = f64(x["Kd_layer"][:, b, hk, t])
-            Vdep = f64(x["Vd_layer"][:, b, hk, t])
+            # layer-major source: depth row l of token t is Kd_layer[l, b, hk, t];
+            # a window keeps the last w.window layers
+            l0 = w.L - w.window if w.window else 0
+            Kdep = f64(x["Kd_layer"][l0:, b, hk, t])
+            Vdep = f64(x["Vd_layer"][l0:, b, hk, t])
         else:
             Kdep = Vdep = np.zeros((0, w.d))
         O[i], LSE[i] = oracle.row(q, Ks, Vs, Kdep, Vdep)

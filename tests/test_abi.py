@@ -64,6 +64,9 @@ FAKE = 0x10000   # aligned fake device address: never dereferenced (validation f
     (dict(dtype=7), 1),
     (dict(depth_layout=1, C=0), 1),                                      # chunked needs C
     (dict(depth_layout=1, C=48), 1),                                     # T % C
+    (dict(flags=2), 1),                                                  # unknown flag
+    (dict(depth_window=3), 1),                                           # window > L
+    (dict(depth_window=-1), 1),
 ])
 def test_fwd_rejects_bad_shapes(lib, kw, status):
     base = dict(B=1, Hq=4, Hk=2, T=64, d=128, L=2, C=16)

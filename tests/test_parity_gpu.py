@@ -234,3 +234,44 @@ def test_bwd_workspace_error_on_device():
         moda.moda_bwd(sh, x["Q"], x["K"], x["V"], out["Kd"], out["Vd"], out["O"], out["LSE"],
                       x["dO"], g["dQ"], g["dK"], g["dV"], g["dKd"], g["dVd"], ws, need - 16)
     assert ei.value.status == 4
+
+
+# ------------------------------------------- non-causal and depth window ----
+MODES = [(False, 0), (True, 3), (False, 2), (True, 8)]
+MODE_CASES = [(1, 8, 2, 128, 300, 8), (2, 4, 4, 64, 130, 5), (1, 6, 2, 128, 97, 3)]
+
+
+@pytest.mark.parametrize("mode", MODES, ids=lambda m: "causal%d_win%d" % m)
+@pytest.mark.parametrize("case", MODE_CASES, ids=lambda c: "B%d_Hq%d_Hk%d_d%d_T%d_L%d" % c)
+def test_modes_fwd_bwd_small(case, mode):
+    causal, window = mode
+    if window > case[5]:
+        pytest.skip("window larger than L")
+    w = small_w(*case, backward=True).with_(causal=causal, window=window)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x)
+    O, LSE = oracle_fwd_full(w, x)
+    assert_out_close(f64(out["O"]), O, "bf16", "O")
+    assert err_stats(f64(out["LSE"]), LSE)[0] <= LSE_MAX_ABS
+    for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(w, x)):
+        assert_grad_close(f64(out[name]), r, name)
+
+
+def test_modes_fp32():
+    for causal, window in MODES:
+        w = I.TINY_FP32.with_(causal=causal, window=window, backward=True)
+        x = I.make_inputs(w, device=DEV)
+        out = run_gpu(w, x)
+        O, _ = oracle_fwd_full(w, x)
+        assert_out_close(f64(out["O"]), O, "fp32", f"O causal={causal} window={window}")
+        for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(w, x)):
+            assert err_stats(f64(out[name]), r)[0] <= 1e-4, name
+
+
+def test_modes_layer_T4k_sampled():
+    for causal, window in ((False, 0), (True, 4)):
+        w = I.LAYER_1P5B.with_(causal=causal, window=window)
+        x = I.make_inputs(w, device=DEV)
+        out = run_gpu(w, x)
+        _check_rows(w, x, out)
+        _check_slices(w, x, out, [(0, 2)])
