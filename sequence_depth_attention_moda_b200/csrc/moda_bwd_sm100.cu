@@ -222,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 mbar_wait(&bars[kA_QFull + it % kKvStages], (it / kKvStages) & 1, a.status, abort_flag);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        // whole warp, converged: warp-uniform waits, one elected lane issues
+        {
             const uint32_t id_s = idesc_bf16(128, kKvBQ, false, false);
             const uint32_t id_g = idesc_bf16(128, D, false, true);
             const uint64_t kd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kK));
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             auto issue_s = [&](int j) -> bool {
                 const int st = j % kKvStages;
                 const int buf = j & 1;
-                if (!mbar_wait(&bars[kA_QFull + st], (j / kKvStages) & 1, a.status, abort_flag)) return false;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_QFull + st], (j / kKvStages) & 1, a.status, abort_flag))) return false;
                 MODA_TR(10, j);
                 tc_fence_after();
                 const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
@@ -240,25 +241,25 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                     const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
+                    umma_ss_elect(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                     const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
+                    umma_ss_elect(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&bars[kA_SFull + buf]);
+                umma_commit_elect(&bars[kA_SFull + buf]);
                 return true;
             };
-            bool ok = mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag) && (n_it == 0 || issue_s(0));
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag)) && (n_it == 0 || issue_s(0));
             for (int it = 0; ok && it < n_it; ++it) {
                 MODA_TR(0, it);
                 if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
                 MODA_TR(1, it);
                 const int st = it % kKvStages;
                 const int buf = it & 1;
-                if (!mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
                 MODA_TR(2, it);
                 tc_fence_after();
                 const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
@@ -266,13 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
 #pragma unroll
                 for (int kk = 0; kk < kKvBQ / 16; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, acc);
-                    umma_ts(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g, acc);
+                    umma_ts_elect(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, acc);
+                    umma_ts_elect(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g, acc);
                 }
-                umma_commit(&bars[kA_QEmpty + st]);
+                umma_commit_elect(&bars[kA_QEmpty + st]);
                 MODA_TR(3, it);
             }
-            umma_commit(&bars[kA_Final]);
+            umma_commit_elect(&bars[kA_Final]);
         }
     } else {
         const int quarter = warp & 3;
@@ -523,7 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer --
-        if (lane == 0) {
+        // whole warp, converged: warp-uniform waits, one elected lane issues
+        {
             const uint32_t id_seq = idesc_bf16(128, kDqBN, false, false);
             const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
             const uint32_t id_dq = idesc_bf16(128, D, false, true);
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             auto issue_s = [&](int j) -> bool {
                 const int st = j % kDqStages;
                 const int buf = j & 1;
-                if (!mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag)) return false;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag))) return false;
                 MODA_TRQ(8, j);
                 tc_fence_after();
                 const uint32_t id = j < n_seq ? id_seq : id_dep;
@@ -548,18 +550,18 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t offq = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                     const uint64_t offk = ((kk >> 2) * kDqSlab + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + kColS + buf * 64, qd0 + offq, kd + offk, id, kk > 0 ? 1u : 0u);
+                    umma_ss_elect(tmem + kColS + buf * 64, qd0 + offq, kd + offk, id, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t offq = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                     const uint64_t offk = ((kk >> 2) * kDqSlab + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + kColDP + buf * 64, dod0 + offq, vd + offk, id, kk > 0 ? 1u : 0u);
+                    umma_ss_elect(tmem + kColDP + buf * 64, dod0 + offq, vd + offk, id, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&bars[kB_SFull + buf]);
+                umma_commit_elect(&bars[kB_SFull + buf]);
                 return true;
             };
-            bool ok = mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag) && issue_s(0);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag)) && issue_s(0);
             for (int i = 0; ok && i < nb; ++i) {
                 // the next block's scores first: its buffer was released when
                 // the math warps finished block i-1 (waited below last round)
@@ -570,34 +572,34 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 const int buf = i & 1;
                 const bool seq = i < n_seq;
                 const int n = seq ? kDqBN : a.dep_rows;
-                if (!mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
                 MODA_TRQ(2, i);
                 tc_fence_after();
                 const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
                 if (n == kDqBN) {
 #pragma unroll
                     for (int kk = 0; kk < kDqBN / 16; ++kk)
-                        umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
+                        umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
                                 (i > 0 || kk > 0) ? 1u : 0u);
                 } else {
                     for (int kk = 0; kk < n / 16; ++kk)
-                        umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
+                        umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
                                 (i > 0 || kk > 0) ? 1u : 0u);
                 }
                 if (!seq) {
 #pragma unroll
                     for (int kk = 0; kk < BM / 16; ++kk) {
-                        umma_ss(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
+                        umma_ss_elect(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
                                 desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
-                        umma_ss(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
+                        umma_ss_elect(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
                                 desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
                     }
-                    umma_commit(&bars[kB_DDFull]);
+                    umma_commit_elect(&bars[kB_DDFull]);
                 }
-                umma_commit(&bars[kB_KVEmpty + st]);
+                umma_commit_elect(&bars[kB_KVEmpty + st]);
                 MODA_TRQ(3, i);
             }
-            umma_commit(&bars[kB_Final]);
+            umma_commit_elect(&bars[kB_Final]);
         }
     } else {
         // ------------------------------------------------------ math --------

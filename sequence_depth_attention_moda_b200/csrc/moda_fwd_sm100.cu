@@ -16,9 +16,9 @@
 // group, and the depth rows of the tile's Tq tokens are one contiguous range
 // [t0*L, (t0+Tq)*L) of the token-major depth tensor.
 //
-// CTA roles (224 threads):
+// CTA roles (352 threads):
 //   warp 0      TMA producer of Q (once) and of the K (or K_depth) tiles;
-//   warp 6      TMA producer of the V (or V_depth) tiles.  K and V have rings
+//   warp 10     TMA producer of the V (or V_depth) tiles.  K and V have rings
 //               of their own: a K stage frees as soon as S_i = Q K_i^T is
 //               done, a V stage only when O += P_i V_i is, so the next K
 //               tiles stream in while PV still holds older V tiles.
@@ -28,10 +28,15 @@
 //               before PV_i, so two score tiles are always ahead of the
 //               softmax and the tensor pipe's issue-to-completion latency
 //               (hundreds of cycles) is off the softmax's critical path.
-//   warps 2..5  softmax, one thread per tile row: tcgen05.ld of S, masks,
-//               running max, exp2, row sum, P (bf16) written back over S with
-//               tcgen05.st; O in TMEM is rescaled only when the running max
-//               grew by more than 2^8 (exact: the final o / acc cancels it).
+//   warps 2..9  softmax, two warps per TMEM lane quarter (16 rows each) and
+//               two threads per tile row: with the 16x32bx2 TMEM shapes,
+//               thread t < 16 holds columns [0, 64) of its row and thread
+//               t + 16 columns [64, 128), so the row max and sum take one
+//               shuffle.  Per block: tcgen05.ld of S, masks, running max,
+//               exp2, row sum, P (bf16) written back over S with tcgen05.st;
+//               O in TMEM is rescaled only when the running max grew by more
+//               than 2^8 (exact: the final o / acc cancels it).  Two warps
+//               per SM sub-partition keep its MUFU (exp2) unit fed.
 // TMEM columns: S0 [0,128), S1 [128,256), S2 [256,384), O [384, 384+d).
 // Softmax: row max as four partial maxima of three-input max; exp2 on the MUFU unit (a build
 // knob moves a share of column pairs to ex2_fma on the FMA pipe; measured
@@ -58,13 +63,17 @@ constexpr int BN = 128;          // sequence keys per block
 #endif
 constexpr int kKStages = MODA_FWD_KSTAGES;   // K ring: a stage frees when S_i is done
 constexpr int kVStages = MODA_FWD_VSTAGES;   // V ring: a stage frees when PV_i is done
-constexpr int kThreads = 224;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kSoftmaxWarps = 8;             // warps 2..9
+constexpr int kVWarp = 2 + kSoftmaxWarps;    // V producer
+constexpr int kThreads = 32 * (kVWarp + 1);
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kSlabBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBufs = 3;            // S / P buffers in TMEM
 constexpr uint32_t kColO = 384;      // O accumulator after the three S buffers
+#ifndef MODA_FWD_OFFSET
+#define MODA_FWD_OFFSET 0            // cycles the rows-16..31 softmax warps start late
+#endif
 #ifndef MODA_FWD_SWEXP
 #define MODA_FWD_SWEXP 0             // of every 4 column pairs, this many use ex2_fma
 #endif
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         }
         for (int s = 0; s < kSBufs; ++s) {
             mbar_init(&bars[kSFull + s], 1);
-            mbar_init(&bars[kPReady + s], kSoftmaxThreads);
+            mbar_init(&bars[kPReady + s], kSoftmaxWarps);   // one arrive per softmax warp
         }
         mbar_init(&bars[kOFinal], 1);
         *abort_flag = 0;
@@ -179,9 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == 0 || warp == 6) {
+    if (warp == 0 || warp == kVWarp) {
         // ------------------------------------------------------ producers ---
-        // warp 0: Q, then K_i (sequence) / K_depth tiles; warp 6: V tiles.
+        // warp 0: Q, then K_i (sequence) / K_depth tiles; warp kVWarp: V tiles.
         if (lane == 0) {
             const bool is_k = warp == 0;
             const int nst = is_k ? kKStages : kVStages;
@@ -223,123 +232,138 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer --
-        if (lane == 0) {
-            const uint32_t id_seq = idesc_bf16(128, BN, false, false);
-            const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
-            const uint32_t id_pv = idesc_bf16(128, D, false, true);
-            // Descriptors are built once; a K step adds its byte offset / 16
-            // to the 14-bit address field (shared addresses stay < 256 KB).
-            const uint64_t qd0 = desc_kmajor_sw128(smem_u32(sQ));
-            bool ok = mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
-            // S(j) = Q K_j^T into buffer j % 3.  The buffer last held P(j-3),
-            // read by PV(j-3), which is issued before S(j) (in-order pipe).
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % kKStages;
-                const int sb = j % kSBufs;
-                MODA_TRF(0, j);
-                if (!mbar_wait(&bars[kKFull + st], (j / kKStages) & 1, a.status, abort_flag)) return false;
-                MODA_TRF(1, j);
-                tc_fence_after();
-                const uint64_t kd0 = desc_kmajor_sw128(smem_u32(sK + st * Lay::kTile));
-                const uint32_t id = j < n_seq ? id_seq : id_dep;
+        // The whole warp runs this loop converged, so descriptors and waits
+        // are warp-uniform; elect.sync picks the lane that issues each MMA
+        // and commit.
+        const bool tl = lane == 0;                    // trace lane
+        const uint32_t id_seq = idesc_bf16(128, BN, false, false);
+        const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
+        const uint32_t id_pv = idesc_bf16(128, D, false, true);
+        // Descriptors are built once; a K step adds its byte offset / 16 to
+        // the 14-bit address field (shared addresses stay < 256 KB).
+        const uint64_t qd0 = desc_kmajor_sw128(smem_u32(sQ));
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], 0, a.status, abort_flag));
+        // S(j) = Q K_j^T into buffer j % 3.  The buffer last held P(j-3),
+        // read by PV(j-3), which is issued before S(j) (in-order pipe).
+        auto issue_s = [&](int j) -> bool {
+            const int st = j % kKStages;
+            const int sb = j % kSBufs;
+            if (tl) MODA_TRF(0, j);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kKFull + st], (j / kKStages) & 1, a.status,
+                                                   abort_flag))) return false;
+            if (tl) MODA_TRF(1, j);
+            tc_fence_after();
+            const uint64_t kd0 = desc_kmajor_sw128(smem_u32(sK + st * Lay::kTile));
+            const uint32_t id = j < n_seq ? id_seq : id_dep;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + sb * 128, qd0 + off, kd0 + off, id, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&bars[kSFull + sb]);
-                MODA_TRF(2, j);
-                return true;
-            };
-            // O += P(j) V_j with P read from TMEM buffer j % 3.
-            auto issue_pv = [&](int j) -> bool {
-                const int st = j % kVStages;
-                const int sb = j % kSBufs;
-                if (!mbar_wait(&bars[kPReady + sb], (j / kSBufs) & 1, a.status, abort_flag)) return false;
-                MODA_TRF(4, j);
-                if (!mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status, abort_flag)) return false;
-                tc_fence_after();
-                const int krows = j < n_seq ? BN : a.dep_rows;
-                const uint64_t vd0 = desc_mnmajor_sw128(smem_u32(sV + st * Lay::kTile), kSlabBytes);
-                if (krows == BN) {
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
-                                (j > 0 || kk > 0) ? 1u : 0u);
-                } else {
-                    for (int kk = 0; kk < krows / 16; ++kk)
-                        umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
-                                (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&bars[kVEmpty + st]);
-                MODA_TRF(3, j);
-                return true;
-            };
-            // Two score tiles run ahead of the softmax.  S(i+2) goes in
-            // before PV(i): its buffer held P(i-1), whose PV(i-1) is already
-            // in the (in-order) pipe, so it never waits for P(i); each issue
-            // blocks until the shallow MMA queue has room, so this order is
-            // what keeps the next scores ready when the softmax needs them.
-            if (ok) ok = issue_s(0);
-            if (ok && nb > 1) ok = issue_s(1);
-            for (int i = 0; ok && i < nb; ++i) {
-                if (i + 2 < nb && !issue_s(i + 2)) { ok = false; break; }
-                if (!issue_pv(i)) { ok = false; break; }
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t off = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                umma_ss_elect(tmem + sb * 128, qd0 + off, kd0 + off, id, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&bars[kOFinal]);
+            umma_commit_elect(&bars[kSFull + sb]);
+            if (tl) MODA_TRF(2, j);
+            return true;
+        };
+        // O += P(j) V_j with P read from TMEM buffer j % 3.
+        auto issue_pv = [&](int j) -> bool {
+            const int st = j % kVStages;
+            const int sb = j % kSBufs;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kPReady + sb], (j / kSBufs) & 1, a.status,
+                                                   abort_flag))) return false;
+            if (tl) MODA_TRF(4, j);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status,
+                                                   abort_flag))) return false;
+            tc_fence_after();
+            const int krows = j < n_seq ? BN : a.dep_rows;
+            const uint64_t vd0 = desc_mnmajor_sw128(smem_u32(sV + st * Lay::kTile), kSlabBytes);
+            if (krows == BN) {
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_ts_elect(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+            } else {
+                for (int kk = 0; kk < krows / 16; ++kk)
+                    umma_ts_elect(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit_elect(&bars[kVEmpty + st]);
+            if (tl) MODA_TRF(3, j);
+            return true;
+        };
+        // Two score tiles run ahead of the softmax.  S(i+2) goes in before
+        // PV(i): its buffer held P(i-1), whose PV(i-1) is already in the
+        // (in-order) pipe, so it never waits for P(i); each issue blocks
+        // until the shallow MMA queue has room, so this order is what keeps
+        // the next scores ready when the softmax needs them.
+        if (ok) ok = issue_s(0);
+        if (ok && nb > 1) ok = issue_s(1);
+        for (int i = 0; ok && i < nb; ++i) {
+            if (i + 2 < nb && !issue_s(i + 2)) { ok = false; break; }
+            if (!issue_pv(i)) { ok = false; break; }
         }
-    } else if (warp >= 2 && warp <= 5) {
+        umma_commit_elect(&bars[kOFinal]);
+    } else if (warp >= 2 && warp < 2 + kSoftmaxWarps) {
         // ------------------------------------------------------ softmax -----
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
-        const int r = quarter * 32 + lane;            // tile row
+        const int sub = (warp - 2) >> 2;              // rows 16*sub .. of the quarter
+        const int half = lane >> 4;                   // column half of the row
+        const int r = quarter * 32 + sub * 16 + (lane & 15);   // tile row
         const bool row_real = r < R;
         const int g = row_real ? r / a.Tq : 0;
         const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
+        const int c0 = half * 64;                     // first S column this thread holds
+        const bool tr = r == 0 && half == 0;          // trace threads
+        const bool tr2 = r == 32 && half == 0;        // quarter 1: the MMA warp's sub-partition
         const float sl2 = a.scale_log2;
-        float m = -INFINITY, l = 0.0f;
+        float m = -INFINITY, l = 0.0f;                // l: this half's share of the row sum
         bool ok = true;
         for (int i = 0; i < nb; ++i) {
             const int sb = i % kSBufs;
-            if (r == 0) MODA_TRF(5, i);
-            if (!mbar_wait(&bars[kSFull + sb], (i / kSBufs) & 1, a.status, abort_flag)) { ok = false; break; }
-            if (r == 0) MODA_TRF(6, i);
+            if (tr) MODA_TRF(5, i);
+            // every wait result is made warp-uniform: the shuffles and the
+            // .sync.aligned TMEM accesses below need the whole warp
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + sb], (i / kSBufs) & 1, a.status,
+                                                   abort_flag))) { ok = false; break; }
+            if (tr) MODA_TRF(6, i);
+            if (tr2) MODA_TRF(12, i);
             tc_fence_after();
-            uint32_t sr[128];
+            uint32_t sr[64];
             const uint32_t s_addr = lane_base + sb * 128;
-            tmem_ld32(s_addr, sr);
-            tmem_ld32(s_addr + 32, sr + 32);
-            tmem_ld32(s_addr + 64, sr + 64);
-            tmem_ld32(s_addr + 96, sr + 96);
+            tmem_ld16x2_32<64>(s_addr, sr);            // columns c0 .. c0+31
+            tmem_ld16x2_32<64>(s_addr + 32, sr + 32);  // columns c0+32 .. c0+63
             tmem_wait_ld();
-            if (r == 0) MODA_TRF(7, i);
+            reg_fence<64>(sr);
+            if (tr) MODA_TRF(7, i);
             // masks, then the row max as four independent partial maxima
             if (i < n_seq) {
-                const int kb = i * BN;
+                const int kb = i * BN + c0;
                 const int lim = a.causal ? t_row : a.T - 1;   // last visible key
-                if (kb + BN - 1 > lim) {
+                if (kb + 63 > lim) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
+                    for (int c = 0; c < 64; ++c)
                         if (kb + c > lim) sr[c] = __float_as_uint(-INFINITY);
                 }
             } else {
-                const int base = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows);
+                const int base = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows) - c0;
                 const int lo = base + a.win_lo;
-                const int hi = min(base + a.L, a.dep_rows);
+                const int hi = min(base + a.L, a.dep_rows - c0);
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
+                for (int c = 0; c < 64; ++c)
                     if (c < lo || c >= hi) sr[c] = __float_as_uint(-INFINITY);
             }
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 128; c += 8) {
+            for (int c = 0; c < 64; c += 8) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
                     mx4[u] = fmax3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
             }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             const float m_new = fmaxf(m, mx * sl2);
-            if (r == 0) MODA_TRF(8, i);
+            if (tr) MODA_TRF(8, i);
+            if (tr2) MODA_TRF(13, i);
             if (i == 0) {
                 m = m_new;
             } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
@@ -347,28 +371,32 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 // the V-stage release PV_{i-1} commits.  S_i was issued after
                 // PV_{i-2}, so at most PV_{i-1} is in flight, and PV_{i+2}
                 // (the stage's next use) needs P_{i+2}: the parity is exact.
-                if (!mbar_wait(&bars[kVEmpty + (i - 1) % kVStages], ((i - 1) / kVStages) & 1, a.status,
-                               abort_flag)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + (i - 1) % kVStages],
+                                                       ((i - 1) / kVStages) & 1, a.status, abort_flag))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const float alpha = ex2(m - m_new);
                 l *= alpha;
                 m = m_new;
 #pragma unroll
-                for (int c = 0; c < D; c += 32) {
+                for (int c = 0; c < D / 2; c += 32) {   // this thread's half of the O row
                     uint32_t o[32];
-                    tmem_ld32(lane_base + kColO + c, o);
+                    tmem_ld16x2_32<D / 2>(lane_base + kColO + c, o);
                     tmem_wait_ld();
+                    reg_fence<32>(o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(lane_base + kColO + c, o);
+                    tmem_st16x2_32<D / 2>(lane_base + kColO + c, o);
                 }
                 tmem_wait_st();
             }
-            if (r == 0) MODA_TRF(9, i);
+            if (tr) MODA_TRF(9, i);
             float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            uint32_t pk[64];
+            uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
+            for (int c = 0; c < 32; ++c) {
                 const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -m);
                 const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m);
                 float p0, p1;
@@ -382,30 +410,35 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 rs4[c & 3] += p0 + p1;
                 pk[c] = pack_bf16(p0, p1);
             }
-            const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-            l += rs;
-            if (r == 0) MODA_TRF(10, i);
-            tmem_st32(s_addr, pk);
-            tmem_st32(s_addr + 32, pk + 32);
+            l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+            if (tr) MODA_TRF(10, i);
+            if (tr2) MODA_TRF(14, i);
+            // P columns c0/2 .. c0/2+31 (bf16 pairs) over the S columns this
+            // warp has already read (its own loads completed above)
+            __syncwarp();
+            tmem_st16x2_32<32>(s_addr, pk);
             tmem_wait_st();
-            if (r == 0) MODA_TRF(11, i);
+            if (tr) MODA_TRF(11, i);
             tc_fence_before();
-            mbar_arrive(&bars[kPReady + sb]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kPReady + sb]);
+            if (tr2) MODA_TRF(15, i);
         }
         // ---------------------------------------------------- epilogue ------
-        if (ok) ok = mbar_wait(&bars[kOFinal], 0, a.status, abort_flag);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFinal], 0, a.status, abort_flag));
+        const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
         if (ok) {
             tc_fence_after();
-            uint32_t o[D];
+            uint32_t o[D / 2];
 #pragma unroll
-            for (int c = 0; c < D; c += 32) tmem_ld32(lane_base + kColO + c, o + c);
+            for (int c = 0; c < D / 2; c += 32) tmem_ld16x2_32<D / 2>(lane_base + kColO + c, o + c);
             tmem_wait_ld();
             if (row_real && t_row < a.T) {
-                const float inv = 1.0f / l;
+                const float inv = 1.0f / l_row;
                 const size_t qrow = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T + t_row;
-                uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D);
+                uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + half * (D / 2));
 #pragma unroll
-                for (int c = 0; c < D; c += 8) {
+                for (int c = 0; c < D / 2; c += 8) {
                     uint4 v;
                     v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv, __uint_as_float(o[c + 1]) * inv);
                     v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
@@ -413,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     v.w = pack_bf16(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
                     dst[c / 8] = v;
                 }
-                a.LSE[qrow] = (m + log2f(l)) * 0.6931471805599453f;
+                if (half == 0) a.LSE[qrow] = (m + log2f(l_row)) * 0.6931471805599453f;
             }
         }
     }
