@@ -43,8 +43,10 @@ using namespace ptx;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kThreads = 192;            // warp 0 TMA, warp 1 MMA, warps 2..5 math
+constexpr int kThreads = 192;            // dq: warp 0 TMA, warp 1 MMA, warps 2..5 math
 constexpr int kMathThreads = 128;
+constexpr int kKvMathWarps = 8;          // dkdv: warps 2..9, two per TMEM lane quarter
+constexpr int kKvThreads = 64 + 32 * kKvMathWarps;
 constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -146,7 +148,7 @@ enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 1 + kKvStages, kA_SFull = 1 + 2 
        kA_PReady = 3 + 2 * kKvStages, kA_Final = 5 + 2 * kKvStages, kA_NumBars = 6 + 2 * kKvStages };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant__ DkdvArgs a) {
+__global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_constant__ DkdvArgs a) {
     using Lay = DkdvLayout<D>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -175,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[kA_SFull + s], 1);
-            mbar_init(&bars[kA_PReady + s], kMathThreads);
+            mbar_init(&bars[kA_PReady + s], kKvMathWarps);   // one arrive per math warp
         }
         mbar_init(&bars[kA_Final], 1);
         *abort_flag = 0;
@@ -276,88 +278,131 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             umma_commit_elect(&bars[kA_Final]);
         }
     } else {
+        // Math warps 2..9: two per TMEM lane quarter, each on 16 key rows;
+        // threads t and t + 16 of a warp share a key row and hold query
+        // columns [0, 32) and [32, 64) of the block (16x32bx2 TMEM shapes).
         const int quarter = warp & 3;
-        const int kr = quarter * 32 + lane;               // key row within the tile
+        const int sub = (warp - 2) >> 2;
+        const int half = lane >> 4;
+        const int kr = quarter * 32 + sub * 16 + (lane & 15);   // key row within the tile
         const int k = kt * BN + kr;
-        const int mt = threadIdx.x - 64;                  // 0..127 among the math threads
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int c0 = half * 32;                          // first query column of this thread
+        const int mt = threadIdx.x - 64;                   // 0..255 among the math threads
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
         const float sl2 = a.scale_log2;
+        // Row statistics (LSE in base 2, D) of a query block: threads mt < 64
+        // fetch one column each, one block ahead, so the global-load latency
+        // hides behind the current block's work.
+        float lse_n = INFINITY, d_n = 0.0f;
+        auto fetch_stats = [&](int itn) {
+            const int gn = itn / nqb;
+            const int t = (qb0 + (itn - gn * nqb)) * kKvBQ + mt;
+            const size_t qrow = (static_cast<size_t>(b) * a.Hq + hk * a.G + gn) * a.T + t;
+            lse_n = t < a.T ? a.LSE[qrow] * kLog2e : INFINITY;
+            d_n = t < a.T ? a.Drow[qrow] : 0.0f;
+        };
+        if (mt < kKvBQ && n_it > 0) fetch_stats(0);
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int g = it / nqb;
             const int qb = qb0 + (it - g * nqb);
             const int buf = it & 1;
-            const size_t qrow0 = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T;
             float* sbuf = stat + buf * 128;
             if (mt < kKvBQ) {
-                const int t = qb * kKvBQ + mt;
-                sbuf[mt] = t < a.T ? a.LSE[qrow0 + t] * kLog2e : INFINITY;
-                sbuf[64 + mt] = t < a.T ? a.Drow[qrow0 + t] : 0.0f;
+                sbuf[mt] = lse_n;
+                sbuf[64 + mt] = d_n;
+                if (it + 1 < n_it) fetch_stats(it + 1);
             }
-            named_bar_sync(1, kMathThreads);
+            named_bar_sync(1, 32 * kKvMathWarps);
             if (mt == 0) MODA_TR(4, it);
-            if (!mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status,
+                                                   abort_flag))) { ok = false; break; }
             if (mt == 0) MODA_TR(5, it);
             tc_fence_after();
             const int tq0 = qb * kKvBQ;
             const bool diag = a.causal && tq0 < kt * BN + BN;   // some key after some query
-            uint32_t s[64], dp[64], pk[32], dk[32];
-            tmem_ld32(lane_base + buf * 64, s);
-            tmem_ld32(lane_base + buf * 64 + 32, s + 32);
-            tmem_ld32(lane_base + 128 + buf * 64, dp);
-            tmem_ld32(lane_base + 128 + buf * 64 + 32, dp + 32);
+            uint32_t s[32], dp[32], pk[16], dk[16];
+            tmem_ld16x2_32<32>(lane_base + buf * 64, s);
+            tmem_ld16x2_32<32>(lane_base + 128 + buf * 64, dp);
             tmem_wait_ld();
+            reg_fence<32>(s);
+            reg_fence<32>(dp);
             if (mt == 0) MODA_TR(6, it);
-            // visible columns c >= k - tq0 on the diagonal blocks; selects, no
-            // branch per element (masked: score -inf, dP = D, so P = dS = 0)
-            const int vlo = diag ? k - tq0 : 0;
-            const float4* sl4 = reinterpret_cast<const float4*>(sbuf);
-            const float4* sd4 = reinterpret_cast<const float4*>(sbuf + 64);
+            const float4* sl4 = reinterpret_cast<const float4*>(sbuf + c0);
+            const float4* sd4 = reinterpret_cast<const float4*>(sbuf + 64 + c0);
+            if (!diag) {                   // every column visible (CTA-uniform branch)
 #pragma unroll
-            for (int e = 0; e < 64; e += 4) {
-                const float4 l4 = sl4[e / 4];
-                const float4 d4 = sd4[e / 4];
-                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
-                float p4[4], g4[4];
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 l4 = sl4[e / 4];
+                    const float4 d4 = sd4[e / 4];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float p4[4], g4[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = e + u;
-                    const bool vis = c >= vlo;
-                    const float sv = vis ? __uint_as_float(s[c]) : -INFINITY;
-                    const float dv = vis ? __uint_as_float(dp[c]) : dvv[u];
-                    p4[u] = ex2(fmaf(sv, sl2, -lv[u]));
-                    g4[u] = p4[u] * (dv - dvv[u]);
+                    for (int u = 0; u < 4; ++u) {
+                        p4[u] = ex2(fmaf(__uint_as_float(s[e + u]), sl2, -lv[u]));
+                        g4[u] = p4[u] * (__uint_as_float(dp[e + u]) - dvv[u]);
+                    }
+                    pk[e / 2] = pack_bf16(p4[0], p4[1]);
+                    pk[e / 2 + 1] = pack_bf16(p4[2], p4[3]);
+                    dk[e / 2] = pack_bf16(g4[0], g4[1]);
+                    dk[e / 2 + 1] = pack_bf16(g4[2], g4[3]);
                 }
-                pk[e / 2] = pack_bf16(p4[0], p4[1]);
-                pk[e / 2 + 1] = pack_bf16(p4[2], p4[3]);
-                dk[e / 2] = pack_bf16(g4[0], g4[1]);
-                dk[e / 2 + 1] = pack_bf16(g4[2], g4[3]);
+            } else {
+                // visible columns c >= k - tq0; selects, no branch per element
+                // (masked: score -inf, dP = D, so P = dS = 0)
+                const int vlo = k - tq0 - c0;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 l4 = sl4[e / 4];
+                    const float4 d4 = sd4[e / 4];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float p4[4], g4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = e + u;
+                        const bool vis = c >= vlo;
+                        const float sv = vis ? __uint_as_float(s[c]) : -INFINITY;
+                        const float dv = vis ? __uint_as_float(dp[c]) : dvv[u];
+                        p4[u] = ex2(fmaf(sv, sl2, -lv[u]));
+                        g4[u] = p4[u] * (dv - dvv[u]);
+                    }
+                    pk[e / 2] = pack_bf16(p4[0], p4[1]);
+                    pk[e / 2 + 1] = pack_bf16(p4[2], p4[3]);
+                    dk[e / 2] = pack_bf16(g4[0], g4[1]);
+                    dk[e / 2 + 1] = pack_bf16(g4[2], g4[3]);
+                }
             }
             if (mt == 0) MODA_TR(7, it);
-            tmem_st32(lane_base + buf * 64, pk);
-            tmem_st32(lane_base + 128 + buf * 64, dk);
+            // P^T and dS^T (bf16 pairs) over the columns this warp has read
+            __syncwarp();
+            tmem_st16x2_16<16>(lane_base + buf * 64, pk);
+            tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
             tmem_wait_st();
             if (mt == 0) MODA_TR(8, it);
             tc_fence_before();
-            mbar_arrive(&bars[kA_PReady + buf]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kA_PReady + buf]);
         }
-        if (ok) ok = mbar_wait(&bars[kA_Final], 0, a.status, abort_flag);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_Final], 0, a.status, abort_flag));
         if (ok) {
             tc_fence_after();
-            // dK (scaled) then dV, one row of D values at a time
+            // dK (scaled) then dV; this thread writes columns [half*D/2, (half+1)*D/2)
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                uint32_t gr[D];
+                uint32_t gr[D / 2];
 #pragma unroll
-                for (int c = 0; c < D; c += 32) tmem_ld32(lane_base + (which ? 256 : 384) + c, gr + c);
+                for (int c = 0; c < D / 2; c += 32)
+                    tmem_ld16x2_32<D / 2>(lane_base + (which ? 256 : 384) + c, gr + c);
                 tmem_wait_ld();
+                reg_fence<D / 2>(gr);
                 if (k < a.T) {
                     const size_t row = static_cast<size_t>(bh) * a.T + k;
-                    uint4* dst = reinterpret_cast<uint4*>((which ? a.dV : a.dK) + row * D);
+                    uint4* dst = reinterpret_cast<uint4*>((which ? a.dV : a.dK) + row * D + half * (D / 2));
                     const float sc = which ? 1.0f : a.scale;
 #pragma unroll
-                    for (int c = 0; c < D; c += 8) {
+                    for (int c = 0; c < D / 2; c += 8) {
                         uint4 u;
                         u.x = pack_bf16(__uint_as_float(gr[c]) * sc, __uint_as_float(gr[c + 1]) * sc);
                         u.y = pack_bf16(__uint_as_float(gr[c + 2]) * sc, __uint_as_float(gr[c + 3]) * sc);
@@ -808,7 +853,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
                                       (int)smem)) != cudaSuccess)
             return e;
         const long long grid = (long long)p.B * p.Hk * A.n_kt;
-        dkdv_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(A);
+        dkdv_kernel<D><<<(unsigned)grid, kKvThreads, smem, stream>>>(A);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         phase_mark(2, stream);
     }

@@ -281,6 +281,20 @@ __device__ __forceinline__ void tmem_st16x2_32(uint32_t taddr, const uint32_t* r
         : "memory");
 }
 
+// Half-row store of 16 columns (16x32bx2, 16 repetitions): thread t < 16
+// writes lane (lane of taddr) + t, columns [c, c + 16); thread t >= 16 writes
+// lane (lane of taddr) + t - 16, columns [c + SPLIT, c + SPLIT + 16).
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st16x2_16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %17, "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "n"(SPLIT)
+        : "memory");
+}
+
 // Orders every later use of r[0..N) after the preceding tcgen05.wait::ld: the
 // registers a tcgen05.ld writes are only valid after that wait, which the
 // compiler cannot see, so each gets an empty asm that "redefines" it.
