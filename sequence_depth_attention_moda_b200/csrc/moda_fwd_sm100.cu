@@ -66,7 +66,7 @@ constexpr int kVStages = MODA_FWD_VSTAGES;   // V ring: a stage frees when PV_i 
 constexpr int kSoftmaxWarps = 8;             // warps 2..9
 constexpr int kVWarp = 2 + kSoftmaxWarps;    // V producer
 constexpr int kThreads = 32 * (kVWarp + 1);
-constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLazyLimit = 1024.0f;     // largest half-row sum of p kept without a rescale
 constexpr uint32_t kSlabBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBufs = 3;            // S / P buffers in TMEM
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             tmem_wait_ld();
             reg_fence<64>(sr);
             if (tr) MODA_TRF(7, i);
-            // masks, then the row max as four independent partial maxima
+            // masks: invisible scores become -inf (p = 0)
             if (i < n_seq) {
                 const int kb = i * BN + c0;
                 const int lim = a.causal ? t_row : a.T - 1;   // last visible key
@@ -352,21 +352,54 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 for (int c = 0; c < 64; ++c)
                     if (c < lo || c >= hi) sr[c] = __float_as_uint(-INFINITY);
             }
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            // Row max of this block (both halves of the row), base 2.
+            auto block_max = [&]() -> float {
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 64; c += 8) {
+                for (int c = 0; c < 64; c += 8) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    mx4[u] = fmax3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
-            }
-            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            const float m_new = fmaxf(m, mx * sl2);
+                    for (int u = 0; u < 4; ++u)
+                        mx4[u] = fmax3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
+                }
+                float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                return mx * sl2;
+            };
+            // p = 2^(s*sl2 - m) for this thread's 64 columns, packed to bf16;
+            // returns this half-row's sum.
+            uint32_t pk[32];
+            auto exp_block = [&]() -> float {
+                float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -m);
+                    const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m);
+                    float p0, p1;
+                    if ((c & 3) < 4 - MODA_FWD_SWEXP) {     // MUFU
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                    } else {                                 // FMA pipe
+                        p0 = ex2_fma(x0);
+                        p1 = ex2_fma(x1);
+                    }
+                    rs4[c & 3] += p0 + p1;
+                    pk[c] = pack_bf16(p0, p1);
+                }
+                return (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+            };
+            // The online softmax is exact for any reference point m, so a
+            // block is first exponentiated against the running m without
+            // computing its max.  Only when some p could exceed 2^10 (a
+            // half-row sum above 2^10 is necessary for that, and catches
+            // overflow too) does the warp take the block max, rescale O and
+            // l to the new reference and recompute P.  The first block sets m.
+            if (i == 0) m = block_max();
             if (tr) MODA_TRF(8, i);
             if (tr2) MODA_TRF(13, i);
-            if (i == 0) {
-                m = m_new;
-            } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
+            float rs = exp_block();
+            if (tr) MODA_TRF(9, i);
+            if (i > 0 && __any_sync(0xffffffffu, !(rs <= kLazyLimit))) {
+                const float m_new = fmaxf(m, block_max());
                 // O must hold P_{i-1} V_{i-1} before it is rescaled: wait for
                 // the V-stage release PV_{i-1} commits.  S_i was issued after
                 // PV_{i-2}, so at most PV_{i-1} is in flight, and PV_{i+2}
@@ -391,26 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     tmem_st16x2_32<D / 2>(lane_base + kColO + c, o);
                 }
                 tmem_wait_st();
+                rs = exp_block();
             }
-            if (tr) MODA_TRF(9, i);
-            float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -m);
-                const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m);
-                float p0, p1;
-                if ((c & 3) < 4 - MODA_FWD_SWEXP) {     // MUFU
-                    p0 = ex2(x0);
-                    p1 = ex2(x1);
-                } else {                                 // FMA pipe
-                    p0 = ex2_fma(x0);
-                    p1 = ex2_fma(x1);
-                }
-                rs4[c & 3] += p0 + p1;
-                pk[c] = pack_bf16(p0, p1);
-            }
-            l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+            l += rs;
             if (tr) MODA_TRF(10, i);
             if (tr2) MODA_TRF(14, i);
             // P columns c0/2 .. c0/2+31 (bf16 pairs) over the S columns this
