@@ -110,6 +110,12 @@ __global__ void __launch_bounds__(256) rowdot_kernel(long long nrows,
 // Query blocks are 64 rows, so S^T and dP^T are double-buffered in TMEM:
 //   S^T0 [0,64) S^T1 [64,128) | dP^T0 [128,192) dP^T1 [192,256) |
 //   dV [256, 256+D) | dK [384, 384+D)
+// The per-query statistics enter through the MMAs: one more K=16 step per
+// product multiplies a constant key-side tile whose rows are (1, 1, 0, ...)
+// by query-side rows (-b_hi, -b_lo, 0, ...), where b_hi + b_lo is LSE / scale
+// (for S^T) or D (for dP^T) split into two bf16 parts.  TMEM then holds
+// s - LSE/scale and dP - D, and the math warps need no statistics at all:
+// P^T = 2^(scale*log2(e) * S'^T), dS^T = P^T * dP'^T.
 struct DkdvArgs {
     TmaMap tk, tv, tq, tdo;
     const float* LSE;
@@ -124,7 +130,7 @@ struct DkdvArgs {
 
 constexpr int kKvBQ = 64;               // query rows per iteration
 #ifndef MODA_DKDV_STAGES
-#define MODA_DKDV_STAGES 4
+#define MODA_DKDV_STAGES 3
 #endif
 constexpr int kKvStages = MODA_DKDV_STAGES;   // Q/dO ring depth
 constexpr uint32_t kKvSlab = 64 * 128;
@@ -138,8 +144,12 @@ struct DkdvLayout {
     static constexpr uint32_t kV = kKTile;
     static constexpr uint32_t kQ = 2 * kKTile;                  // kKvStages stages
     static constexpr uint32_t kDO = kQ + kKvStages * kQTile;    // kKvStages stages
-    static constexpr uint32_t kStat = kDO + kKvStages * kQTile; // 2 x (lse2[64], D[64]) floats
-    static constexpr uint32_t kBar = kStat + 1024;
+    // bias rows of each stage (64 query rows x 128 B, 128-byte swizzle; only
+    // the first 32 B of a row are read): LSE / scale, then D
+    static constexpr uint32_t kAL = kDO + kKvStages * kQTile;
+    static constexpr uint32_t kAD = kAL + kKvStages * kKvSlab;
+    static constexpr uint32_t kAA = kAD + kKvStages * kKvSlab;  // key-side (1, 1, 0, ...) rows, 128 x 128 B
+    static constexpr uint32_t kBar = kAA + kSlabBytes;
     static constexpr uint32_t kBytes = kBar + 256;
     static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
 };
@@ -156,7 +166,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kA_NumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    float* stat = reinterpret_cast<float*>(smem + Lay::kStat);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -183,6 +192,14 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         *abort_flag = 0;
         fence_mbarrier_init();
     }
+    // key-side bias rows: elements 0 and 1 are 1.0, the rest of the first 32 B
+    // zero (16-byte chunks c = 0, 1 of row r sit at chunk c ^ (r & 7))
+    for (int i = threadIdx.x; i < 2 * BN; i += kKvThreads) {
+        const int r = i >> 1, c = i & 1;
+        *reinterpret_cast<uint4*>(smem + Lay::kAA + r * 128 + ((c ^ (r & 7)) << 4)) =
+            c == 0 ? make_uint4(pack_bf16(1.0f, 1.0f), 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(tmem_holder, kTmemCols);
         tmem_relinquish();
@@ -193,6 +210,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
     const uint32_t tmem = *tmem_holder;
 
     if (warp == 0) {
+        // producer, whole warp: per query block, the bias rows (lanes write
+        // rows lane and lane + 32), then Q and dO by TMA (lane 0)
         if (lane == 0) {
             prefetch_tmap(&a.tk); prefetch_tmap(&a.tv); prefetch_tmap(&a.tq); prefetch_tmap(&a.tdo);
             mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * Lay::kKTile);
@@ -200,16 +219,45 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 tma_load_3d(smem + Lay::kK + s * kSlabBytes, &a.tk, &bars[kA_KVFull], s * 64, kt * BN, bh);
                 tma_load_3d(smem + Lay::kV + s * kSlabBytes, &a.tv, &bars[kA_KVFull], s * 64, kt * BN, bh);
             }
-            int issued = 0;
-            for (int it = 0; it < n_it; ++it) {
-                const int st = it % kKvStages;
-                if (it >= kKvStages &&
-                    !mbar_wait(&bars[kA_QEmpty + st], ((it / kKvStages) - 1) & 1, a.status, abort_flag))
-                    break;
-                MODA_TR(9, it);
-                const int g = it / nqb;
-                const int qb = qb0 + (it - g * nqb);
-                const int qh = b * a.Hq + hk * a.G + g;
+        }
+        const float inv_scale = 1.0f / a.scale;
+        int issued = 0;
+        for (int it = 0; it < n_it; ++it) {
+            const int st = it % kKvStages;
+            if (it >= kKvStages &&
+                !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + st], ((it / kKvStages) - 1) & 1,
+                                                   a.status, abort_flag)))
+                break;
+            if (lane == 0) MODA_TR(9, it);
+            const int g = it / nqb;
+            const int qb = qb0 + (it - g * nqb);
+            const int qh = b * a.Hq + hk * a.G + g;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int rr = lane + 32 * h2;                 // query row of the block
+                const int t = qb * kKvBQ + rr;
+                const size_t qrow = static_cast<size_t>(qh) * a.T + t;
+                float lh = -INFINITY, ll = 0.0f, dh = 0.0f, dl = 0.0f;   // rows past T: p = 0
+                if (t < a.T) {
+                    const float bl = -a.LSE[qrow] * inv_scale;
+                    const float bd = -a.Drow[qrow];
+                    lh = __bfloat162float(__float2bfloat16_rn(bl));
+                    ll = bl - lh;
+                    dh = __bfloat162float(__float2bfloat16_rn(bd));
+                    dl = bd - dh;
+                }
+                const uint32_t o0 = rr * 128 + ((0 ^ (rr & 7)) << 4);
+                const uint32_t o1 = rr * 128 + ((1 ^ (rr & 7)) << 4);
+                unsigned char* al = smem + Lay::kAL + st * kKvSlab;
+                unsigned char* ad = smem + Lay::kAD + st * kKvSlab;
+                *reinterpret_cast<uint4*>(al + o0) = make_uint4(pack_bf16(lh, ll), 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(al + o1) = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(ad + o0) = make_uint4(pack_bf16(dh, dl), 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(ad + o1) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();   // generic writes -> the tensor core's reads
+            __syncwarp();
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[kA_QFull + st], 2 * Lay::kQTile);
                 for (int s = 0; s < Lay::kSlabs; ++s) {
                     tma_load_3d(smem + Lay::kQ + st * Lay::kQTile + s * kKvSlab, &a.tq,
@@ -217,8 +265,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     tma_load_3d(smem + Lay::kDO + st * Lay::kQTile + s * kKvSlab, &a.tdo,
                                 &bars[kA_QFull + st], s * 64, qb * kKvBQ, qh);
                 }
-                issued = it + 1;
             }
+            issued = it + 1;
+        }
+        if (lane == 0) {
             mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
             for (int it = max(0, issued - kKvStages); it < issued; ++it)
                 mbar_wait(&bars[kA_QFull + it % kKvStages], (it / kKvStages) & 1, a.status, abort_flag);
@@ -230,7 +280,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             const uint32_t id_g = idesc_bf16(128, D, false, true);
             const uint64_t kd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kK));
             const uint64_t vd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kV));
-            // S^T(j) = K Q_j^T and dP^T(j) = V dO_j^T into buffer j & 1.
+            const uint64_t ad0 = desc_kmajor_sw128(smem_u32(smem + Lay::kAA));
+            // S^T(j) = K Q_j^T - LSE/scale and dP^T(j) = V dO_j^T - D into buffer j & 1.
             auto issue_s = [&](int j) -> bool {
                 const int st = j % kKvStages;
                 const int buf = j & 1;
@@ -245,12 +296,16 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
                     umma_ss_elect(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
                 }
+                umma_ss_elect(tmem + buf * 64, ad0, desc_kmajor_sw128(smem_u32(smem + Lay::kAL + st * kKvSlab)),
+                              id_s, 1u);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                     const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
                     umma_ss_elect(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
                 }
+                umma_ss_elect(tmem + 128 + buf * 64, ad0,
+                              desc_kmajor_sw128(smem_u32(smem + Lay::kAD + st * kKvSlab)), id_s, 1u);
                 umma_commit_elect(&bars[kA_SFull + buf]);
                 return true;
             };
@@ -290,30 +345,11 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         const int mt = threadIdx.x - 64;                   // 0..255 among the math threads
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
         const float sl2 = a.scale_log2;
-        // Row statistics (LSE in base 2, D) of a query block: threads mt < 64
-        // fetch one column each, one block ahead, so the global-load latency
-        // hides behind the current block's work.
-        float lse_n = INFINITY, d_n = 0.0f;
-        auto fetch_stats = [&](int itn) {
-            const int gn = itn / nqb;
-            const int t = (qb0 + (itn - gn * nqb)) * kKvBQ + mt;
-            const size_t qrow = (static_cast<size_t>(b) * a.Hq + hk * a.G + gn) * a.T + t;
-            lse_n = t < a.T ? a.LSE[qrow] * kLog2e : INFINITY;
-            d_n = t < a.T ? a.Drow[qrow] : 0.0f;
-        };
-        if (mt < kKvBQ && n_it > 0) fetch_stats(0);
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int g = it / nqb;
             const int qb = qb0 + (it - g * nqb);
             const int buf = it & 1;
-            float* sbuf = stat + buf * 128;
-            if (mt < kKvBQ) {
-                sbuf[mt] = lse_n;
-                sbuf[64 + mt] = d_n;
-                if (it + 1 < n_it) fetch_stats(it + 1);
-            }
-            named_bar_sync(1, 32 * kKvMathWarps);
             if (mt == 0) MODA_TR(4, it);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status,
                                                    abort_flag))) { ok = false; break; }
@@ -322,56 +358,32 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             const int tq0 = qb * kKvBQ;
             const bool diag = a.causal && tq0 < kt * BN + BN;   // some key after some query
             uint32_t s[32], dp[32], pk[16], dk[16];
-            tmem_ld16x2_32<32>(lane_base + buf * 64, s);
-            tmem_ld16x2_32<32>(lane_base + 128 + buf * 64, dp);
+            tmem_ld16x2_32<32>(lane_base + buf * 64, s);          // s - LSE/scale
+            tmem_ld16x2_32<32>(lane_base + 128 + buf * 64, dp);   // dP - D
             tmem_wait_ld();
             reg_fence<32>(s);
             reg_fence<32>(dp);
             if (mt == 0) MODA_TR(6, it);
-            const float4* sl4 = reinterpret_cast<const float4*>(sbuf + c0);
-            const float4* sd4 = reinterpret_cast<const float4*>(sbuf + 64 + c0);
             if (!diag) {                   // every column visible (CTA-uniform branch)
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    const float4 l4 = sl4[e / 4];
-                    const float4 d4 = sd4[e / 4];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float p4[4], g4[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        p4[u] = ex2(fmaf(__uint_as_float(s[e + u]), sl2, -lv[u]));
-                        g4[u] = p4[u] * (__uint_as_float(dp[e + u]) - dvv[u]);
-                    }
-                    pk[e / 2] = pack_bf16(p4[0], p4[1]);
-                    pk[e / 2 + 1] = pack_bf16(p4[2], p4[3]);
-                    dk[e / 2] = pack_bf16(g4[0], g4[1]);
-                    dk[e / 2 + 1] = pack_bf16(g4[2], g4[3]);
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = ex2(__uint_as_float(s[e]) * sl2);
+                    const float p1 = ex2(__uint_as_float(s[e + 1]) * sl2);
+                    pk[e / 2] = pack_bf16(p0, p1);
+                    dk[e / 2] = pack_bf16(p0 * __uint_as_float(dp[e]), p1 * __uint_as_float(dp[e + 1]));
                 }
             } else {
-                // visible columns c >= k - tq0; selects, no branch per element
-                // (masked: score -inf, dP = D, so P = dS = 0)
+                // visible columns c >= k - tq0; a select, no branch per element
+                // (masked: score -inf, so P = dS = 0)
                 const int vlo = k - tq0 - c0;
 #pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    const float4 l4 = sl4[e / 4];
-                    const float4 d4 = sd4[e / 4];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float p4[4], g4[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c = e + u;
-                        const bool vis = c >= vlo;
-                        const float sv = vis ? __uint_as_float(s[c]) : -INFINITY;
-                        const float dv = vis ? __uint_as_float(dp[c]) : dvv[u];
-                        p4[u] = ex2(fmaf(sv, sl2, -lv[u]));
-                        g4[u] = p4[u] * (dv - dvv[u]);
-                    }
-                    pk[e / 2] = pack_bf16(p4[0], p4[1]);
-                    pk[e / 2 + 1] = pack_bf16(p4[2], p4[3]);
-                    dk[e / 2] = pack_bf16(g4[0], g4[1]);
-                    dk[e / 2 + 1] = pack_bf16(g4[2], g4[3]);
+                for (int e = 0; e < 32; e += 2) {
+                    const float s0 = e >= vlo ? __uint_as_float(s[e]) : -INFINITY;
+                    const float s1 = e + 1 >= vlo ? __uint_as_float(s[e + 1]) : -INFINITY;
+                    const float p0 = ex2(s0 * sl2);
+                    const float p1 = ex2(s1 * sl2);
+                    pk[e / 2] = pack_bf16(p0, p1);
+                    dk[e / 2] = pack_bf16(p0 * __uint_as_float(dp[e]), p1 * __uint_as_float(dp[e + 1]));
                 }
             }
             if (mt == 0) MODA_TR(7, it);
