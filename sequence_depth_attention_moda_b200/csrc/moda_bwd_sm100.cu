@@ -43,7 +43,7 @@ using namespace ptx;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kThreads = 192;            // dq: warp 0 TMA, warp 1 MMA, warps 2..5 math
+constexpr int kThreads = 224;            // dq: warp 0 TMA, warps 1 and 6 MMA, warps 2..5 math
 constexpr int kMathThreads = 128;
 constexpr int kKvMathWarps = 8;          // dkdv: warps 2..9, two per TMEM lane quarter
 constexpr int kKvThreads = 64 + 32 * kKvMathWarps;
@@ -470,8 +470,7 @@ struct DqLayout {
     static constexpr uint32_t kV = kK + kDqStages * kKTile;      // kDqStages stages
     static constexpr uint32_t kDS = kV + kDqStages * kKTile;     // [128 q][64 depth] bf16, 128-B swizzle
     static constexpr uint32_t kP = kDS + kSlabBytes;
-    static constexpr uint32_t kStage = kP + kSlabBytes;          // [64 rows][D] bf16 x 2 (dKd, dVd)
-    static constexpr uint32_t kBar = kStage + 2 * 64 * D * 2;
+    static constexpr uint32_t kBar = kP + kSlabBytes;
     static constexpr uint32_t kBytes = kBar + 256;
     static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
 };
@@ -579,9 +578,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             for (int i = max(0, issued - kDqStages); i < issued; ++i)
                 mbar_wait(&bars[kB_KVFull + i % kDqStages], (i / kDqStages) & 1, a.status, abort_flag);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer --
-        // whole warp, converged: warp-uniform waits, one elected lane issues
+    } else if (warp == 1 || warp == 6) {
+        // ------------------------------------------------------ MMA issuers -
+        // Two warps on different sub-partitions share the issue work: warp 6
+        // the score products S(j), dP(j); warp 1 dQ(i) and the depth
+        // gradients.  Each runs converged (warp-uniform waits, one elected
+        // lane issues); a commit tracks only its own warp's MMAs, and the
+        // waits below order every TMEM reuse across the two.
         {
             const uint32_t id_seq = idesc_bf16(128, kDqBN, false, false);
             const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
@@ -618,47 +621,56 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 umma_commit_elect(&bars[kB_SFull + buf]);
                 return true;
             };
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag)) && issue_s(0);
-            for (int i = 0; ok && i < nb; ++i) {
-                // the next block's scores first: its buffer was released when
-                // the math warps finished block i-1 (waited below last round)
-                MODA_TRQ(0, i);
-                if (i + 1 < nb && !issue_s(i + 1)) { ok = false; break; }
-                MODA_TRQ(1, i);
-                const int st = i % kDqStages;
-                const int buf = i & 1;
-                const bool seq = i < n_seq;
-                const int n = seq ? kDqBN : a.dep_rows;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
-                MODA_TRQ(2, i);
-                tc_fence_after();
-                const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
-                if (n == kDqBN) {
-#pragma unroll
-                    for (int kk = 0; kk < kDqBN / 16; ++kk)
-                        umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
-                                (i > 0 || kk > 0) ? 1u : 0u);
-                } else {
-                    for (int kk = 0; kk < n / 16; ++kk)
-                        umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
-                                (i > 0 || kk > 0) ? 1u : 0u);
+            if (warp == 6) {
+                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag));
+                for (int j = 0; ok && j < nb; ++j) {
+                    // buffer j & 1 last held dS(j-2), which dQ(j-2) reads: wait
+                    // until that has completed (its K/V-stage release)
+                    if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVEmpty + (j - 2) % kDqStages],
+                                                                     ((j - 2) / kDqStages) & 1, a.status,
+                                                                     abort_flag))) { ok = false; break; }
+                    MODA_TRQ(0, j);
+                    if (!issue_s(j)) { ok = false; break; }
+                    MODA_TRQ(1, j);
                 }
-                if (!seq) {
-#pragma unroll
-                    for (int kk = 0; kk < BM / 16; ++kk) {
-                        umma_ss_elect(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
-                                desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
-                        umma_ss_elect(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
-                                desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+            } else {
+                bool ok = true;
+                for (int i = 0; ok && i < nb; ++i) {
+                    const int st = i % kDqStages;
+                    const int buf = i & 1;
+                    const bool seq = i < n_seq;
+                    const int n = seq ? kDqBN : a.dep_rows;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
+                    MODA_TRQ(2, i);
+                    tc_fence_after();
+                    const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
+                    if (n == kDqBN) {
+    #pragma unroll
+                        for (int kk = 0; kk < kDqBN / 16; ++kk)
+                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
+                                    (i > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        for (int kk = 0; kk < n / 16; ++kk)
+                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
+                                    (i > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit_elect(&bars[kB_DDFull]);
+                    if (!seq) {
+    #pragma unroll
+                        for (int kk = 0; kk < BM / 16; ++kk) {
+                            umma_ss_elect(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
+                                    desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                            umma_ss_elect(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
+                                    desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit_elect(&bars[kB_DDFull]);
+                    }
+                    umma_commit_elect(&bars[kB_KVEmpty + st]);
+                    MODA_TRQ(3, i);
                 }
-                umma_commit_elect(&bars[kB_KVEmpty + st]);
-                MODA_TRQ(3, i);
+                umma_commit_elect(&bars[kB_Final]);
             }
-            umma_commit_elect(&bars[kB_Final]);
         }
-    } else {
+    } else if (warp <= 5) {
         // ------------------------------------------------------ math --------
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
@@ -674,12 +686,11 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const float sl2 = a.scale_log2;
         unsigned char* sDS = smem + Lay::kDS;
         unsigned char* sP = smem + Lay::kP;
-        __nv_bfloat16* stK = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kStage);
-        __nv_bfloat16* stV = stK + 64 * D;
         const size_t dep_base = (static_cast<size_t>(bh) * a.T + t0) * a.L;  // first depth row of the tile
 
-        // dKd / dVd of depth block jd: TMEM lane = d index, column = depth row.
-        // Transposed through shared memory, then 16-byte row stores.
+        // dKd / dVd of depth block jd: TMEM lane = d index, column = depth row,
+        // so for each depth row the four warps store 128 consecutive d values
+        // (64 contiguous bytes per warp) straight to global memory.
         auto depth_epilogue = [&](int jd) {
             uint32_t xk[64], xv[64];
             tmem_ld32(lane_base + kColDKd, xk);
@@ -687,25 +698,20 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             tmem_ld32(lane_base + kColDVd, xv);
             tmem_ld32(lane_base + kColDVd + 32, xv + 32);
             tmem_wait_ld();
-            named_bar_sync(1, kMathThreads);             // staging free (previous readers done)
+            reg_fence<64>(xk);
+            reg_fence<64>(xv);
             if (r < D) {
+                const int row0 = jd * a.dep_rows;
+                const int nvalid = min(a.dep_rows, dep_total - row0);
+                __nv_bfloat16* gk = a.dKd + (dep_base + row0) * D + r;
+                __nv_bfloat16* gv = a.dVd + (dep_base + row0) * D + r;
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
-                    stK[c * D + r] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
-                    stV[c * D + r] = __float2bfloat16_rn(__uint_as_float(xv[c]));
+                    if (c < nvalid) {
+                        gk[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
+                        gv[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xv[c]));
+                    }
                 }
-            }
-            named_bar_sync(1, kMathThreads);
-            const int row0 = jd * a.dep_rows;
-            const int nvalid = min(a.dep_rows, dep_total - row0);
-            constexpr int kVecPerRow = D / 8;
-            const uint4* sk4 = reinterpret_cast<const uint4*>(stK);
-            const uint4* sv4 = reinterpret_cast<const uint4*>(stV);
-            uint4* gk = reinterpret_cast<uint4*>(a.dKd + (dep_base + row0) * D);
-            uint4* gv = reinterpret_cast<uint4*>(a.dVd + (dep_base + row0) * D);
-            for (int u = mt; u < nvalid * kVecPerRow; u += kMathThreads) {
-                gk[u] = sk4[u];
-                gv[u] = sv4[u];
             }
         };
 
