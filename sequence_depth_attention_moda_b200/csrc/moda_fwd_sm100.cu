@@ -102,8 +102,36 @@ struct FwdArgs {
     int B, Hq, Hk, T, L, G, Tq, n_qt, dep_rows;
     int causal;       // 0: every row sees keys 0..T-1
     int win_lo;       // first visible depth row of a token
+    int n_tiles;      // B * Hk * n_qt query tiles, longest first
     float scale_log2;
 };
+
+// Query tile `idx` of the longest-first order: the last query tiles of every
+// (b, hk) come first.  Blocks are n_seq key blocks, then the depth blocks.
+struct FwdTile {
+    int b, hk, bh, t0, t_end, n_seq, nb;
+};
+// Tile of CTA c in round r of a persistent launch with G CTAs: rounds of G
+// tiles of the longest-first order, dealt alternately forwards and backwards
+// (a snake), so every CTA's total stays close to the mean.  Only the last
+// round can run past n_tiles; the caller skips such slots.
+__device__ __forceinline__ int snake_tile(int r, int c, int G) {
+    return r * G + ((r & 1) ? G - 1 - c : c);
+}
+__device__ __forceinline__ FwdTile fwd_tile(const FwdArgs& a, int idx) {
+    const int nbh = a.B * a.Hk;
+    FwdTile t;
+    const int qt = a.n_qt - 1 - idx / nbh;
+    t.bh = idx % nbh;
+    t.b = t.bh / a.Hk;
+    t.hk = t.bh - t.b * a.Hk;
+    t.t0 = qt * a.Tq;
+    t.t_end = min(t.t0 + a.Tq, a.T);                   // one past the last real token
+    t.n_seq = ((a.causal ? t.t_end : a.T) - 1) / BN + 1;
+    const int n_dep = a.L > 0 ? ((t.t_end - t.t0) * a.L + a.dep_rows - 1) / a.dep_rows : 0;
+    t.nb = t.n_seq + n_dep;
+    return t;
+}
 
 template <int D>
 struct Layout {
@@ -122,7 +150,7 @@ struct Layout {
 // Barrier slots.
 enum { kQFull = 0, kKFull = 1, kVFull = kKFull + kKStages, kVEmpty = kVFull + kVStages,
        kSFull = kVEmpty + kVStages, kPReady = kSFull + kSBufs, kOFinal = kPReady + kSBufs,
-       kNumBars = kOFinal + 1 };
+       kOFree = kOFinal + 1, kNumBars = kOFree + 1 };
 static_assert(kKStages == kSBufs, "a K stage is released by the score barrier of its S buffer");
 
 template <int D>
@@ -141,18 +169,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Longest tiles first: block 0.. take the last query tiles of every head.
-    const int nbh = a.B * a.Hk;
-    const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / nbh;
-    const int bh = static_cast<int>(blockIdx.x) % nbh;
-    const int b = bh / a.Hk;
-    const int hk = bh - b * a.Hk;
-    const int t0 = qt * a.Tq;
+    // Persistent: CTA c takes tile snake_tile(r, c, gridDim.x) of every round
+    // r.  Ring stages and barrier phases follow a per-CTA running block count j
+    // over all of its tiles, which every role computes alike.
     const int R = a.G * a.Tq;
-    const int t_end = min(t0 + a.Tq, a.T);           // one past the last real token
-    const int n_seq = ((a.causal ? t_end : a.T) - 1) / BN + 1;
-    const int n_dep = a.L > 0 ? ((t_end - t0) * a.L + a.dep_rows - 1) / a.dep_rows : 0;
-    const int nb = n_seq + n_dep;
+    const int cta = static_cast<int>(blockIdx.x);
+    const int tstep = static_cast<int>(gridDim.x);
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kQFull], 1);
@@ -166,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             mbar_init(&bars[kPReady + s], kSoftmaxWarps);   // one arrive per softmax warp
         }
         mbar_init(&bars[kOFinal], 1);
+        mbar_init(&bars[kOFree], kSoftmaxWarps);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -201,32 +224,48 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             const void* m_dep = is_k ? static_cast<const void*>(&a.tkd) : static_cast<const void*>(&a.tvd);
             prefetch_tmap(m_seq);
             if (a.L > 0) prefetch_tmap(m_dep);
-            if (is_k) {
-                prefetch_tmap(&a.tq);
-                const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
-                mbar_arrive_expect_tx(&bars[kQFull], q_bytes);
-                for (int s = 0; s < Lay::kSlabs; ++s)
-                    tma_load_3d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, t0, b * a.Hq + hk * a.G);
-            }
-            int issued = 0;
-            for (int i = 0; i < nb; ++i) {
-                const int st = i % nst;
-                // K stage of block i-nst is free once S(i-nst) is done: that is
-                // the score barrier of its buffer (three K stages, three S
-                // buffers), so no separate commit is needed for K.
-                if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1, a.status, abort_flag))
-                    break;
-                unsigned char* dst = ring + st * Lay::kTile;
-                const bool seq = i < n_seq;
-                const int row0 = seq ? i * BN : t0 * a.L + (i - n_seq) * a.dep_rows;
-                const uint32_t bytes = Lay::kSlabs * 128u * (seq ? BN : a.dep_rows);
-                mbar_arrive_expect_tx(&full[st], bytes);
-                for (int s = 0; s < Lay::kSlabs; ++s)
-                    tma_load_3d(dst + s * kSlabBytes, seq ? m_seq : m_dep, &full[st], s * 64, row0, bh);
-                issued = i + 1;
+            if (is_k) prefetch_tmap(&a.tq);
+            const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
+            int j = 0, kt = 0, issued = 0, nq = 0;
+            bool ok = true;
+            for (int rnd = 0; ok && rnd * tstep < a.n_tiles; ++rnd) {
+                const int tile = snake_tile(rnd, cta, tstep);
+                if (tile >= a.n_tiles) continue;
+                const FwdTile T = fwd_tile(a, tile);
+                if (is_k) {
+                    // Q has one buffer: the previous tile's last score MMA must
+                    // be done before it is overwritten (the next phase of that
+                    // S buffer needs this Q, so the parity is exact)
+                    if (kt > 0 && !mbar_wait(&bars[kSFull + (j - 1) % kSBufs], ((j - 1) / kSBufs) & 1,
+                                             a.status, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&bars[kQFull], q_bytes);
+                    for (int s = 0; s < Lay::kSlabs; ++s)
+                        tma_load_3d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, T.t0,
+                                    T.b * a.Hq + T.hk * a.G);
+                    ++nq;
+                }
+                for (int i = 0; i < T.nb; ++i, ++j) {
+                    const int st = j % nst;
+                    // K stage of block j-nst is free once S(j-nst) is done: that
+                    // is the score barrier of its buffer (three K stages, three S
+                    // buffers), so no separate commit is needed for K.
+                    if (j >= nst && !mbar_wait(&empty[st], ((j / nst) - 1) & 1, a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    unsigned char* dst = ring + st * Lay::kTile;
+                    const bool seq = i < T.n_seq;
+                    const int row0 = seq ? i * BN : T.t0 * a.L + (i - T.n_seq) * a.dep_rows;
+                    const uint32_t bytes = Lay::kSlabs * 128u * (seq ? BN : a.dep_rows);
+                    mbar_arrive_expect_tx(&full[st], bytes);
+                    for (int s = 0; s < Lay::kSlabs; ++s)
+                        tma_load_3d(dst + s * kSlabBytes, seq ? m_seq : m_dep, &full[st], s * 64, row0, T.bh);
+                    issued = j + 1;
+                }
+                ++kt;
             }
             // Let every load this thread started land before the CTA retires.
-            if (is_k) mbar_wait(&bars[kQFull], 0, a.status, abort_flag);
+            if (nq > 0) mbar_wait(&bars[kQFull], (nq - 1) & 1, a.status, abort_flag);
             for (int i = max(0, issued - nst); i < issued; ++i)
                 mbar_wait(&full[i % nst], (i / nst) & 1, a.status, abort_flag);
         }
@@ -242,10 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         // Descriptors are built once; a K step adds its byte offset / 16 to
         // the 14-bit address field (shared addresses stay < 256 KB).
         const uint64_t qd0 = desc_kmajor_sw128(smem_u32(sQ));
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], 0, a.status, abort_flag));
-        // S(j) = Q K_j^T into buffer j % 3.  The buffer last held P(j-3),
-        // read by PV(j-3), which is issued before S(j) (in-order pipe).
-        auto issue_s = [&](int j) -> bool {
+        // S(j) = Q K_j^T into buffer j % 3 (i: the block's index in its tile).
+        // The buffer last held P(j-3), read by PV(j-3), which is issued before
+        // S(j) (in-order pipe).
+        auto issue_s = [&](int j, int i, const FwdTile& T) -> bool {
             const int st = j % kKStages;
             const int sb = j % kSBufs;
             if (tl) MODA_TRF(0, j);
@@ -254,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             if (tl) MODA_TRF(1, j);
             tc_fence_after();
             const uint64_t kd0 = desc_kmajor_sw128(smem_u32(sK + st * Lay::kTile));
-            const uint32_t id = j < n_seq ? id_seq : id_dep;
+            const uint32_t id = i < T.n_seq ? id_seq : id_dep;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint64_t off = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
@@ -264,8 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             if (tl) MODA_TRF(2, j);
             return true;
         };
-        // O += P(j) V_j with P read from TMEM buffer j % 3.
-        auto issue_pv = [&](int j) -> bool {
+        // O += P(j) V_j with P read from TMEM buffer j % 3; the tile's first
+        // block overwrites O.
+        auto issue_pv = [&](int j, int i, const FwdTile& T) -> bool {
             const int st = j % kVStages;
             const int sb = j % kSBufs;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kPReady + sb], (j / kSBufs) & 1, a.status,
@@ -274,17 +314,17 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status,
                                                    abort_flag))) return false;
             tc_fence_after();
-            const int krows = j < n_seq ? BN : a.dep_rows;
+            const int krows = i < T.n_seq ? BN : a.dep_rows;
             const uint64_t vd0 = desc_mnmajor_sw128(smem_u32(sV + st * Lay::kTile), kSlabBytes);
             if (krows == BN) {
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
                     umma_ts_elect(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
-                                  (j > 0 || kk > 0) ? 1u : 0u);
+                                  (i > 0 || kk > 0) ? 1u : 0u);
             } else {
                 for (int kk = 0; kk < krows / 16; ++kk)
                     umma_ts_elect(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
-                                  (j > 0 || kk > 0) ? 1u : 0u);
+                                  (i > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit_elect(&bars[kVEmpty + st]);
             if (tl) MODA_TRF(3, j);
@@ -295,13 +335,31 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         // (in-order) pipe, so it never waits for P(i); each issue blocks
         // until the shallow MMA queue has room, so this order is what keeps
         // the next scores ready when the softmax needs them.
-        if (ok) ok = issue_s(0);
-        if (ok && nb > 1) ok = issue_s(1);
-        for (int i = 0; ok && i < nb; ++i) {
-            if (i + 2 < nb && !issue_s(i + 2)) { ok = false; break; }
-            if (!issue_pv(i)) { ok = false; break; }
+        bool ok = true;
+        int j0 = 0, kt = 0;
+        for (int rnd = 0; ok && rnd * tstep < a.n_tiles; ++rnd) {
+            const int tile = snake_tile(rnd, cta, tstep);
+            if (tile >= a.n_tiles) continue;
+            const FwdTile T = fwd_tile(a, tile);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], kt & 1, a.status, abort_flag));
+            if (ok) ok = issue_s(j0, 0, T);
+            if (ok && T.nb > 1) ok = issue_s(j0 + 1, 1, T);
+            for (int i = 0; ok && i < T.nb; ++i) {
+                if (i + 2 < T.nb && !issue_s(j0 + i + 2, i + 2, T)) { ok = false; break; }
+                // the tile's first PV overwrites O: the softmax warps must have
+                // read the previous tile's O out
+                if (i == 0 && kt > 0 &&
+                    !__all_sync(0xffffffffu, mbar_wait(&bars[kOFree], (kt - 1) & 1, a.status, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                if (i == 0) tc_fence_after();
+                if (!issue_pv(j0 + i, i, T)) { ok = false; break; }
+            }
+            umma_commit_elect(&bars[kOFinal]);
+            j0 += T.nb;
+            ++kt;
         }
-        umma_commit_elect(&bars[kOFinal]);
     } else if (warp >= 2 && warp < 2 + kSoftmaxWarps) {
         // ------------------------------------------------------ softmax -----
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
@@ -310,160 +368,175 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         const int r = quarter * 32 + sub * 16 + (lane & 15);   // tile row
         const bool row_real = r < R;
         const int g = row_real ? r / a.Tq : 0;
-        const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
         const int c0 = half * 64;                     // first S column this thread holds
         const bool tr = r == 0 && half == 0;          // trace threads
         const bool tr2 = r == 32 && half == 0;        // quarter 1: the MMA warp's sub-partition
         const float sl2 = a.scale_log2;
-        float m = -INFINITY, l = 0.0f;                // l: this half's share of the row sum
         bool ok = true;
-        for (int i = 0; i < nb; ++i) {
-            const int sb = i % kSBufs;
-            if (tr) MODA_TRF(5, i);
-            // every wait result is made warp-uniform: the shuffles and the
-            // .sync.aligned TMEM accesses below need the whole warp
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + sb], (i / kSBufs) & 1, a.status,
-                                                   abort_flag))) { ok = false; break; }
-            if (tr) MODA_TRF(6, i);
-            if (tr2) MODA_TRF(12, i);
-            tc_fence_after();
-            uint32_t sr[64];
-            const uint32_t s_addr = lane_base + sb * 128;
-            tmem_ld16x2_32<64>(s_addr, sr);            // columns c0 .. c0+31
-            tmem_ld16x2_32<64>(s_addr + 32, sr + 32);  // columns c0+32 .. c0+63
-            tmem_wait_ld();
-            reg_fence<64>(sr);
-            if (tr) MODA_TRF(7, i);
-            // masks: invisible scores become -inf (p = 0)
-            if (i < n_seq) {
-                const int kb = i * BN + c0;
-                const int lim = a.causal ? t_row : a.T - 1;   // last visible key
-                if (kb + 63 > lim) {
+        int j0 = 0, kt = 0;
+        for (int rnd = 0; ok && rnd * tstep < a.n_tiles; ++rnd) {
+            const int tile = snake_tile(rnd, cta, tstep);
+            if (tile >= a.n_tiles) continue;
+            const FwdTile T = fwd_tile(a, tile);
+            const int t0 = T.t0, n_seq = T.n_seq, nb = T.nb;
+            const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
+            float m = -INFINITY, l = 0.0f;                // l: this half's share of the row sum
+            for (int i = 0; i < nb; ++i) {
+                const int j = j0 + i;                     // running block count: ring phases
+                const int sb = j % kSBufs;
+                if (tr) MODA_TRF(5, j);
+                // every wait result is made warp-uniform: the shuffles and the
+                // .sync.aligned TMEM accesses below need the whole warp
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + sb], (j / kSBufs) & 1, a.status,
+                                                       abort_flag))) { ok = false; break; }
+                if (tr) MODA_TRF(6, j);
+                if (tr2) MODA_TRF(12, j);
+                tc_fence_after();
+                uint32_t sr[64];
+                const uint32_t s_addr = lane_base + sb * 128;
+                tmem_ld16x2_32<64>(s_addr, sr);            // columns c0 .. c0+31
+                tmem_ld16x2_32<64>(s_addr + 32, sr + 32);  // columns c0+32 .. c0+63
+                tmem_wait_ld();
+                reg_fence<64>(sr);
+                if (tr) MODA_TRF(7, j);
+                // masks: invisible scores become -inf (p = 0)
+                if (i < n_seq) {
+                    const int kb = i * BN + c0;
+                    const int lim = a.causal ? t_row : a.T - 1;   // last visible key
+                    if (kb + 63 > lim) {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (kb + c > lim) sr[c] = __float_as_uint(-INFINITY);
+                    }
+                } else {
+                    const int base = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows) - c0;
+                    const int lo = base + a.win_lo;
+                    const int hi = min(base + a.L, a.dep_rows - c0);
 #pragma unroll
                     for (int c = 0; c < 64; ++c)
-                        if (kb + c > lim) sr[c] = __float_as_uint(-INFINITY);
+                        if (c < lo || c >= hi) sr[c] = __float_as_uint(-INFINITY);
                 }
-            } else {
-                const int base = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows) - c0;
-                const int lo = base + a.win_lo;
-                const int hi = min(base + a.L, a.dep_rows - c0);
+                // Row max of this block (both halves of the row), base 2.
+                auto block_max = [&]() -> float {
+                    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c < lo || c >= hi) sr[c] = __float_as_uint(-INFINITY);
-            }
-            // Row max of this block (both halves of the row), base 2.
-            auto block_max = [&]() -> float {
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    for (int c = 0; c < 64; c += 8) {
 #pragma unroll
-                for (int c = 0; c < 64; c += 8) {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        mx4[u] = fmax3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
-                }
-                float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                return mx * sl2;
-            };
-            // p = 2^(s*sl2 - m) for this thread's 64 columns, packed to bf16;
-            // returns this half-row's sum.
-            uint32_t pk[32];
-            auto exp_block = [&]() -> float {
-                float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -m);
-                    const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m);
-                    float p0, p1;
-                    if ((c & 3) < 4 - MODA_FWD_SWEXP) {     // MUFU
-                        p0 = ex2(x0);
-                        p1 = ex2(x1);
-                    } else {                                 // FMA pipe
-                        p0 = ex2_fma(x0);
-                        p1 = ex2_fma(x1);
+                        for (int u = 0; u < 4; ++u)
+                            mx4[u] = fmax3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
                     }
-                    rs4[c & 3] += p0 + p1;
-                    pk[c] = pack_bf16(p0, p1);
-                }
-                return (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-            };
-            // The online softmax is exact for any reference point m, so a
-            // block is first exponentiated against the running m without
-            // computing its max.  Only when some p could exceed 2^10 (a
-            // half-row sum above 2^10 is necessary for that, and catches
-            // overflow too) does the warp take the block max, rescale O and
-            // l to the new reference and recompute P.  The first block sets m.
-            if (i == 0) m = block_max();
-            if (tr) MODA_TRF(8, i);
-            if (tr2) MODA_TRF(13, i);
-            float rs = exp_block();
-            if (tr) MODA_TRF(9, i);
-            if (i > 0 && __any_sync(0xffffffffu, !(rs <= kLazyLimit))) {
-                const float m_new = fmaxf(m, block_max());
-                // O must hold P_{i-1} V_{i-1} before it is rescaled: wait for
-                // the V-stage release PV_{i-1} commits.  S_i was issued after
-                // PV_{i-2}, so at most PV_{i-1} is in flight, and PV_{i+2}
-                // (the stage's next use) needs P_{i+2}: the parity is exact.
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + (i - 1) % kVStages],
-                                                       ((i - 1) / kVStages) & 1, a.status, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const float alpha = ex2(m - m_new);
-                l *= alpha;
-                m = m_new;
+                    float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    return mx * sl2;
+                };
+                // p = 2^(s*sl2 - m) for this thread's 64 columns, packed to bf16;
+                // returns this half-row's sum.
+                uint32_t pk[32];
+                auto exp_block = [&]() -> float {
+                    float rs4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-                for (int c = 0; c < D / 2; c += 32) {   // this thread's half of the O row
-                    uint32_t o[32];
-                    tmem_ld16x2_32<D / 2>(lane_base + kColO + c, o);
-                    tmem_wait_ld();
-                    reg_fence<32>(o);
+                    for (int c = 0; c < 32; ++c) {
+                        const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -m);
+                        const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m);
+                        float p0, p1;
+                        if ((c & 3) < 4 - MODA_FWD_SWEXP) {     // MUFU
+                            p0 = ex2(x0);
+                            p1 = ex2(x1);
+                        } else {                                 // FMA pipe
+                            p0 = ex2_fma(x0);
+                            p1 = ex2_fma(x1);
+                        }
+                        rs4[c & 3] += p0 + p1;
+                        pk[c] = pack_bf16(p0, p1);
+                    }
+                    return (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+                };
+                // The online softmax is exact for any reference point m, so a
+                // block is first exponentiated against the running m without
+                // computing its max.  Only when some p could exceed 2^10 (a
+                // half-row sum above 2^10 is necessary for that, and catches
+                // overflow too) does the warp take the block max, rescale O and
+                // l to the new reference and recompute P.  The first block sets m.
+                if (i == 0) m = block_max();
+                if (tr) MODA_TRF(8, j);
+                if (tr2) MODA_TRF(13, j);
+                float rs = exp_block();
+                if (tr) MODA_TRF(9, j);
+                if (i > 0 && __any_sync(0xffffffffu, !(rs <= kLazyLimit))) {
+                    const float m_new = fmaxf(m, block_max());
+                    // O must hold P_{i-1} V_{i-1} before it is rescaled: wait for
+                    // the V-stage release PV_{i-1} commits.  S_i was issued after
+                    // PV_{i-2}, so at most PV_{i-1} is in flight, and PV_{i+2}
+                    // (the stage's next use) needs P_{i+2}: the parity is exact.
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + (j - 1) % kVStages],
+                                                           ((j - 1) / kVStages) & 1, a.status, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float alpha = ex2(m - m_new);
+                    l *= alpha;
+                    m = m_new;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st16x2_32<D / 2>(lane_base + kColO + c, o);
+                    for (int c = 0; c < D / 2; c += 32) {   // this thread's half of the O row
+                        uint32_t o[32];
+                        tmem_ld16x2_32<D / 2>(lane_base + kColO + c, o);
+                        tmem_wait_ld();
+                        reg_fence<32>(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st16x2_32<D / 2>(lane_base + kColO + c, o);
+                    }
+                    tmem_wait_st();
+                    rs = exp_block();
                 }
+                l += rs;
+                if (tr) MODA_TRF(10, j);
+                if (tr2) MODA_TRF(14, j);
+                // P columns c0/2 .. c0/2+31 (bf16 pairs) over the S columns this
+                // warp has already read (its own loads completed above)
+                __syncwarp();
+                tmem_st16x2_32<32>(s_addr, pk);
                 tmem_wait_st();
-                rs = exp_block();
+                if (tr) MODA_TRF(11, j);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kPReady + sb]);
+                if (tr2) MODA_TRF(15, j);
             }
-            l += rs;
-            if (tr) MODA_TRF(10, i);
-            if (tr2) MODA_TRF(14, i);
-            // P columns c0/2 .. c0/2+31 (bf16 pairs) over the S columns this
-            // warp has already read (its own loads completed above)
-            __syncwarp();
-            tmem_st16x2_32<32>(s_addr, pk);
-            tmem_wait_st();
-            if (tr) MODA_TRF(11, i);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kPReady + sb]);
-            if (tr2) MODA_TRF(15, i);
-        }
-        // ---------------------------------------------------- epilogue ------
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFinal], 0, a.status, abort_flag));
-        const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
-        if (ok) {
-            tc_fence_after();
-            uint32_t o[D / 2];
+            // ---------------------------------------------------- epilogue ------
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFinal], kt & 1, a.status, abort_flag));
+            const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+            if (ok) {
+                tc_fence_after();
+                uint32_t o[D / 2];
 #pragma unroll
-            for (int c = 0; c < D / 2; c += 32) tmem_ld16x2_32<D / 2>(lane_base + kColO + c, o + c);
-            tmem_wait_ld();
-            if (row_real && t_row < a.T) {
-                const float inv = 1.0f / l_row;
-                const size_t qrow = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T + t_row;
-                uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + half * (D / 2));
+                for (int c = 0; c < D / 2; c += 32) tmem_ld16x2_32<D / 2>(lane_base + kColO + c, o + c);
+                tmem_wait_ld();
+                reg_fence<D / 2>(o);
+                // O is in registers: the next tile's first PV may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kOFree]);
+                if (row_real && t_row < a.T) {
+                    const float inv = 1.0f / l_row;
+                    const size_t qrow = (static_cast<size_t>(T.b) * a.Hq + T.hk * a.G + g) * a.T + t_row;
+                    uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + half * (D / 2));
 #pragma unroll
-                for (int c = 0; c < D / 2; c += 8) {
-                    uint4 v;
-                    v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv, __uint_as_float(o[c + 1]) * inv);
-                    v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-                    v.z = pack_bf16(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
-                    v.w = pack_bf16(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
-                    dst[c / 8] = v;
+                    for (int c = 0; c < D / 2; c += 8) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(o[c + 0]) * inv, __uint_as_float(o[c + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
+                        dst[c / 8] = v;
+                    }
+                    if (half == 0) a.LSE[qrow] = (m + log2f(l_row)) * 0.6931471805599453f;
                 }
-                if (half == 0) a.LSE[qrow] = (m + log2f(l_row)) * 0.6931471805599453f;
             }
+            j0 += nb;
+            ++kt;
         }
     }
     tc_fence_before();
@@ -506,7 +579,17 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     e = cudaFuncSetAttribute(moda_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    const long long grid = (long long)p.B * p.Hk * a.n_qt;
+    // Short tiles (on average fewer than 64 key blocks): one persistent CTA per
+    // SM walks its share, so tile start-up and epilogue overlap the previous
+    // tile.  Long tiles: one CTA per tile (each takes exactly its own tile),
+    // which measured faster there.
+    const long long n_tiles = (long long)p.B * p.Hk * a.n_qt;
+    if (n_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    a.n_tiles = static_cast<int>(n_tiles);
+    const long long seq_blocks = p.causal ? ((long long)p.T + BN - 1) / BN / 2 + 1 : ((long long)p.T + BN - 1) / BN;
+    const long long avg_blocks = seq_blocks + ((long long)a.Tq * p.L + a.dep_rows - 1) / a.dep_rows;
+    const long long sms = device_sm_count() > 0 ? device_sm_count() : 1;
+    const long long grid = (avg_blocks < 64 && n_tiles > sms) ? sms : n_tiles;
     moda_fwd_sm100_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }

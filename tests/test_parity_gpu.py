@@ -275,3 +275,17 @@ def test_modes_layer_T4k_sampled():
         out = run_gpu(w, x)
         _check_rows(w, x, out)
         _check_slices(w, x, out, [(0, 2)])
+
+
+def test_fwd_bwd_many_tiles_per_cta():
+    """512 short query tiles: the forward runs persistent CTAs that each walk
+    several tiles (ring phases and the Q / O hand-offs cross tile boundaries);
+    checked in full, with a ragged last tile (T = 1000)."""
+    w = small_w(4, 16, 8, 64, 1000, 6, backward=True)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x)
+    O, LSE = oracle_fwd_full(w, x)
+    assert_out_close(f64(out["O"]), O, "bf16", "O")
+    assert err_stats(f64(out["LSE"]), LSE)[0] <= LSE_MAX_ABS
+    for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(w, x)):
+        assert_grad_close(f64(out[name]), r, name)
