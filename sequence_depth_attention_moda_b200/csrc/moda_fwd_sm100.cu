@@ -111,13 +111,6 @@ struct FwdArgs {
 struct FwdTile {
     int b, hk, bh, t0, t_end, n_seq, nb;
 };
-// Tile of CTA c in round r of a persistent launch with G CTAs: rounds of G
-// tiles of the longest-first order, dealt alternately forwards and backwards
-// (a snake), so every CTA's total stays close to the mean.  Only the last
-// round can run past n_tiles; the caller skips such slots.
-__device__ __forceinline__ int snake_tile(int r, int c, int G) {
-    return r * G + ((r & 1) ? G - 1 - c : c);
-}
 __device__ __forceinline__ FwdTile fwd_tile(const FwdArgs& a, int idx) {
     const int nbh = a.B * a.Hk;
     FwdTile t;

@@ -35,6 +35,14 @@ moda_status api_fail(moda_status s, const char* msg);
 // SM count of the current device (cached).
 int device_sm_count();
 
+// Tile of CTA c in round r of a persistent launch with G CTAs: rounds of G
+// tiles of a longest-first order, dealt alternately forwards and backwards
+// (a snake), so every CTA's total stays close to the mean.  Only the last
+// round can run past the tile count; callers skip such slots.
+__host__ __device__ inline int snake_tile(int r, int c, int G) {
+    return r * G + ((r & 1) ? G - 1 - c : c);
+}
+
 // Records the calling thread's k-th phase marker on `stream`, if one is set
 // (see moda_set_phase_events); a no-op otherwise.
 void phase_mark(int k, cudaStream_t stream);
