@@ -146,7 +146,9 @@ enum { kQFull = 0, kKFull = 1, kVFull = kKFull + kKStages, kVEmpty = kVFull + kV
        kOFree = kOFinal + 1, kNumBars = kOFree + 1 };
 static_assert(kKStages == kSBufs, "a K stage is released by the score barrier of its S buffer");
 
-template <int D>
+// kPersist: CTAs walk several tiles (grid = SM count); otherwise each CTA
+// takes exactly tile blockIdx.x and the tile loops compile away.
+template <int D, bool kPersist>
 __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __grid_constant__ FwdArgs a) {
     using Lay = Layout<D>;
     extern __shared__ unsigned char smem_raw[];
@@ -168,6 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
     const int R = a.G * a.Tq;
     const int cta = static_cast<int>(blockIdx.x);
     const int tstep = static_cast<int>(gridDim.x);
+    const int n_rounds = kPersist ? (a.n_tiles + tstep - 1) / tstep : 1;
+    auto tile_of = [&](int rnd) { return kPersist ? snake_tile(rnd, cta, tstep) : cta; };
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kQFull], 1);
@@ -221,8 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
             int j = 0, kt = 0, issued = 0, nq = 0;
             bool ok = true;
-            for (int rnd = 0; ok && rnd * tstep < a.n_tiles; ++rnd) {
-                const int tile = snake_tile(rnd, cta, tstep);
+            for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+                const int tile = tile_of(rnd);
                 if (tile >= a.n_tiles) continue;
                 const FwdTile T = fwd_tile(a, tile);
                 if (is_k) {
@@ -330,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         // the next scores ready when the softmax needs them.
         bool ok = true;
         int j0 = 0, kt = 0;
-        for (int rnd = 0; ok && rnd * tstep < a.n_tiles; ++rnd) {
-            const int tile = snake_tile(rnd, cta, tstep);
+        for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+            const int tile = tile_of(rnd);
             if (tile >= a.n_tiles) continue;
             const FwdTile T = fwd_tile(a, tile);
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], kt & 1, a.status, abort_flag));
@@ -368,8 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         const float sl2 = a.scale_log2;
         bool ok = true;
         int j0 = 0, kt = 0;
-        for (int rnd = 0; ok && rnd * tstep < a.n_tiles; ++rnd) {
-            const int tile = snake_tile(rnd, cta, tstep);
+        for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+            const int tile = tile_of(rnd);
             if (tile >= a.n_tiles) continue;
             const FwdTile T = fwd_tile(a, tile);
             const int t0 = T.t0, n_seq = T.n_seq, nb = T.nb;
@@ -569,7 +573,10 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
         a.tvd = a.tv;
     }
     const uint32_t smem = Layout<D>::kDynSmem;
-    e = cudaFuncSetAttribute(moda_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(moda_fwd_sm100_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(moda_fwd_sm100_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     // Short tiles (on average fewer than 64 key blocks): one persistent CTA per
@@ -582,8 +589,10 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     const long long seq_blocks = p.causal ? ((long long)p.T + BN - 1) / BN / 2 + 1 : ((long long)p.T + BN - 1) / BN;
     const long long avg_blocks = seq_blocks + ((long long)a.Tq * p.L + a.dep_rows - 1) / a.dep_rows;
     const long long sms = device_sm_count() > 0 ? device_sm_count() : 1;
-    const long long grid = (avg_blocks < 64 && n_tiles > sms) ? sms : n_tiles;
-    moda_fwd_sm100_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(a);
+    if (avg_blocks < 64 && n_tiles > sms)
+        moda_fwd_sm100_kernel<D, true><<<(unsigned)sms, kThreads, smem, stream>>>(a);
+    else
+        moda_fwd_sm100_kernel<D, false><<<(unsigned)n_tiles, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
