@@ -207,6 +207,32 @@ moda_status moda_set_phase_events(void* const* events, int n);
 moda_status moda_check_status(moda_stream_t stream);
 
 /*
+ * Decoding: one new token per sequence attends to T cached keys and to its
+ * own L depth rows under one softmax (paper summary of arXiv 2603.15619,
+ * "Mixture-of-Depths Attention (MoDA): The Unified Operator", the newest query
+ * position; "Complexity Analysis", Table 1: decoding costs O(L*T*D + L^2*D)
+ * per token across the layers).
+ *   shape     B, Hq, Hk, d, dtype, softmax_scale, depth_window as for
+ *             moda_fwd; T = cached keys including the new token's own
+ *             (T >= 1 when B > 0); L = depth rows of the new token; C, the
+ *             depth layout and MODA_FLAG_NONCAUSAL have no effect.
+ *             Supported: d in {64, 128}, G = Hq / Hk <= 16, bf16 or fp32.
+ *   q         [B, Hq, d]     the new token's queries       (device)
+ *   K, V      [B, Hk, T, d]  the cached keys and values    (device)
+ *   Kd, Vd    [B, Hk, L, d]  the new token's depth rows    (device; NULL if L == 0)
+ *   o         [B, Hq, d]     output, same dtype            (device)
+ *   lse       [B, Hq]        fp32 natural-log LSE          (device)
+ *   ws        moda_decode_workspace_size(shape) bytes      (device, caller-owned)
+ * All buffers are contiguous and 16-byte aligned; nothing is allocated.
+ * Returns MODA_ERR_INVALID_ARG / MODA_ERR_UNSUPPORTED for shapes outside the
+ * above, MODA_ERR_MISALIGNED, MODA_ERR_WORKSPACE if ws_bytes is too small.
+ */
+size_t moda_decode_workspace_size(const moda_shape* shape);
+moda_status moda_decode(const moda_shape* shape, const void* q, const void* K, const void* V,
+                        const void* Kd, const void* Vd, void* o, float* lse,
+                        void* ws, size_t ws_bytes, moda_stream_t stream);
+
+/*
  * Failure-path self-test (the pages have no counterpart).  Queues on `stream`
  * one small kernel whose warps wait, through the same bounded mbarrier wait
  * the forward and backward kernels use, on a barrier that nothing arrives on.

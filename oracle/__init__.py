@@ -18,6 +18,8 @@ definitions it follows:
 * Paper summary, "Hardware-Efficient Implementation" (layer-major versus
   token-major depth layout, for the repack).
 
+``decode`` evaluates the newest token's rows through the same C row function.
+
 Parity status: the forward, backward and repack are pinned by the CPU tests in
 ``tests/test_oracle.py`` (library special cases, closed forms, invariants, an
 independent dense brute force, autograd and finite differences).
@@ -175,6 +177,31 @@ def row(q, Kseq, Vseq, Kdep, Vdep, scale: float = 0.0, lib=None, return_p: bool 
                         _ptr(Kdep if L else None), _ptr(Vdep if L else None),
                         _ptr(o), _ptr(lse), _ptr(p))
     return (o, float(lse[0]), p) if return_p else (o, float(lse[0]))
+
+
+def decode(q, K, V, Kd=None, Vd=None, window: int = 0, scale: float = 0.0, lib=None):
+    """Decoding: the newest token's query rows against T cached keys and its
+    own L depth rows -- one row of the operator per (b, h) (the causal mask
+    admits every cached key).  q [B,Hq,d]; K, V [B,Hk,T,d]; Kd, Vd [B,Hk,L,d]
+    or None; window > 0 keeps the last `window` depth rows.  Returns
+    (o [B,Hq,d], lse [B,Hq]) in float64."""
+    lib = lib or load_library()
+    q, K, V = _f64(q), _f64(K), _f64(V)
+    B, Hq, d = q.shape
+    Hk = K.shape[1]
+    G = Hq // Hk
+    L = 0 if Kd is None or np.size(Kd) == 0 else Kd.shape[2]
+    Kd = _f64(Kd) if L else np.zeros((B, Hk, 0, d))
+    Vd = _f64(Vd) if L else np.zeros((B, Hk, 0, d))
+    lo = L - window if 0 < window < L else 0
+    o = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            o[b, h], lse[b, h] = row(q[b, h], K[b, hk], V[b, hk], Kd[b, hk, lo:], Vd[b, hk, lo:],
+                                     scale=scale, lib=lib)
+    return o, lse
 
 
 def repack(src, B: int, Hk: int, T: int, d: int, L: int, lib=None) -> np.ndarray:

@@ -31,7 +31,8 @@ MODA_FLAG_NONCAUSAL = 1
 
 # Every symbol include/moda.h declares.
 EXPORTED = ("moda_workspace_size", "moda_repack_depth", "moda_fwd", "moda_bwd",
-            "moda_bwd_noalloc", "moda_set_phase_events", "moda_check_status",
+            "moda_bwd_noalloc", "moda_decode", "moda_decode_workspace_size",
+            "moda_set_phase_events", "moda_check_status",
             "moda_selftest_wait_timeout", "moda_status_string", "moda_last_error_message",
             "moda_version")
 
@@ -79,6 +80,10 @@ def load(path: Optional[str] = None):
         lib.moda_bwd.restype = i
         lib.moda_bwd_noalloc.argtypes = [sp] + [vp] * 13 + [vp]
         lib.moda_bwd_noalloc.restype = i
+        lib.moda_decode_workspace_size.argtypes = [sp]
+        lib.moda_decode_workspace_size.restype = sz
+        lib.moda_decode.argtypes = [sp] + [vp] * 7 + [vp, sz, vp]
+        lib.moda_decode.restype = i
         lib.moda_set_phase_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
         lib.moda_set_phase_events.restype = i
         lib.moda_check_status.argtypes = [vp]
@@ -178,6 +183,20 @@ def moda_set_phase_events(events) -> None:
 
 def moda_check_status(stream=None):
     _check(load().moda_check_status(_stream(stream)), "moda_check_status")
+
+
+def moda_decode_workspace_size(shape: moda_shape) -> int:
+    n = load().moda_decode_workspace_size(ctypes.byref(shape))
+    if n == ctypes.c_size_t(-1).value:   # report the validation error itself
+        _check(load().moda_decode(ctypes.byref(shape), *([None] * 7), None, 0, None),
+               "moda_decode_workspace_size")
+    return int(n)
+
+
+def moda_decode(shape: moda_shape, q, K, V, Kd, Vd, o, lse, ws, ws_bytes: int, stream=None):
+    _check(load().moda_decode(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd),
+                              _ptr(o), _ptr(lse), _ptr(ws), int(ws_bytes), _stream(stream)),
+           "moda_decode")
 
 
 def moda_selftest_wait_timeout(stream=None):

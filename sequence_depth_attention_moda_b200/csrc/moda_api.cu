@@ -220,6 +220,49 @@ moda_status moda_bwd(const moda_shape* shape, const void* Q, const void* K, cons
     return e == cudaSuccess ? MODA_OK : cuda_fail(e, "backward launch");
 }
 
+namespace {
+// Decoding limits on top of the shared shape checks.
+moda_status validate_decode(const moda_shape* shape, moda::Problem* p) {
+    using namespace moda;
+    moda_status st = validate(shape, p);
+    if (st != MODA_OK) return st;
+    if (p->B > 0 && p->T < 1) return fail(MODA_ERR_INVALID_ARG, "decoding needs T >= 1 cached keys");
+    if (p->d != 64 && p->d != 128)
+        return fail(MODA_ERR_UNSUPPORTED, "decoding supports d in {64, 128} (d=%d)", p->d);
+    if (p->G > 16) return fail(MODA_ERR_UNSUPPORTED, "decoding supports G <= 16 (G=%d)", p->G);
+    return MODA_OK;
+}
+}  // namespace
+
+size_t moda_decode_workspace_size(const moda_shape* shape) {
+    moda::Problem p;
+    if (validate_decode(shape, &p) != MODA_OK) return static_cast<size_t>(-1);
+    if (p.B == 0) return 0;
+    return moda::decode_workspace_bytes(p);
+}
+
+moda_status moda_decode(const moda_shape* shape, const void* q, const void* K, const void* V,
+                        const void* Kd, const void* Vd, void* o, float* lse, void* ws,
+                        size_t ws_bytes, moda_stream_t stream) {
+    using namespace moda;
+    Problem p;
+    moda_status st = validate_decode(shape, &p);
+    if (st != MODA_OK) return st;
+    if (p.B == 0) return MODA_OK;
+    if ((st = check_ptrs({{q, "q"}, {K, "K"}, {V, "V"}, {o, "o"}, {lse, "lse"}, {ws, "ws"}})) != MODA_OK)
+        return st;
+    if (p.L > 0 && (st = check_ptrs({{Kd, "Kd"}, {Vd, "Vd"}})) != MODA_OK) return st;
+    if (!device_status_word()) return fail(MODA_ERR_CUDA, "no usable CUDA device");
+    const size_t need = decode_workspace_bytes(p);
+    if (ws_bytes < need)
+        return fail(MODA_ERR_WORKSPACE, "decoding needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    phase_mark(0, s);
+    cudaError_t e = launch_decode(p, q, K, V, Kd, Vd, o, lse, ws, s);
+    if (e == cudaSuccess) phase_mark(1, s);
+    return e == cudaSuccess ? MODA_OK : cuda_fail(e, "decode launch");
+}
+
 moda_status moda_check_status(moda_stream_t stream) {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");

@@ -47,6 +47,14 @@ __host__ __device__ inline int snake_tile(int r, int c, int G) {
 // (see moda_set_phase_events); a no-op otherwise.
 void phase_mark(int k, cudaStream_t stream);
 
+// ---- decoding (moda_decode.cu) ----------------------------------------------
+// One query token per (b, Hq head) against T cached keys and L depth rows;
+// ws holds decode_workspace_bytes(p) bytes of partials.
+size_t decode_workspace_bytes(const Problem& p);
+cudaError_t launch_decode(const Problem& p, const void* q, const void* K, const void* V,
+                          const void* Kd, const void* Vd, void* out, float* lse, void* ws,
+                          cudaStream_t stream);
+
 // ---- depth repack (moda_repack.cu) -----------------------------------------
 cudaError_t launch_repack(int B, int Hk, int T, int d, int L, int elem_bytes,
                           const void* src, void* dst, cudaStream_t stream);

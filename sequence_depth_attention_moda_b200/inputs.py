@@ -62,7 +62,11 @@ LONG_64K = Workload("long_context_T64k", B=1, Hq=16, Hk=4, d=128, T=65536, L=32,
 TRAIN_FWD_BWD = Workload("train_T4k_L48", B=8, Hq=32, Hk=8, d=128, T=4096, L=48, C=64,
                          backward=True, seed=1005)
 
-WORKLOADS: Dict[str, Workload] = {w.name: w for w in (TINY_FP32, LAYER_1P5B, LONG_64K, TRAIN_FWD_BWD)}
+# Decoding: one new token per sequence over T cached keys (its L depth rows).
+DECODE_T32K = Workload("decode_T32k_L48", B=8, Hq=32, Hk=8, d=128, T=32768, L=48, C=64, seed=1006)
+
+WORKLOADS: Dict[str, Workload] = {w.name: w for w in (TINY_FP32, LAYER_1P5B, LONG_64K, TRAIN_FWD_BWD,
+                                                      DECODE_T32K)}
 
 
 def depth_group_sweep() -> List[Workload]:
@@ -108,3 +112,29 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
     if w.backward if grad_out is None else grad_out:
         out["dO"] = draw((w.B, w.Hq, w.T, w.d))
     return out
+
+
+def make_decode_inputs(w: Workload, device="cpu", seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Decoding inputs for workload ``w``: q [B,Hq,d] (the new token's
+    queries), K, V [B,Hk,T,d] (the cache, the new token's own key last) and
+    Kd, Vd [B,Hk,L,d] (the new token's depth rows), drawn in that order like
+    make_inputs."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed if seed is None else seed)
+    dt = w.torch_dtype()
+    inv = 1.0 / (w.d ** 0.5)
+
+    def draw(shape, scaled=False):
+        x = torch.randn(shape, generator=g, device=dev, dtype=torch.float32)
+        if scaled:
+            x.mul_(inv)
+        return x.to(dt).contiguous()
+
+    return {
+        "q": draw((w.B, w.Hq, w.d), w.qk_scaled),
+        "K": draw((w.B, w.Hk, w.T, w.d), w.qk_scaled),
+        "V": draw((w.B, w.Hk, w.T, w.d)),
+        "Kd": draw((w.B, w.Hk, w.L, w.d), w.qk_scaled),
+        "Vd": draw((w.B, w.Hk, w.L, w.d)),
+    }

@@ -396,7 +396,20 @@ def pin_modes_bwd_autograd(lib):
             _close(a, g.numpy(), 1e-11, f"{nm} causal={causal} window={window}")
 
 
-ALL_PINS = [pin_l0_is_causal_sdpa, pin_t1_self_plus_depth, pin_dense_bruteforce,
+def pin_decode_is_last_row(lib):
+    """Decoding the newest token equals the last row of the full operator
+    over the whole sequence (with and without a depth window)."""
+    B, Hq, Hk, T, d, L = 2, 6, 2, 9, 8, 4
+    Q, K, V, Kd, Vd, _ = rand_case(B, Hq, Hk, T, d, L, 141)
+    last = lambda x: x.reshape(B, Hk, T, L, d)[:, :, T - 1]
+    for window in (0, 3):
+        O, LSE = oracle.fwd(Q, K, V, Kd, Vd, lib=lib, window=window)
+        o, lse = oracle.decode(Q[:, :, T - 1], K, V, last(Kd), last(Vd), window=window, lib=lib)
+        _close(o, O[:, :, T - 1], 1e-12, f"decode O window={window}")
+        _close(lse, LSE[:, :, T - 1], 1e-12, f"decode LSE window={window}")
+
+
+ALL_PINS = [pin_decode_is_last_row, pin_l0_is_causal_sdpa, pin_t1_self_plus_depth, pin_dense_bruteforce,
             pin_algorithm1, pin_zero_query_closed_form, pin_depth_permutation,
             pin_gqa_is_repeat_interleave, pin_convexity, pin_bwd_autograd,
             pin_bwd_finite_differences, pin_repack_definition, pin_noncausal_l0_is_sdpa,

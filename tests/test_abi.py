@@ -120,3 +120,27 @@ def test_phase_events_validation(lib):
     arr = (ctypes.c_void_p * 9)()
     assert lib.moda_set_phase_events(arr, 9) == 1
     assert lib.moda_set_phase_events(arr, 0) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=0), 1),                                                      # no cached key
+    (dict(d=96, dtype=moda.MODA_FP32), 3),                               # decode d
+    (dict(Hq=64, Hk=2), 3),                                              # G > 16
+    (dict(depth_window=5), 1),
+])
+def test_decode_rejects_bad_shapes(lib, kw, status):
+    base = dict(B=1, Hq=4, Hk=2, T=64, d=128, L=2, C=0)
+    base.update(kw)
+    sh = moda.make_shape(**base)
+    rc = lib.moda_decode(ctypes.byref(sh), *([FAKE] * 7), FAKE, 1 << 20, None)
+    assert rc == status, (rc, moda.moda_last_error_message())
+    assert lib.moda_decode_workspace_size(ctypes.byref(sh)) == ctypes.c_size_t(-1).value
+
+
+def test_decode_rejects_null_and_empty_batch(lib):
+    sh = moda.make_shape(1, 4, 2, 64, 128, 2, 0)
+    rc = lib.moda_decode(ctypes.byref(sh), None, *([FAKE] * 6), FAKE, 1 << 20, None)
+    assert rc == 1 and "q" in moda.moda_last_error_message()
+    sh0 = moda.make_shape(0, 4, 2, 64, 128, 2, 0)
+    assert lib.moda_decode(ctypes.byref(sh0), *([None] * 7), None, 0, None) == 0
+    assert moda.moda_decode_workspace_size(sh0) == 0
