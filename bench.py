@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the L=0 twin and T=64K lines")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decoding path (one JSON line; small device footprint)")
     return ap.parse_args()
 
 
@@ -320,6 +322,43 @@ def e2e_measure(w: I.Workload, x, steps: int, world: int):
     return ms, h2d, d2h
 
 
+def decode_measure(w: I.Workload, rank: int, world: int, peaks, iters: int):
+    """Decoding one new token per sequence over the cached keys: CUDA-event
+    time per moda_decode call (inputs 1.1 GB, larger than L2), the HBM
+    roofline of its algorithmic bytes (cache K, V and the depth rows read
+    once; q read, o and LSE written) and tokens per second."""
+    import sequence_depth_attention_moda_b200 as moda
+    x = I.make_decode_inputs(w, device="cuda", seed=w.seed + 1000 * rank)
+    sh = moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, 0)
+    nws = moda.moda_decode_workspace_size(sh)
+    ws = torch.empty(max(nws, 16), device="cuda", dtype=torch.uint8)
+    o = torch.empty_like(x["q"])
+    lse = torch.empty(w.B, w.Hq, device="cuda", dtype=torch.float32)
+
+    def call():
+        moda.moda_decode(sh, x["q"], x["K"], x["V"], x["Kd"], x["Vd"], o, lse, ws, nws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / iters, world)
+    nbytes = sum(x[k].numel() * x[k].element_size() for k in ("q", "K", "V", "Kd", "Vd"))
+    nbytes += o.numel() * o.element_size() + lse.numel() * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hk": w.Hk, "d": w.d, "T": w.T, "L": w.L,
+            "ms": round(ms, 4), "tokens_per_s": round(world * w.B / (ms * 1e-3), 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "bytes_per_call": nbytes}}
+
+
 def cpu_baseline_sample(w: I.Workload, x):
     """The oracle, as it stands, on one (b, hk) slice of the workload
     (forward + backward of G heads over all T tokens and L depth rows)."""
@@ -422,6 +461,8 @@ def run_ours(args):
         extra["long_context_T64k_fwd"] = long_res
         del xl
         torch.cuda.empty_cache()
+        extra["decode_T32k"] = decode_measure(I.DECODE_T32K, rank, world, peaks, max(10, args.steps // 2))
+        torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_e2e:
@@ -500,10 +541,22 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_decode_only(args):
+    """The decoding workload alone (one GPU)."""
+    torch.cuda.set_device(0)
+    res = decode_measure(I.DECODE_T32K, 0, 1, load_peaks(), max(1, args.steps))
+    print(json.dumps({"metric": "MoDA decoding tokens/s (one new token per sequence)",
+                      "value": res["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1,
+                      "steps": args.steps, "warmup": 3, "higher_is_better": True,
+                      "data": "synthetic", "decode": res}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.decode_only:
+        run_decode_only(args)
     else:
         run_ours(args)
 

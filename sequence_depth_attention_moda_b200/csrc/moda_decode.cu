@@ -91,6 +91,30 @@ __device__ __forceinline__ void loadn(const float* p, float* v) {
     }
 }
 
+// Raw V row slice of one lane (NDL elements), kept packed until used.
+template <typename E, int N> struct VRaw;
+template <> struct VRaw<__nv_bfloat16, 4> {
+    uint2 u;
+    __device__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint2*>(p)); }
+    __device__ void get(float* v) const {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+    }
+};
+template <> struct VRaw<__nv_bfloat16, 2> {
+    unsigned int u;
+    __device__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const unsigned int*>(p)); }
+    __device__ void get(float* v) const {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+        v[0] = a.x; v[1] = a.y;
+    }
+};
+
+#ifndef MODA_DEC_PREFETCH_V
+#define MODA_DEC_PREFETCH_V 1
+#endif
+
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
@@ -143,7 +167,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecArgs
 #pragma unroll
         for (int e = 0; e < NDL; ++e) o[g][e] = 0.0f;
     }
+    // bf16 tiles of 32 keys load their V rows (lane = head dimensions) before
+    // the scores, so that latency overlaps the score work
+    constexpr bool kPre = MODA_DEC_PREFETCH_V && sizeof(E) == 2;
+    using VR = VRaw<__nv_bfloat16, NDL>;
     for (int kt = k0 + warp * 32; kt < k1; kt += 32 * kDecWarps) {
+        const int nk = min(32, k1 - kt);
+        const E* vt = vb + static_cast<size_t>(kt) * D + lane * NDL;
+        VR vpre[kPre ? 32 : 1];
+        if (kPre && nk == 32) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+                vpre[jj].load(reinterpret_cast<const __nv_bfloat16*>(vt + static_cast<size_t>(jj) * D));
+        }
         // scores of this lane's key for the G heads (base 2)
         const int key = kt + lane;
         const bool valid = key < k1;
@@ -152,7 +188,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecArgs
         for (int g = 0; g < GMAX; ++g) s[g] = 0.0f;
         if (valid) {
             const E* kr = kb + static_cast<size_t>(key) * D;
-#pragma unroll 4
+#pragma unroll
             for (int c = 0; c < D / 8; ++c) {
                 float kv[8];
                 load8(kr, c, kv);
@@ -182,15 +218,33 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecArgs
             for (int e = 0; e < NDL; ++e) o[g][e] *= alpha;
         }
         // O += P V with lane = head dimensions [NDL*lane, NDL*lane + NDL)
-        const int nk = min(32, k1 - kt);
-        for (int jj = 0; jj < nk; ++jj) {
-            float vv[NDL];
-            loadn<NDL>(vb + static_cast<size_t>(kt + jj) * D + lane * NDL, vv);
+        auto accumulate = [&](int jj, const float* vv) {
 #pragma unroll
             for (int g = 0; g < GMAX; ++g) {
                 const float pj = __shfl_sync(0xffffffffu, p[g], jj);
 #pragma unroll
                 for (int e = 0; e < NDL; ++e) o[g][e] = fmaf(pj, vv[e], o[g][e]);
+            }
+        };
+        if (kPre && nk == 32) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                float vv[NDL];
+                vpre[jj].get(vv);
+                accumulate(jj, vv);
+            }
+        } else if (nk == 32) {           // full tile: several V rows in flight
+#pragma unroll 8
+            for (int jj = 0; jj < 32; ++jj) {
+                float vv[NDL];
+                loadn<NDL>(vt + static_cast<size_t>(jj) * D, vv);
+                accumulate(jj, vv);
+            }
+        } else {
+            for (int jj = 0; jj < nk; ++jj) {
+                float vv[NDL];
+                loadn<NDL>(vt + static_cast<size_t>(jj) * D, vv);
+                accumulate(jj, vv);
             }
         }
     }
@@ -233,9 +287,13 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restri
     if (threadIdx.x == 0) lse[row] = (M + log2f(l)) * 0.6931471805599453f;
 }
 
+#ifndef MODA_DEC_CTAS_PER_SM
+#define MODA_DEC_CTAS_PER_SM 4
+#endif
 int seq_splits(const Problem& p) {
     const long long bh = static_cast<long long>(p.B) * p.Hk;
-    const long long want = (2LL * device_sm_count() + bh - 1) / bh;     // ~2 CTAs per SM
+    // enough CTAs to fill every SM (loads in flight hide the HBM latency)
+    const long long want = (static_cast<long long>(MODA_DEC_CTAS_PER_SM) * device_sm_count() + bh - 1) / bh;
     const long long by_len = (static_cast<long long>(p.T) + 255) / 256;  // >= 256 keys each
     long long n = want < by_len ? want : by_len;
     return static_cast<int>(n < 1 ? 1 : n);
