@@ -56,6 +56,12 @@ CASES = [  # B, Hq, Hk, d, T, L, window, dtype
     (2, 6, 2, 128, 300, 6, 0, "bf16"),     # G = 3
     (1, 4, 2, 64, 500, 5, 2, "fp32"),
     (1, 2, 2, 128, 33, 40, 0, "fp32"),     # more depth rows than keys per warp tile
+    (2, 8, 2, 128, 65, 100, 0, "bf16"),    # two depth tiles; last sequence tile holds one key
+    (1, 4, 1, 128, 64, 100, 70, "bf16"),   # depth window starting inside a tile
+    (1, 2, 1, 64, 63, 64, 0, "bf16"),      # one key short of a tile, exactly one depth tile
+    (64, 16, 8, 64, 200, 4, 0, "bf16"),    # many KV heads per CTA range, ring wraps
+    (2, 32, 8, 128, 4096, 48, 0, "bf16"),  # d = 128: the ring wraps (7 items per CTA)
+    (8, 8, 8, 128, 100, 0, 0, "bf16"),     # G = 1, no depth
 ]
 
 
