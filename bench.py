@@ -125,10 +125,10 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
-def traffic_from_profile(kernel: str, kernel_src: str):
+def traffic_from_profile(kernel: str, kernel_src: str, table: str = "dram_traffic_layer_T4k.md"):
     """Per-launch DRAM bytes (read + write) of `kernel` from the committed ncu
     summary, or None when its source has changed since the capture."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic_layer_T4k.md")
+    path = os.path.join(ROOT, "profiles", table)
     if not os.path.exists(path):
         return None
     m = re.search(r"^\| %s \| (\d+) \| [^|]+ \| ([0-9a-f]{16}) \|" % re.escape(kernel),
@@ -352,11 +352,15 @@ def decode_measure(w: I.Workload, rank: int, world: int, peaks, iters: int):
     nbytes = sum(x[k].numel() * x[k].element_size() for k in ("q", "K", "V", "Kd", "Vd"))
     nbytes += o.numel() * o.element_size() + lse.numel() * 4
     gbs = nbytes / (ms * 1e-3) / 1e9
+    src = os.path.join(ROOT, "sequence_depth_attention_moda_b200", "csrc", "moda_decode.cu")
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hk": w.Hk, "d": w.d, "T": w.T, "L": w.L,
             "ms": round(ms, 4), "tokens_per_s": round(world * w.B / (ms * 1e-3), 1),
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+            "roofline": {"kernel": "decode_mma_kernel (+ decode_combine_kernel, both timed)",
+                         "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "bytes_per_call": nbytes}}
+                         "bytes_per_call": nbytes,
+                         "traffic": traffic_from_profile("decode_mma_kernel", src,
+                                                         "dram_traffic_decode_T32k.md")}}
 
 
 def cpu_baseline_sample(w: I.Workload, x):
