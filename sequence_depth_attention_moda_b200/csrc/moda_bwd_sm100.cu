@@ -43,8 +43,8 @@ using namespace ptx;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kThreads = 224;            // dq: warp 0 TMA, warps 1 and 6 MMA, warps 2..5 math
-constexpr int kMathThreads = 128;
+constexpr int kThreads = 352;            // dq: warp 0 TMA, warps 1 and 6 MMA, warps 2..5 and 7..10 math
+constexpr int kMathThreads = 256;
 constexpr int kKvMathWarps = 8;          // dkdv: warps 2..9, two per TMEM lane quarter
 constexpr int kKvThreads = 64 + 32 * kKvMathWarps;
 constexpr uint32_t kSlabBytes = 128 * 128;
@@ -644,15 +644,18 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     MODA_TRQ(2, i);
                     tc_fence_after();
                     const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
+                    // dS of keys [16kk, 16kk + 16) sits at column (kk / 2) * 32 +
+                    // (kk % 2) * 8 of the buffer (each math half packs its 32 keys
+                    // into the first 16 of its own 32 columns)
                     if (n == kDqBN) {
     #pragma unroll
                         for (int kk = 0; kk < kDqBN / 16; ++kk)
-                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
-                                    (i > 0 || kk > 0) ? 1u : 0u);
+                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+                                    kmn + kk * (2048 >> 4), id_dq, (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
                         for (int kk = 0; kk < n / 16; ++kk)
-                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + kk * 8, kmn + kk * (2048 >> 4), id_dq,
-                                    (i > 0 || kk > 0) ? 1u : 0u);
+                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+                                    kmn + kk * (2048 >> 4), id_dq, (i > 0 || kk > 0) ? 1u : 0u);
                     }
                     if (!seq) {
     #pragma unroll
@@ -670,11 +673,16 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 umma_commit_elect(&bars[kB_Final]);
             }
         }
-    } else if (warp <= 5) {
+    } else {
         // ------------------------------------------------------ math --------
+        // Warps 2..5 and 7..10: two per TMEM lane quarter (they share its
+        // sub-partition and interleave).  Thread = query row r; the warp's
+        // half takes columns [c0, c0 + 32) of every 64-row block.
         const int quarter = warp & 3;
+        const int half = warp >= 7 ? 1 : 0;
+        const int c0 = 32 * half;
         const int r = quarter * 32 + lane;
-        const int mt = threadIdx.x - 64;                  // 0..127
+        const int mt = threadIdx.x - 64;                  // 0 for warp 2, lane 0
         const bool row_real = r < R;
         const int g = row_real ? r / a.Tq : 0;
         const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
@@ -689,24 +697,23 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const size_t dep_base = (static_cast<size_t>(bh) * a.T + t0) * a.L;  // first depth row of the tile
 
         // dKd / dVd of depth block jd: TMEM lane = d index, column = depth row,
-        // so for each depth row the four warps store 128 consecutive d values
-        // (64 contiguous bytes per warp) straight to global memory.
+        // so for each depth row the four warps of a half store 128 consecutive
+        // d values (64 contiguous bytes per warp) straight to global memory;
+        // the half takes depth rows [c0, c0 + 32) of the block.
         auto depth_epilogue = [&](int jd) {
-            uint32_t xk[64], xv[64];
-            tmem_ld32(lane_base + kColDKd, xk);
-            tmem_ld32(lane_base + kColDKd + 32, xk + 32);
-            tmem_ld32(lane_base + kColDVd, xv);
-            tmem_ld32(lane_base + kColDVd + 32, xv + 32);
+            uint32_t xk[32], xv[32];
+            tmem_ld32(lane_base + kColDKd + c0, xk);
+            tmem_ld32(lane_base + kColDVd + c0, xv);
             tmem_wait_ld();
-            reg_fence<64>(xk);
-            reg_fence<64>(xv);
+            reg_fence<32>(xk);
+            reg_fence<32>(xv);
             if (r < D) {
-                const int row0 = jd * a.dep_rows;
-                const int nvalid = min(a.dep_rows, dep_total - row0);
+                const int row0 = jd * a.dep_rows + c0;
+                const int nvalid = min(a.dep_rows, dep_total - jd * a.dep_rows) - c0;
                 __nv_bfloat16* gk = a.dKd + (dep_base + row0) * D + r;
                 __nv_bfloat16* gv = a.dVd + (dep_base + row0) * D + r;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     if (c < nvalid) {
                         gk[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
                         gv[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xv[c]));
@@ -724,12 +731,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             if (!mbar_wait(&bars[kB_SFull + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
             if (mt == 0) MODA_TRQ(5, i);
             tc_fence_after();
-            uint32_t s[64], dp[64], dsk[32], pk[32];
-            tmem_ld32(lane_base + kColS + buf * 64, s);
-            tmem_ld32(lane_base + kColS + buf * 64 + 32, s + 32);
-            tmem_ld32(lane_base + kColDP + buf * 64, dp);
-            tmem_ld32(lane_base + kColDP + buf * 64 + 32, dp + 32);
+            uint32_t s[32], dp[32], dsk[16], pk[16];
+            tmem_ld32(lane_base + kColS + buf * 64 + c0, s);
+            tmem_ld32(lane_base + kColDP + buf * 64 + c0, dp);
             tmem_wait_ld();
+            reg_fence<32>(s);
+            reg_fence<32>(dp);
             int lo = 0, hi = kDqBN, kb = 0;
             const int lim = a.causal ? t_row : a.T - 1;   // last visible sequence key
             if (seq) {
@@ -739,12 +746,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 lo = base + a.win_lo;
                 hi = min(base + a.L, a.dep_rows);
             }
-            const bool all_visible = seq && kb + kDqBN - 1 <= lim;
+            const bool all_visible = seq && kb + c0 + 31 <= lim;
             // Masked entries get score -inf and dP 0 by selects (no branch per
             // element), so exp2 runs unconditionally and yields exactly 0.
             if (all_visible) {
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
+                for (int e = 0; e < 32; e += 2) {
                     const float p0 = ex2(fmaf(__uint_as_float(s[e]), sl2, -lse2));
                     const float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), sl2, -lse2));
                     dsk[e / 2] = pack_bf16(p0 * (__uint_as_float(dp[e]) - Dr),
@@ -752,18 +759,18 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     pk[e / 2] = pack_bf16(p0, p1);
                 }
             } else {
-                // visible columns: seq c <= t_row - kb; depth lo <= c < hi
+                // visible block columns: seq c <= t_row - kb; depth lo <= c < hi
                 const int vlo = seq ? 0 : lo;
                 const int vhi = seq ? lim - kb + 1 : hi;
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
+                for (int e = 0; e < 32; e += 2) {
                     float p2[2], d2[2];
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int c = e + u;
+                        const int c = c0 + e + u;
                         const bool vis = c >= vlo && c < vhi;
-                        const float sv = vis ? __uint_as_float(s[c]) : -INFINITY;
-                        const float dv = vis ? __uint_as_float(dp[c]) : Dr;
+                        const float sv = vis ? __uint_as_float(s[e + u]) : -INFINITY;
+                        const float dv = vis ? __uint_as_float(dp[e + u]) : Dr;
                         p2[u] = ex2(fmaf(sv, sl2, -lse2));
                         d2[u] = p2[u] * (dv - Dr);
                     }
@@ -772,7 +779,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 }
             }
             if (mt == 0) MODA_TRQ(6, i);
-            tmem_st32(lane_base + kColS + buf * 64, dsk);
+            // packed dS of keys [c0, c0 + 32) into columns [c0, c0 + 16): inside
+            // this half's own score columns, which only it reads
+            tmem_st16(lane_base + kColS + buf * 64 + c0, dsk);
             if (!seq) {
                 // the previous depth block's MMAs are done before its staging
                 // tiles and TMEM columns are reused
@@ -781,10 +790,11 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     tc_fence_after();
                     depth_epilogue(jd - 1);
                 }
-                // row r of the [q][depth] staging tiles, 128-byte swizzle
+                // row r of the [q][depth] staging tiles, 128-byte swizzle;
+                // this half's depth columns are 16-byte chunks 4*half .. 4*half+3
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint32_t off = r * 128 + ((ch ^ (r & 7)) << 4);
+                for (int ch = 0; ch < 4; ++ch) {
+                    const uint32_t off = r * 128 + (((4 * half + ch) ^ (r & 7)) << 4);
                     *reinterpret_cast<uint4*>(sDS + off) =
                         make_uint4(dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
                     *reinterpret_cast<uint4*>(sP + off) =
@@ -809,15 +819,16 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         if (ok) ok = mbar_wait(&bars[kB_Final], 0, a.status, abort_flag);
         if (ok) {
             tc_fence_after();
-            uint32_t o[D];
+            uint32_t o[D / 2];                                // this half's D/2 columns of dQ
 #pragma unroll
-            for (int c = 0; c < D; c += 32) tmem_ld32(lane_base + kColDQ + c, o + c);
+            for (int c = 0; c < D / 2; c += 32) tmem_ld32(lane_base + kColDQ + half * (D / 2) + c, o + c);
             tmem_wait_ld();
+            reg_fence<D / 2>(o);
             if (row_live) {
-                uint4* dst = reinterpret_cast<uint4*>(a.dQ + qrow * D);
+                uint4* dst = reinterpret_cast<uint4*>(a.dQ + qrow * D + half * (D / 2));
                 const float sc = a.scale;
 #pragma unroll
-                for (int c = 0; c < D; c += 8) {
+                for (int c = 0; c < D / 2; c += 8) {
                     uint4 v;
                     v.x = pack_bf16(__uint_as_float(o[c]) * sc, __uint_as_float(o[c + 1]) * sc);
                     v.y = pack_bf16(__uint_as_float(o[c + 2]) * sc, __uint_as_float(o[c + 3]) * sc);
