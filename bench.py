@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the L=0 twin and T=64K lines")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--configs", action="store_true",
+                    help="per-config kernel times against their rooflines (every workload, the "
+                         "G x L x C sweep, L = 0 twins); one JSON line, one GPU")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decoding path (one JSON line; small device footprint)")
     return ap.parse_args()
@@ -150,9 +153,9 @@ class Runner:
         self.x = x
         self.backward = backward
         dev = x["Q"].device
-        self.sh = moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C)
-        bf = torch.bfloat16
-        self.Kd = torch.empty(w.B, w.Hk, w.T * w.L, w.d, device=dev, dtype=bf) if w.L else None
+        self.sh = moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C,
+                                  moda.MODA_FP32 if w.dtype == "fp32" else moda.MODA_BF16)
+        self.Kd = torch.empty(w.B, w.Hk, w.T * w.L, w.d, device=dev, dtype=w.torch_dtype()) if w.L else None
         self.Vd = torch.empty_like(self.Kd) if w.L else None
         self.O = torch.empty_like(x["Q"])
         self.LSE = torch.empty(w.B, w.Hq, w.T, device=dev, dtype=torch.float32)
@@ -545,6 +548,104 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _median_ms(call, runs: int, flush: torch.Tensor) -> float:
+    """Median CUDA-event time of `call` over `runs` runs after 3 warm-up
+    calls, with L2 flushed (a 256 MB write) before every timed run."""
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(runs):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return float(np.median(times))
+
+
+def config_measure(w: I.Workload, peaks, flush: torch.Tensor, runs: int = 20, twin: bool = True):
+    """One workload: repack, forward and (for training workloads) backward
+    timed one call at a time; each against its attainable time
+    max(FLOPs / tensor peak, algorithmic bytes / HBM bandwidth)."""
+    import sequence_depth_attention_moda_b200 as moda
+    e = 2 if w.dtype == "bf16" else 4
+    x = I.make_inputs(w, device="cuda", grad_out=w.backward)
+
+    def one(wl):
+        r = Runner(wl, x, backward=wl.backward)
+        r.step()                                   # fills the token-major depth tensors
+        xx = r.x
+        fwd = lambda: moda.moda_fwd(r.sh, xx["Q"], xx["K"], xx["V"], r.Kd, r.Vd, r.O, r.LSE)
+        res = {"fwd_ms": _median_ms(fwd, runs, flush)}
+        if wl.backward:
+            bwd = lambda: moda.moda_bwd(r.sh, xx["Q"], xx["K"], xx["V"], r.Kd, r.Vd, r.O, r.LSE, xx["dO"],
+                                        r.dQ, r.dK, r.dV, r.dKd, r.dVd, r.ws, r.nws)
+            res["bwd_ms"] = _median_ms(bwd, runs, flush)
+        if wl.L:
+            def rep():
+                moda.moda_repack_depth(r.sh, xx["Kd_layer"], r.Kd)
+                moda.moda_repack_depth(r.sh, xx["Vd_layer"], r.Vd)
+            res["repack_ms"] = _median_ms(rep, runs, flush)
+        moda.moda_check_status()
+        del r
+        return res
+
+    def roof(flops, nbytes, ms):
+        t_tensor = flops / (peaks["bf16_tflops"] * 1e12) * 1e3
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+        att = max(t_tensor, t_hbm)
+        return {"ms": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+                "attainable_ms": round(att, 4), "frac_of_attainable": round(att / ms, 4)}
+
+    q_el = w.B * w.Hq * w.T * w.d
+    kv_el = w.B * w.Hk * w.T * w.d
+    dep_el = w.B * w.Hk * w.T * w.L * w.d
+    ff = w.fwd_flops()
+    out = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hk": w.Hk, "d": w.d, "T": w.T, "L": w.L, "C": w.C,
+           "dtype": w.dtype}
+    m = one(w)
+    out["fwd"] = roof(ff, e * (2 * q_el + 2 * kv_el + 2 * dep_el) + 4 * w.B * w.Hq * w.T, m["fwd_ms"])
+    if w.backward:
+        out["bwd"] = roof(BWD_FACTOR * ff, e * (4 * q_el + 4 * kv_el + 4 * dep_el) + 3 * 4 * w.B * w.Hq * w.T,
+                          m["bwd_ms"])
+    if w.L:
+        rb = 2 * 2 * dep_el * e
+        out["repack"] = {"ms": round(m["repack_ms"], 4), "gbs": round(rb / (m["repack_ms"] * 1e-3) / 1e9, 1),
+                         "frac_of_hbm": round(rb / (m["repack_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    if twin and w.L:
+        m0 = one(w.with_(L=0))
+        out["L0_fwd_ms"] = round(m0["fwd_ms"], 4)
+        out["fwd_time_vs_L0"] = round(m0["fwd_ms"] / m["fwd_ms"], 4)   # L=0 time / time: <= 1
+        if w.backward:
+            out["L0_bwd_ms"] = round(m0["bwd_ms"], 4)
+    del x
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_configs(args):
+    """Every workload's kernels against their rooflines (one GPU)."""
+    torch.cuda.set_device(0)
+    import sequence_depth_attention_moda_b200 as moda
+    moda.load()
+    peaks = load_peaks()
+    flush = torch.empty(256 << 20, device="cuda", dtype=torch.uint8)
+    rows = [config_measure(w, peaks, flush) for w in (I.TINY_FP32, I.LAYER_1P5B, I.LONG_64K, I.TRAIN_FWD_BWD)]
+    seen_g = set()
+    for w in I.depth_group_sweep():
+        rows.append(config_measure(w, peaks, flush, twin=w.G not in seen_g))
+        seen_g.add(w.G)
+    print(json.dumps({"metric": "per-config kernel time against max(FLOPs/peak, bytes/bandwidth)",
+                      "n_gpus": 1, "runs": 20, "warmup": 3, "l2": "flushed (256 MB write) before every run",
+                      "peaks": {"bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
+                                "source": peaks["source"]},
+                      "configs": rows}), flush=True)
+
+
 def run_decode_only(args):
     """The decoding workload alone (one GPU)."""
     torch.cuda.set_device(0)
@@ -561,6 +662,8 @@ def main():
         run_reference(args)
     elif args.decode_only:
         run_decode_only(args)
+    elif args.configs:
+        run_configs(args)
     else:
         run_ours(args)
 
