@@ -144,3 +144,45 @@ def test_decode_rejects_null_and_empty_batch(lib):
     sh0 = moda.make_shape(0, 4, 2, 64, 128, 2, 0)
     assert lib.moda_decode(ctypes.byref(sh0), *([None] * 7), None, 0, None) == 0
     assert moda.moda_decode_workspace_size(sh0) == 0
+
+
+def _decode_ranges_maxc(B, Hk, T, L, window, sms):
+    """Independent count of how many CTAs can share one KV head's items when
+    n items (per KV head: ceil(rows/64) depth tiles, then ceil(T/64) sequence
+    tiles) are cut into `sms` contiguous ranges of floor-divided bounds."""
+    rows = L - (L - window if 0 < window < L else 0)
+    per = -(-rows // 64) + -(-T // 64)
+    n = B * Hk * per
+    P = min(n, sms)
+    bounds = [c * n // P for c in range(P + 1)]
+    worst = 1
+    for bh in range(B * Hk):
+        first, last = bh * per, (bh + 1) * per - 1
+        ctas = [c for c in range(P) if bounds[c] <= last and bounds[c + 1] > first]
+        assert ctas == list(range(ctas[0], ctas[-1] + 1))
+        worst = max(worst, len(ctas))
+    return worst
+
+
+@pytest.mark.parametrize("B,Hq,Hk,T,d,L,window,dtype", [
+    (8, 32, 8, 32768, 128, 48, 0, moda.MODA_BF16),   # the decoding workload
+    (3, 16, 2, 4097, 128, 16, 4, moda.MODA_BF16),    # window; CTAs span KV heads
+    (64, 16, 8, 200, 64, 4, 0, moda.MODA_BF16),      # many KV heads per CTA
+    (1, 4, 4, 1, 64, 3, 0, moda.MODA_BF16),          # fewer items than SMs
+    (2, 8, 2, 1000, 128, 8, 0, moda.MODA_FP32),      # fp32: fixed splits
+])
+def test_decode_workspace_size(lib, B, Hq, Hk, T, d, L, window, dtype):
+    """Workspace = one (m, l, o[d]) fp32 record per query head, per CTA that
+    can share its KV head's items, per consumer warp (bf16); fp32: per split
+    (>= 256 keys each, about 4 CTAs per SM) plus the depth split, per warp.
+    Without a GPU the library assumes a 148-SM B200."""
+    sh = moda.make_shape(B, Hq, Hk, T, d, L, 0, dtype, depth_window=window)
+    got = lib.moda_decode_workspace_size(ctypes.byref(sh))
+    if dtype == moda.MODA_BF16:
+        parts = _decode_ranges_maxc(B, Hk, T, L, window, 148) * 3
+    else:
+        want = -(-4 * 148 // (B * Hk))
+        splits = max(1, min(want, -(-T // 256)))
+        parts = (splits + (1 if L > 0 else 0)) * 8
+    need = B * Hq * parts * (d + 2) * 4
+    assert got == -(-need // 256) * 256, (got, need)
