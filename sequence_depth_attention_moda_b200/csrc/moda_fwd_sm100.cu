@@ -390,8 +390,29 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 if (tr) MODA_TRF(6, j);
                 if (tr2) MODA_TRF(12, j);
                 tc_fence_after();
-                uint32_t sr[64];
                 const uint32_t s_addr = lane_base + sb * 128;
+                if (i >= n_seq) {
+                    // A depth block none of the warp's 16 rows can see (each
+                    // row sees only its own token's rows): every score would be
+                    // masked to -inf, so P is exactly 0 and the row sums do not
+                    // change.  Write the zeros without loading or exponentiating.
+                    const int base = t_row * a.L - (t0 * a.L + (i - n_seq) * a.dep_rows) - c0;
+                    const int vis_lo = max(base + a.win_lo, 0);
+                    const int vis_hi = min(min(base + a.L, a.dep_rows - c0), 64);
+                    if (__all_sync(0xffffffffu, vis_lo >= vis_hi)) {
+                        uint32_t zero[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) zero[c] = 0u;
+                        __syncwarp();
+                        tmem_st16x2_32<32>(s_addr, zero);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars[kPReady + sb]);
+                        continue;
+                    }
+                }
+                uint32_t sr[64];
                 tmem_ld16x2_32<64>(s_addr, sr);            // columns c0 .. c0+31
                 tmem_ld16x2_32<64>(s_addr + 32, sr + 32);  // columns c0+32 .. c0+63
                 tmem_wait_ld();
