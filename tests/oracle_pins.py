@@ -414,3 +414,20 @@ ALL_PINS = [pin_decode_is_last_row, pin_l0_is_causal_sdpa, pin_t1_self_plus_dept
             pin_gqa_is_repeat_interleave, pin_convexity, pin_bwd_autograd,
             pin_bwd_finite_differences, pin_repack_definition, pin_noncausal_l0_is_sdpa,
             pin_modes_dense_bruteforce, pin_window_is_truncated_depth, pin_modes_bwd_autograd]
+
+
+def pin_worked_example(lib):
+    """The exact worked example (tests/golden): forward, LSE and all five
+    gradients equal values derived by hand-checkable Fraction arithmetic
+    from the definition, to 1e-12."""
+    from worked_example import load
+    x, e = load()
+    O, LSE = oracle.fwd(x["Q"], x["K"], x["V"], x["Kd"], x["Vd"], lib=lib)
+    _close(O, e["O"], 1e-12, "worked example O")
+    _close(LSE, e["LSE"], 1e-12, "worked example LSE")
+    grads = oracle.bwd(x["Q"], x["K"], x["V"], x["Kd"], x["Vd"], x["dO"], lib=lib)
+    for name, got in zip(("dQ", "dK", "dV", "dKd", "dVd"), grads):
+        _close(got, e[name], 1e-12, f"worked example {name}")
+
+
+ALL_PINS.append(pin_worked_example)

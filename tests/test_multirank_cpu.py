@@ -41,7 +41,7 @@ def _worker(rank, world, port, out):
 @pytest.mark.timeout(120)
 def test_two_gloo_ranks_time_max_and_distinct_batches():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # no fork of a threaded process
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, join=True,
                        start_method="spawn")

@@ -53,3 +53,22 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"no pin caught the planted mistake {name}"
+
+
+# The exact worked example alone decides every mutant of the default
+# (causal, full-depth) operator; the modes and the repack have their own pins.
+WORKED_EXAMPLE_CATCHES = [m for m in MUTANTS if m[0] not in
+                          ("noncausal_ignored", "depth_window_ignored", "repack_layer_major_kept")]
+
+
+@pytest.mark.parametrize("name,old,new", WORKED_EXAMPLE_CATCHES, ids=[m[0] for m in WORKED_EXAMPLE_CATCHES])
+def test_worked_example_alone_catches(tmp_path, name, old, new):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "mutant.c"
+    src.write_text(open(SRC).read().replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", str(src), "-o", str(so), "-lm"])
+    lib = oracle.load_library(str(so))
+    with pytest.raises(AssertionError):
+        oracle_pins.pin_worked_example(lib)
