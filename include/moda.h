@@ -223,7 +223,10 @@ moda_status moda_check_status(moda_stream_t stream);
  *   o         [B, Hq, d]     output, same dtype            (device)
  *   lse       [B, Hq]        fp32 natural-log LSE          (device)
  *   ws        moda_decode_workspace_size(shape) bytes      (device, caller-owned)
- * All buffers are contiguous and 16-byte aligned; nothing is allocated.
+ * All buffers are contiguous and 16-byte aligned; nothing is allocated.  The
+ * workspace holds fp32 partial results whose count follows the key split,
+ * which depends on the current device's SM count: query the size with the
+ * device that runs the call current (148 SMs are assumed without a device).
  * Returns MODA_ERR_INVALID_ARG / MODA_ERR_UNSUPPORTED for shapes outside the
  * above, MODA_ERR_MISALIGNED, MODA_ERR_WORKSPACE if ws_bytes is too small.
  */
