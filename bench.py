@@ -634,13 +634,17 @@ def run_configs(args):
     moda.load()
     peaks = load_peaks()
     flush = torch.empty(256 << 20, device="cuda", dtype=torch.uint8)
-    rows = [config_measure(w, peaks, flush) for w in (I.TINY_FP32, I.LAYER_1P5B, I.LONG_64K, I.TRAIN_FWD_BWD)]
-    seen_g = set()
-    for w in I.depth_group_sweep():
-        rows.append(config_measure(w, peaks, flush, twin=w.G not in seen_g))
-        seen_g.add(w.G)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(int(vis.split(",")[0]) if vis else 0)
+    with clocks:
+        rows = [config_measure(w, peaks, flush) for w in (I.TINY_FP32, I.LAYER_1P5B, I.LONG_64K, I.TRAIN_FWD_BWD)]
+        seen_g = set()
+        for w in I.depth_group_sweep():
+            rows.append(config_measure(w, peaks, flush, twin=w.G not in seen_g))
+            seen_g.add(w.G)
     print(json.dumps({"metric": "per-config kernel time against max(FLOPs/peak, bytes/bandwidth)",
                       "n_gpus": 1, "runs": 20, "warmup": 3, "l2": "flushed (256 MB write) before every run",
+                      "clocks": clocks.summary(),
                       "peaks": {"bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
                                 "source": peaks["source"]},
                       "configs": rows}), flush=True)
