@@ -115,10 +115,22 @@ def make_shape(B, Hq, Hk, T, d, L, C=0, dtype=MODA_BF16, depth_layout=MODA_DEPTH
 
 
 def _ptr(x) -> Optional[int]:
+    """Device address of a buffer argument: None, a raw int address (passed
+    through), or a tensor that must be contiguous and on the current CUDA
+    device (the kernels read row-major device memory; a host or strided
+    tensor is rejected here rather than read wrongly)."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if not x.is_cuda:
+        raise MoDAError(MODA_ERR_INVALID_ARG, "argument", f"tensor on {x.device}, not a CUDA device")
+    if not x.is_contiguous():
+        raise MoDAError(MODA_ERR_INVALID_ARG, "argument", "tensor is not contiguous (row-major)")
+    import torch
+    if x.device.index != torch.cuda.current_device():
+        raise MoDAError(MODA_ERR_INVALID_ARG, "argument",
+                        f"tensor on {x.device}, current device is cuda:{torch.cuda.current_device()}")
     return x.data_ptr()
 
 

@@ -186,3 +186,16 @@ def test_decode_workspace_size(lib, B, Hq, Hk, T, d, L, window, dtype):
         parts = (splits + (1 if L > 0 else 0)) * 8
     need = B * Hq * parts * (d + 2) * 4
     assert got == -(-need // 256) * 256, (got, need)
+
+
+def test_binding_rejects_host_tensors(lib):
+    """A host tensor would hand the kernels a host address: the binding
+    refuses it before calling the library."""
+    import torch
+    sh = moda.make_shape(1, 4, 2, 64, 128, 2, 0)
+    q = torch.zeros(1, 4, 64, 128, dtype=torch.bfloat16)
+    with pytest.raises(moda.MoDAError) as err:
+        moda.moda_fwd(sh, q, None, None, None, None, None, None)
+    assert err.value.status == moda.MODA_ERR_INVALID_ARG and "cpu" in str(err.value)
+    with pytest.raises(moda.MoDAError):
+        moda.moda_decode(sh, torch.zeros(1, 4, 128), *([None] * 6), None, 0)
