@@ -23,11 +23,51 @@ BF16_MAX_ABS, BF16_MEAN_ABS = 2e-2, 2e-3
 FP32_MAX_ABS = 1e-4
 # LSE is fp32 statistics of exactly representable scores: tight.
 LSE_MAX_ABS = 1e-3
-# gradients (the pages state none): max |g - ref| <= 2e-2 * max(1, max|ref|) and
-# mean |g - ref| <= 5e-3 * max(1, mean|ref|).  Rounding a gradient to bf16 on
-# store costs up to 2^-9 relative (about 2e-3 on average over a tensor), and the
-# bf16 P / dS operands of the tensor-core products add the same order again.
-GRAD_MAX_REL, GRAD_MEAN_REL = 2e-2, 5e-3
+# gradients (the pages state none), each bound relative to the reference
+# tensor's own scale, with no absolute floor:
+#   ||g - ref||_2 <= 1e-2 * ||ref||_2
+#   max |g - ref| <= 2e-2 * max |ref|
+#   mean|g - ref| <= 5e-3 * mean|ref|
+# Rounding a gradient to bf16 on store costs up to 2^-9 relative (about 1e-3 on
+# average), and the bf16 P / dS operands of the tensor-core products add the
+# same order again; a reference of exact zeros must come back exactly zero.
+GRAD_NORM_REL, GRAD_MAX_REL, GRAD_MEAN_REL = 1e-2, 2e-2, 5e-3
+
+# Every output the tests allocate sits between two guard bands of this many
+# bytes filled with GUARD_BYTE, and is filled with NaN before the call: after
+# the call the bands must be intact (nothing written outside the tensor) and
+# no NaN may remain (every element written).
+GUARD_BYTES = 4096
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """Outputs allocated inside larger buffers with guard bands (a stand-in
+    for a memory checker: the kernels' stores must stay inside their tensors
+    and cover every element)."""
+
+    def __init__(self):
+        self.items = []
+
+    def empty(self, name: str, shape, dtype, device) -> torch.Tensor:
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        raw = torch.full((2 * GUARD_BYTES + n,), GUARD_BYTE, dtype=torch.uint8, device=device)
+        view = raw[GUARD_BYTES:GUARD_BYTES + n].view(dtype).view(*shape)
+        view.fill_(float("nan"))
+        self.items.append((name, raw, n, view))
+        return view
+
+    def like(self, name: str, t: torch.Tensor) -> torch.Tensor:
+        return self.empty(name, tuple(t.shape), t.dtype, t.device)
+
+    def check(self):
+        if any(raw.is_cuda for _, raw, _, _ in self.items):
+            torch.cuda.synchronize()
+        for name, raw, n, view in self.items:
+            head, tail = raw[:GUARD_BYTES], raw[GUARD_BYTES + n:]
+            assert bool((head == GUARD_BYTE).all()), f"{name}: bytes written before the tensor"
+            assert bool((tail == GUARD_BYTE).all()), f"{name}: bytes written past the end of the tensor"
+            assert not bool(torch.isnan(view).any()), f"{name}: elements left unwritten"
 
 
 def shape_of(w: Workload, layout=moda.MODA_DEPTH_FLAT, C=None):
@@ -40,34 +80,37 @@ def shape_of(w: Workload, layout=moda.MODA_DEPTH_FLAT, C=None):
 def run_gpu(w: Workload, x: Dict[str, torch.Tensor], backward=None, layout=moda.MODA_DEPTH_FLAT,
             C=None, null_depth_if_empty=True):
     """Repack the depth cache, run the forward (and backward) on the current
-    stream; returns a dict of device tensors."""
+    stream; returns a dict of device tensors.  Every output is guarded
+    (``Guarded``) and checked before returning."""
     sh = shape_of(w, layout, C)
     dev = x["Q"].device
     dt = x["Q"].dtype
+    gd = Guarded()
     out = {}
     if w.L > 0:
-        Kd = torch.empty(w.B, w.Hk, w.T * w.L, w.d, device=dev, dtype=dt)
-        Vd = torch.empty_like(Kd)
+        Kd = gd.empty("Kd", (w.B, w.Hk, w.T * w.L, w.d), dt, dev)
+        Vd = gd.empty("Vd", (w.B, w.Hk, w.T * w.L, w.d), dt, dev)
         moda.moda_repack_depth(sh, x["Kd_layer"], Kd)
         moda.moda_repack_depth(sh, x["Vd_layer"], Vd)
     else:
         Kd = Vd = None if null_depth_if_empty else torch.empty(0, device=dev, dtype=dt)
     out["Kd"], out["Vd"] = Kd, Vd
-    O = torch.empty_like(x["Q"])
-    LSE = torch.empty(w.B, w.Hq, w.T, device=dev, dtype=torch.float32)
+    O = gd.like("O", x["Q"])
+    LSE = gd.empty("LSE", (w.B, w.Hq, w.T), torch.float32, dev)
     moda.moda_fwd(sh, x["Q"], x["K"], x["V"], Kd, Vd, O, LSE)
     out["O"], out["LSE"] = O, LSE
     if backward if backward is not None else w.backward:
         nws = moda.moda_workspace_size(sh, True)
         ws = torch.empty(max(nws, 16), device=dev, dtype=torch.uint8)
-        dQ = torch.empty_like(x["Q"])
-        dK = torch.empty_like(x["K"])
-        dV = torch.empty_like(x["V"])
-        dKd = torch.empty_like(Kd) if Kd is not None else None
-        dVd = torch.empty_like(Vd) if Vd is not None else None
+        dQ = gd.like("dQ", x["Q"])
+        dK = gd.like("dK", x["K"])
+        dV = gd.like("dV", x["V"])
+        dKd = gd.like("dKd", Kd) if Kd is not None and Kd.numel() else None
+        dVd = gd.like("dVd", Vd) if Vd is not None and Vd.numel() else None
         moda.moda_bwd(sh, x["Q"], x["K"], x["V"], Kd, Vd, O, LSE, x["dO"], dQ, dK, dV, dKd, dVd,
                       ws, nws)
         out.update(dQ=dQ, dK=dK, dV=dV, dKd=dKd, dVd=dVd)
+    gd.check()
     return out
 
 
@@ -172,14 +215,29 @@ def assert_out_close(got, ref, dtype: str, what: str):
             f"{what}: max-abs {mx:.3e} (<= {BF16_MAX_ABS}), mean-abs {mean:.3e} (<= {BF16_MEAN_ABS})"
 
 
+def grad_errors(got, ref) -> Dict[str, float]:
+    """Normwise, max and mean errors of a gradient and the reference scales."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    d = np.abs(got - ref)
+    return {"norm_err": float(np.sqrt((d * d).sum())), "norm_ref": float(np.sqrt((ref * ref).sum())),
+            "max_err": float(d.max()), "max_ref": float(np.abs(ref).max()),
+            "mean_err": float(d.mean()), "mean_ref": float(np.abs(ref).mean())}
+
+
 def assert_grad_close(got, ref, what: str):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} != {ref.shape}"
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     if ref.size == 0:
         return
-    mx, mean = err_stats(got, ref)
-    lim_mx = GRAD_MAX_REL * max(1.0, float(np.abs(ref).max()))
-    lim_mean = GRAD_MEAN_REL * max(1.0, float(np.abs(ref).mean()))
-    assert mx <= lim_mx and mean <= lim_mean, \
-        f"{what}: max-abs {mx:.3e} (<= {lim_mx:.3e}), mean-abs {mean:.3e} (<= {lim_mean:.3e})"
+    e = grad_errors(got, ref)
+    if e["norm_ref"] == 0.0:
+        assert e["max_err"] == 0.0, f"{what}: reference is exactly zero, max-abs {e['max_err']:.3e}"
+        return
+    ok = (e["norm_err"] <= GRAD_NORM_REL * e["norm_ref"] and e["max_err"] <= GRAD_MAX_REL * e["max_ref"]
+          and e["mean_err"] <= GRAD_MEAN_REL * e["mean_ref"])
+    assert ok, (f"{what}: normwise {e['norm_err'] / e['norm_ref']:.3e} (<= {GRAD_NORM_REL}), "
+                f"max-abs {e['max_err']:.3e} (<= {GRAD_MAX_REL * e['max_ref']:.3e}), "
+                f"mean-abs {e['mean_err']:.3e} (<= {GRAD_MEAN_REL * e['mean_ref']:.3e})")

@@ -8,7 +8,7 @@ import torch
 import oracle
 import sequence_depth_attention_moda_b200 as moda
 from sequence_depth_attention_moda_b200 import inputs as I
-from moda_cases import BF16_MAX_ABS, BF16_MEAN_ABS, FP32_MAX_ABS, LSE_MAX_ABS, err_stats, f64
+from moda_cases import BF16_MAX_ABS, BF16_MEAN_ABS, FP32_MAX_ABS, LSE_MAX_ABS, Guarded, err_stats, f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -28,10 +28,12 @@ def run_decode(w, x):
                          depth_window=w.window)
     nws = moda.moda_decode_workspace_size(sh)
     ws = torch.empty(max(nws, 16), device=DEV, dtype=torch.uint8)
-    o = torch.empty_like(x["q"])
-    lse = torch.empty(w.B, w.Hq, device=DEV, dtype=torch.float32)
+    gd = Guarded()
+    o = gd.like("o", x["q"])
+    lse = gd.empty("lse", (w.B, w.Hq), torch.float32, DEV)
     moda.moda_decode(sh, x["q"], x["K"], x["V"], x["Kd"] if w.L else None, x["Vd"] if w.L else None,
                      o, lse, ws, nws)
+    gd.check()
     return o, lse
 
 

@@ -46,7 +46,7 @@ def test_oracle_reproduces_worked_example():
 @pytest.mark.gpu
 def test_cuda_fp32_path_reproduces_worked_example():
     import sequence_depth_attention_moda_b200 as moda
-    from moda_cases import FP32_MAX_ABS
+    from moda_cases import FP32_MAX_ABS, Guarded
     if not torch.cuda.is_available():
         pytest.fail("CUDA device required for -m gpu tests")
     x, e = load()
@@ -56,14 +56,16 @@ def test_cuda_fp32_path_reproduces_worked_example():
     Q, K, V, dO = dev(x["Q"]), dev(x["K"]), dev(x["V"]), dev(x["dO"])
     Kd, Vd = dev(x["Kd"]), dev(x["Vd"])
     sh = moda.make_shape(B, Hq, Hk, T, d, L, 0, moda.MODA_FP32)
-    O = torch.empty_like(Q)
-    LSE = torch.empty(B, Hq, T, device="cuda", dtype=torch.float32)
+    gd = Guarded()
+    O = gd.like("O", Q)
+    LSE = gd.empty("LSE", (B, Hq, T), torch.float32, "cuda")
     moda.moda_fwd(sh, Q, K, V, Kd, Vd, O, LSE)
     nws = moda.moda_workspace_size(sh, True)
     ws = torch.empty(max(nws, 16), device="cuda", dtype=torch.uint8)
-    g = [torch.empty_like(t) for t in (Q, K, V, Kd, Vd)]
+    g = [gd.like(n, t) for n, t in zip(("dQ", "dK", "dV", "dKd", "dVd"), (Q, K, V, Kd, Vd))]
     moda.moda_bwd(sh, Q, K, V, Kd, Vd, O, LSE, dO, *g, ws, nws)
     moda.moda_check_status()
+    gd.check()
     got = {"O": O, "LSE": LSE, "dQ": g[0], "dK": g[1], "dV": g[2], "dKd": g[3], "dVd": g[4]}
     for name, t in got.items():
         np.testing.assert_allclose(t.double().cpu().numpy(), e[name], rtol=0, atol=FP32_MAX_ABS,

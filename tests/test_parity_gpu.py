@@ -2,12 +2,14 @@
 on the same seeded inputs.
 
 Tolerances (bf16 in / fp32 accumulate): output max-abs <= 2e-2 and mean-abs
-<= 2e-3; fp32 path max-abs <= 1e-4; LSE max-abs <= 1e-3; gradients max-abs <=
-2e-2 * max(1, max|ref|) and mean-abs <= 5e-3 * max(1, mean|ref|) (storing a
-gradient in bf16 alone costs up to ~2e-3 relative on average).  Small
-cases are compared element by element in full; the full-size workloads on
-sampled rows (forward) and sampled (b, hk) slices (backward), which the
-oracle computes exactly for what they cover.
+<= 2e-3; fp32 path max-abs <= 1e-4; LSE max-abs <= 1e-3; gradients relative
+to each reference tensor's own scale, with no floor: normwise <= 1e-2,
+max-abs <= 2e-2 * max|ref|, mean-abs <= 5e-3 * mean|ref| (storing a gradient
+in bf16 alone costs up to 2^-9 relative).  Small cases are compared element
+by element in full; the full-size workloads on sampled rows (forward) and
+sampled (b, hk) slices (backward), which the oracle computes exactly for what
+they cover.  Every output sits between guard bands and starts as NaN (see
+moda_cases.Guarded): writes outside a tensor or elements left unwritten fail.
 """
 import numpy as np
 import pytest
@@ -202,14 +204,14 @@ def test_bwd_layer_T4k_sampled_slices():
     x = I.make_inputs(w, device=DEV)
     out = run_gpu(w, x)
     _check_rows(w, x, out)
-    _check_slices(w, x, out, [(1, 3)])
+    _check_slices(w, x, out, [(0, 0), (0, 2), (1, 1), (w.B - 1, w.Hk - 1)])
 
 
 def test_bwd_train_shape_sampled_slice():
     w = I.TRAIN_FWD_BWD
     x = I.make_inputs(w, device=DEV)
     out = run_gpu(w, x)
-    _check_slices(w, x, out, [(7, 5)])
+    _check_slices(w, x, out, [(0, 0), (2, 6), (5, 3), (w.B - 1, w.Hk - 1)])
 
 
 def test_bwd_deterministic():
