@@ -143,6 +143,31 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
+def _expect(where: str, shape: moda_shape, specs):
+    """Check tensor arguments against the shape before the C call: each spec
+    is (name, tensor or int or None, element count, "io" or "f32").  A tensor
+    must hold at least that many elements of the shape's dtype ("io") or of
+    float32 ("f32"); raw integer addresses and None pass through (the library
+    checks NULL itself)."""
+    import torch
+    io = torch.bfloat16 if shape.dtype == MODA_BF16 else torch.float32
+    for name, x, count, kind in specs:
+        if x is None or isinstance(x, int):
+            continue
+        want = torch.float32 if kind == "f32" else io
+        if x.dtype != want:
+            raise MoDAError(MODA_ERR_INVALID_ARG, where, f"{name} has dtype {x.dtype}, expected {want}")
+        if x.numel() < count:
+            raise MoDAError(MODA_ERR_INVALID_ARG, where,
+                            f"{name} holds {x.numel()} elements, the shape needs {count}")
+
+
+def _sizes(shape: moda_shape):
+    B, Hq, Hk, T, d, L = (max(0, int(v)) for v in (shape.B, shape.Hq, shape.Hk, shape.T, shape.d,
+                                                   shape.L))
+    return {"q": B * Hq * T * d, "kv": B * Hk * T * d, "dep": B * Hk * T * L * d, "lse": B * Hq * T}
+
+
 def _check(rc: int, where: str):
     if rc != MODA_OK:
         detail = load().moda_last_error_message().decode()
@@ -157,17 +182,43 @@ def moda_workspace_size(shape: moda_shape, for_bwd: bool) -> int:
 
 
 def moda_repack_depth(shape: moda_shape, src, dst, stream=None):
+    n = _sizes(shape)["dep"]
+    _expect("moda_repack_depth", shape, [("src", src, n, "io"), ("dst", dst, n, "io")])
     _check(load().moda_repack_depth(ctypes.byref(shape), _ptr(src), _ptr(dst), _stream(stream)),
            "moda_repack_depth")
 
 
 def moda_fwd(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, ws=None, ws_bytes: int = 0, stream=None):
+    n = _sizes(shape)
+    _expect("moda_fwd", shape, [("Q", Q, n["q"], "io"), ("K", K, n["kv"], "io"), ("V", V, n["kv"], "io"),
+                                ("Kd", Kd, n["dep"], "io"), ("Vd", Vd, n["dep"], "io"),
+                                ("O", O, n["q"], "io"), ("LSE", LSE, n["lse"], "f32")])
     _check(load().moda_fwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd),
                            _ptr(O), _ptr(LSE), _ptr(ws), int(ws_bytes), _stream(stream)), "moda_fwd")
 
 
+def _bwd_specs(shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd):
+    n = _sizes(shape)
+    return [("Q", Q, n["q"], "io"), ("K", K, n["kv"], "io"), ("V", V, n["kv"], "io"),
+            ("Kd", Kd, n["dep"], "io"), ("Vd", Vd, n["dep"], "io"), ("O", O, n["q"], "io"),
+            ("LSE", LSE, n["lse"], "f32"), ("dO", dO, n["q"], "io"), ("dQ", dQ, n["q"], "io"),
+            ("dK", dK, n["kv"], "io"), ("dV", dV, n["kv"], "io"), ("dKd", dKd, n["dep"], "io"),
+            ("dVd", dVd, n["dep"], "io")]
+
+
+def _check_ws(where: str, ws, ws_bytes: int):
+    """A workspace tensor must hold the ws_bytes the call claims."""
+    if ws is None or isinstance(ws, int):
+        return
+    have = ws.numel() * ws.element_size()
+    if have < int(ws_bytes):
+        raise MoDAError(MODA_ERR_INVALID_ARG, where, f"ws holds {have} bytes, ws_bytes says {int(ws_bytes)}")
+
+
 def moda_bwd(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, ws,
              ws_bytes: int, stream=None):
+    _expect("moda_bwd", shape, _bwd_specs(shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd))
+    _check_ws("moda_bwd", ws, ws_bytes)
     _check(load().moda_bwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd),
                            _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dKd),
                            _ptr(dVd), _ptr(ws), int(ws_bytes), _stream(stream)), "moda_bwd")
@@ -178,6 +229,8 @@ def moda_bwd_noalloc(shape: moda_shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV,
     """moda_bwd for callers that cannot allocate: no workspace argument; the
     library's built-in scratch holds at most B*Hq*T = 4,194,304 query rows,
     and overlapping calls on the GPU share (and race on) that scratch."""
+    _expect("moda_bwd_noalloc", shape, _bwd_specs(shape, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd,
+                                                  dVd))
     _check(load().moda_bwd_noalloc(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kd),
                                    _ptr(Vd), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK),
                                    _ptr(dV), _ptr(dKd), _ptr(dVd), _stream(stream)),
@@ -206,6 +259,13 @@ def moda_decode_workspace_size(shape: moda_shape) -> int:
 
 
 def moda_decode(shape: moda_shape, q, K, V, Kd, Vd, o, lse, ws, ws_bytes: int, stream=None):
+    B, Hq, Hk, T, d, L = (max(0, int(v)) for v in (shape.B, shape.Hq, shape.Hk, shape.T, shape.d,
+                                                   shape.L))
+    _expect("moda_decode", shape, [("q", q, B * Hq * d, "io"), ("K", K, B * Hk * T * d, "io"),
+                                   ("V", V, B * Hk * T * d, "io"), ("Kd", Kd, B * Hk * L * d, "io"),
+                                   ("Vd", Vd, B * Hk * L * d, "io"), ("o", o, B * Hq * d, "io"),
+                                   ("lse", lse, B * Hq, "f32")])
+    _check_ws("moda_decode", ws, ws_bytes)
     _check(load().moda_decode(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V), _ptr(Kd), _ptr(Vd),
                               _ptr(o), _ptr(lse), _ptr(ws), int(ws_bytes), _stream(stream)),
            "moda_decode")

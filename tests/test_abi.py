@@ -199,3 +199,37 @@ def test_binding_rejects_host_tensors(lib):
     assert err.value.status == moda.MODA_ERR_INVALID_ARG and "cpu" in str(err.value)
     with pytest.raises(moda.MoDAError):
         moda.moda_decode(sh, torch.zeros(1, 4, 128), *([None] * 6), None, 0)
+
+
+def test_binding_rejects_wrong_dtype_and_short_tensors(lib):
+    """A tensor of the wrong dtype, or with fewer elements than the shape
+    implies, would let the kernels read or write past its end: the binding
+    refuses it before calling the library (checked before the device check,
+    so host tensors show it here)."""
+    import torch
+    sh = moda.make_shape(1, 4, 2, 64, 128, 2, 0)
+    bf = dict(dtype=torch.bfloat16)
+    Q, K = torch.zeros(1, 4, 64, 128, **bf), torch.zeros(1, 2, 64, 128, **bf)
+    Kd = torch.zeros(1, 2, 128, 128, **bf)
+    LSE = torch.zeros(1, 4, 64)
+    cases = [
+        (dict(Q=Q.float()), "Q has dtype"),
+        (dict(Kd=Kd[:, :, :100]), "Kd holds"),
+        (dict(LSE=LSE.to(torch.bfloat16)), "LSE has dtype"),
+        (dict(LSE=LSE[:, :, :10]), "LSE holds"),
+    ]
+    for over, msg in cases:
+        a = dict(Q=Q, K=K, V=K, Kd=Kd, Vd=Kd, O=Q, LSE=LSE)
+        a.update(over)
+        with pytest.raises(moda.MoDAError) as err:
+            moda.moda_fwd(sh, a["Q"], a["K"], a["V"], a["Kd"], a["Vd"], a["O"], a["LSE"])
+        assert err.value.status == moda.MODA_ERR_INVALID_ARG and msg in str(err.value), str(err.value)
+    # backward: a short dVd; decoding: a short o; repack: a short destination
+    with pytest.raises(moda.MoDAError, match="dVd holds"):
+        moda.moda_bwd(sh, Q, K, K, Kd, Kd, Q, LSE, Q, Q, K, K, Kd, Kd[:, :1], None, 0)
+    with pytest.raises(moda.MoDAError, match="o holds"):
+        moda.moda_decode(sh, torch.zeros(1, 4, 128, **bf), K, K, torch.zeros(1, 2, 2, 128, **bf),
+                         torch.zeros(1, 2, 2, 128, **bf), torch.zeros(1, 4, 64, **bf),
+                         torch.zeros(1, 4), None, 0)
+    with pytest.raises(moda.MoDAError, match="dst holds"):
+        moda.moda_repack_depth(sh, torch.zeros(2, 1, 2, 64, 128, **bf), Kd[:, :1])
