@@ -4,6 +4,7 @@
 // caller-provided workspace.  The pages have no counterpart to this.
 #include <cstdio>
 #include <mutex>
+#include <utility>
 
 #include "moda.h"
 #include "moda_internal.h"
@@ -44,7 +45,20 @@ moda_status scratch_for_current_device(float** out) {
     return MODA_OK;
 }
 
-bool bad_ptr(const void* p) { return !p || (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+// The same pointer rules and status codes as moda_bwd: NULL is an invalid
+// argument, an address off a 16-byte boundary is misaligned.
+moda_status check_ptr(const void* p, const char* name) {
+    char msg[120];
+    if (!p) {
+        snprintf(msg, sizeof(msg), "moda_bwd_noalloc: %s is NULL", name);
+        return api_fail(MODA_ERR_INVALID_ARG, msg);
+    }
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) {
+        snprintf(msg, sizeof(msg), "moda_bwd_noalloc: %s is not 16-byte aligned", name);
+        return api_fail(MODA_ERR_MISALIGNED, msg);
+    }
+    return MODA_OK;
+}
 
 }  // namespace
 }  // namespace moda
@@ -60,14 +74,15 @@ extern "C" moda_status moda_bwd_noalloc(const moda_shape* shape, const void* Q, 
     moda_status st = api_validate(shape, &p);
     if (st != MODA_OK) return st;
     if (p.B == 0 || p.T == 0) return MODA_OK;
-    const void* need[] = {Q, K, V, O, LSE, dO, dQ, dK, dV};
-    for (const void* ptr : need)
-        if (bad_ptr(ptr))
-            return api_fail(ptr ? MODA_ERR_MISALIGNED : MODA_ERR_INVALID_ARG,
-                            "moda_bwd_noalloc: a tensor pointer is NULL or not 16-byte aligned");
-    if (p.L > 0 && (bad_ptr(Kd) || bad_ptr(Vd) || bad_ptr(dKd) || bad_ptr(dVd)))
-        return api_fail(MODA_ERR_INVALID_ARG,
-                        "moda_bwd_noalloc: depth pointers must be non-NULL and 16-byte aligned when L > 0");
+    const std::pair<const void*, const char*> need[] = {
+        {Q, "Q"}, {K, "K"}, {V, "V"}, {O, "O"}, {LSE, "LSE"}, {dO, "dO"}, {dQ, "dQ"}, {dK, "dK"}, {dV, "dV"}};
+    for (const auto& pr : need)
+        if ((st = check_ptr(pr.first, pr.second)) != MODA_OK) return st;
+    if (p.L > 0) {
+        const std::pair<const void*, const char*> dep[] = {{Kd, "Kd"}, {Vd, "Vd"}, {dKd, "dKd"}, {dVd, "dVd"}};
+        for (const auto& pr : dep)
+            if ((st = check_ptr(pr.first, pr.second)) != MODA_OK) return st;
+    }
     const size_t rows = size_t(p.B) * p.Hq * p.T;
     if (rows > kScratchRows) {
         char msg[200];
@@ -82,6 +97,7 @@ extern "C" moda_status moda_bwd_noalloc(const moda_shape* shape, const void* Q, 
     // D rows need no clearing: the first kernel of the call writes every row
     // of [0, B*Hq*T) before any later kernel reads it.
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    phase_mark(0, s);
     cudaError_t e =
         p.elem_bytes == 2
             ? launch_bwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, scratch, s)
