@@ -14,8 +14,10 @@
  *   O[b,h,t]   = sum_j P_j V[b,hk,j] + sum_l P'_l Vd[b,hk,t*L + l]
  *   LSE[b,h,t] = natural-log log-sum-exp of the row
  *
- * scale = 1/sqrt(d) unless moda_shape.softmax_scale > 0.  The operator is
- * causal only (the pages list the non-causal kernel as unreleased).
+ * scale = 1/sqrt(d) unless moda_shape.softmax_scale > 0.  By default the
+ * operator is causal as written above; MODA_FLAG_NONCAUSAL (the non-causal
+ * kernel the pages list as unreleased) and moda_shape.depth_window (bounded
+ * depth slots) change only which keys and depth rows a row sees.
  *
  * Conventions for every entry point:
  *  - Tensors are dense, contiguous, row-major, in device memory, with base
@@ -172,7 +174,8 @@ moda_status moda_bwd(const moda_shape* shape,
  * per query row) is a fixed 16 MiB array inside the library, so it accepts at
  * most B*Hq*T = 4,194,304 query rows; larger problems get MODA_ERR_WORKSPACE.
  * Every device that loads the library holds that array until the process
- * exits.  The first call on a device looks up the array's device address
+ * exits.  Phase markers (moda_set_phase_events) apply as for moda_bwd.
+ * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture.  All calls share the one array, and each call
  * writes every row it reads before reading it, so nothing needs clearing

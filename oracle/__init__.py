@@ -20,9 +20,12 @@ definitions it follows:
 
 ``decode`` evaluates the newest token's rows through the same C row function.
 
-Parity status: the forward, backward and repack are pinned by the CPU tests in
-``tests/test_oracle.py`` (library special cases, closed forms, invariants, an
-independent dense brute force, autograd and finite differences).
+Parity status: the forward, backward and repack are pinned by the CPU tests
+(the pins live in ``tests/oracle_pins.py`` and run from ``tests/test_oracle.py``):
+library special cases, closed forms, invariants, an independent dense brute
+force, autograd, finite differences and an exact worked example
+(``tests/golden/``); ``tests/test_oracle_mutants.py`` checks that planted
+mistakes fail them.
 """
 from __future__ import annotations
 

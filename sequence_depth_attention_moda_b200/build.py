@@ -56,16 +56,13 @@ def _compile(src: str, force: bool, verbose: bool, extra=(), build_dir: str = BU
     return obj, (res.stdout + res.stderr) if verbose else None
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
-          defines=(), out: str | None = None) -> str:
-    """Compile every .cu under csrc/ for sm_100a and link lib/libmoda.so
-    (or `out`, with extra -D `defines`, into a separate object directory)."""
-    lib_path = out or LIB
-    build_dir = BUILD if not defines else os.path.join(BUILD, "v_" + "_".join(d.replace("=", "") for d in defines))
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
+    """Compile every .cu under csrc/ for sm_100a and link lib/libmoda.so."""
+    lib_path = LIB
+    build_dir = BUILD
     os.makedirs(build_dir, exist_ok=True)
     os.makedirs(os.path.dirname(lib_path), exist_ok=True)
     extra = ["-Xptxas", "-v"] if ptxas_info else []
-    extra += [f"-D{d}" for d in defines]
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         results = list(ex.map(lambda s: _compile(s, force or ptxas_info, verbose or ptxas_info, extra,

@@ -51,31 +51,6 @@ constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Optional hand-off timeline of CTA 0 (clock64 per event and iteration), only
-// in builds with -DMODA_TRACE; read back with moda_trace_copy_bwd().
-#ifdef MODA_TRACE
-constexpr int kTraceSlots = 16, kTraceIters = 96;
-__device__ long long g_trace_bwd[kTraceSlots * kTraceIters];
-__device__ long long g_trace_dq[kTraceSlots * kTraceIters];
-#define MODA_TR(slot, it)                                                   \
-    do {                                                                    \
-        if (blockIdx.x == 0 && (it) >= 0 && (it) < kTraceIters)             \
-            g_trace_bwd[(slot) * kTraceIters + (it)] = clock64();           \
-    } while (0)
-#define MODA_TRQ(slot, it)                                                  \
-    do {                                                                    \
-        if (blockIdx.x == 0 && (it) >= 0 && (it) < kTraceIters)             \
-            g_trace_dq[(slot) * kTraceIters + (it)] = clock64();            \
-    } while (0)
-#else
-#define MODA_TR(slot, it) \
-    do {                  \
-    } while (0)
-#define MODA_TRQ(slot, it) \
-    do {                   \
-    } while (0)
-#endif
-
 // ------------------------------------------------------------ 1. rowdot ----
 template <int D>
 __global__ void __launch_bounds__(256) rowdot_kernel(long long nrows,
@@ -129,10 +104,7 @@ struct DkdvArgs {
 };
 
 constexpr int kKvBQ = 64;               // query rows per iteration
-#ifndef MODA_DKDV_STAGES
-#define MODA_DKDV_STAGES 3
-#endif
-constexpr int kKvStages = MODA_DKDV_STAGES;   // Q/dO ring depth
+constexpr int kKvStages = 3;            // Q/dO ring depth
 constexpr uint32_t kKvSlab = 64 * 128;
 
 template <int D>
@@ -228,7 +200,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + st], ((it / kKvStages) - 1) & 1,
                                                    a.status, abort_flag)))
                 break;
-            if (lane == 0) MODA_TR(9, it);
             const int g = it / nqb;
             const int qb = qb0 + (it - g * nqb);
             const int qh = b * a.Hq + hk * a.G + g;
@@ -286,7 +257,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 const int st = j % kKvStages;
                 const int buf = j & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_QFull + st], (j / kKvStages) & 1, a.status, abort_flag))) return false;
-                MODA_TR(10, j);
                 tc_fence_after();
                 const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
                 const uint64_t dd = desc_kmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile));
@@ -311,13 +281,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             };
             bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag)) && (n_it == 0 || issue_s(0));
             for (int it = 0; ok && it < n_it; ++it) {
-                MODA_TR(0, it);
                 if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
-                MODA_TR(1, it);
                 const int st = it % kKvStages;
                 const int buf = it & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
-                MODA_TR(2, it);
                 tc_fence_after();
                 const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
                 const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
@@ -328,7 +295,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     umma_ts_elect(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g, acc);
                 }
                 umma_commit_elect(&bars[kA_QEmpty + st]);
-                MODA_TR(3, it);
             }
             umma_commit_elect(&bars[kA_Final]);
         }
@@ -342,7 +308,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         const int kr = quarter * 32 + sub * 16 + (lane & 15);   // key row within the tile
         const int k = kt * BN + kr;
         const int c0 = half * 32;                          // first query column of this thread
-        const int mt = threadIdx.x - 64;                   // 0..255 among the math threads
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
         const float sl2 = a.scale_log2;
         bool ok = true;
@@ -350,10 +315,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             const int g = it / nqb;
             const int qb = qb0 + (it - g * nqb);
             const int buf = it & 1;
-            if (mt == 0) MODA_TR(4, it);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status,
                                                    abort_flag))) { ok = false; break; }
-            if (mt == 0) MODA_TR(5, it);
             tc_fence_after();
             const int tq0 = qb * kKvBQ;
             const bool diag = a.causal && tq0 < kt * BN + BN;   // some key after some query
@@ -363,7 +326,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             tmem_wait_ld();
             reg_fence<32>(s);
             reg_fence<32>(dp);
-            if (mt == 0) MODA_TR(6, it);
             if (!diag) {                   // every column visible (CTA-uniform branch)
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -386,13 +348,11 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     dk[e / 2] = pack_bf16(p0 * __uint_as_float(dp[e]), p1 * __uint_as_float(dp[e + 1]));
                 }
             }
-            if (mt == 0) MODA_TR(7, it);
             // P^T and dS^T (bf16 pairs) over the columns this warp has read
             __syncwarp();
             tmem_st16x2_16<16>(lane_base + buf * 64, pk);
             tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
             tmem_wait_st();
-            if (mt == 0) MODA_TR(8, it);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kA_PReady + buf]);
@@ -453,10 +413,7 @@ struct DqArgs {
 };
 
 constexpr int kDqBN = 64;            // rows per key / depth block
-#ifndef MODA_DQ_STAGES
-#define MODA_DQ_STAGES 3
-#endif
-constexpr int kDqStages = MODA_DQ_STAGES;   // K/V ring depth
+constexpr int kDqStages = 3;         // K/V ring depth
 constexpr uint32_t kDqSlab = 64 * 128;   // 64 rows x 64 bf16
 
 template <int D>
@@ -601,7 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 const int st = j % kDqStages;
                 const int buf = j & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag))) return false;
-                MODA_TRQ(8, j);
                 tc_fence_after();
                 const uint32_t id = j < n_seq ? id_seq : id_dep;
                 const uint64_t kd = desc_kmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile));
@@ -629,9 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVEmpty + (j - 2) % kDqStages],
                                                                      ((j - 2) / kDqStages) & 1, a.status,
                                                                      abort_flag))) { ok = false; break; }
-                    MODA_TRQ(0, j);
                     if (!issue_s(j)) { ok = false; break; }
-                    MODA_TRQ(1, j);
                 }
             } else {
                 bool ok = true;
@@ -641,7 +595,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     const bool seq = i < n_seq;
                     const int n = seq ? kDqBN : a.dep_rows;
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
-                    MODA_TRQ(2, i);
                     tc_fence_after();
                     const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
                     // dS of keys [16kk, 16kk + 16) sits at column (kk / 2) * 32 +
@@ -668,7 +621,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                         umma_commit_elect(&bars[kB_DDFull]);
                     }
                     umma_commit_elect(&bars[kB_KVEmpty + st]);
-                    MODA_TRQ(3, i);
                 }
                 umma_commit_elect(&bars[kB_Final]);
             }
@@ -682,7 +634,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const int half = warp >= 7 ? 1 : 0;
         const int c0 = 32 * half;
         const int r = quarter * 32 + lane;
-        const int mt = threadIdx.x - 64;                  // 0 for warp 2, lane 0
         const bool row_real = r < R;
         const int g = row_real ? r / a.Tq : 0;
         const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
@@ -727,9 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         for (int i = 0; i < nb; ++i) {
             const int buf = i & 1;
             const bool seq = i < n_seq;
-            if (mt == 0) MODA_TRQ(4, i);
             if (!mbar_wait(&bars[kB_SFull + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
-            if (mt == 0) MODA_TRQ(5, i);
             tc_fence_after();
             uint32_t s[32], dp[32], dsk[16], pk[16];
             tmem_ld32(lane_base + kColS + buf * 64 + c0, s);
@@ -778,7 +727,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     pk[e / 2] = pack_bf16(p2[0], p2[1]);
                 }
             }
-            if (mt == 0) MODA_TRQ(6, i);
             // packed dS of keys [c0, c0 + 32) into columns [c0, c0 + 16): inside
             // this half's own score columns, which only it reads
             tmem_st16(lane_base + kColS + buf * 64 + c0, dsk);
@@ -804,7 +752,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 ++jd;
             }
             tmem_wait_st();
-            if (mt == 0) MODA_TRQ(7, i);
             tc_fence_before();
             mbar_arrive(&bars[kB_PReady + buf]);
         }
@@ -878,8 +825,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     if ((e = make_tma_3d_bf16(&A.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
     {
         const uint32_t smem = DkdvLayout<D>::kDynSmem;
-        if ((e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem)) != cudaSuccess)
+        if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dkdv_kernel<D>), (int)smem)) != cudaSuccess)
             return e;
         const long long grid = (long long)p.B * p.Hk * A.n_kt;
         dkdv_kernel<D><<<(unsigned)grid, kKvThreads, smem, stream>>>(A);
@@ -916,8 +862,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     }
     {
         const uint32_t smem = DqLayout<D>::kDynSmem;
-        if ((e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem)) != cudaSuccess)
+        if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dq_kernel<D>), (int)smem)) != cudaSuccess)
             return e;
         const long long grid = (long long)p.B * p.Hk * B.n_qt;
         dq_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(B);
@@ -929,16 +874,6 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
 
 }  // namespace
 
-#ifdef MODA_TRACE
-extern "C" int moda_trace_copy_bwd(long long* host, int n) {
-    const int cnt = n < kTraceSlots * kTraceIters ? n : kTraceSlots * kTraceIters;
-    return cudaMemcpyFromSymbol(host, g_trace_bwd, cnt * sizeof(long long)) == cudaSuccess ? cnt : -1;
-}
-extern "C" int moda_trace_copy_dq(long long* host, int n) {
-    const int cnt = n < kTraceSlots * kTraceIters ? n : kTraceSlots * kTraceIters;
-    return cudaMemcpyFromSymbol(host, g_trace_dq, cnt * sizeof(long long)) == cudaSuccess ? cnt : -1;
-}
-#endif
 
 cudaError_t launch_bwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, const void* O, const float* LSE,

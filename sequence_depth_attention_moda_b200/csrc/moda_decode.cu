@@ -627,8 +627,7 @@ cudaError_t launch_mma(const Problem& p, const void* q, const void* K, const voi
     a.n_cta = m.n_cta;
     a.maxc = m.maxc;
     a.scale_log2 = p.scale_log2;
-    if ((e = cudaFuncSetAttribute(decode_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  Lay::kSmem)) != cudaSuccess)
+    if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(decode_mma_kernel<D>), Lay::kSmem)) != cudaSuccess)
         return e;
     decode_mma_kernel<D><<<m.n_cta, kMmaThreads, Lay::kSmem, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

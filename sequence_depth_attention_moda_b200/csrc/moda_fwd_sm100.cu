@@ -38,9 +38,9 @@
 //               than 2^8 (exact: the final o / acc cancels it).  Two warps
 //               per SM sub-partition keep its MUFU (exp2) unit fed.
 // TMEM columns: S0 [0,128), S1 [128,256), S2 [256,384), O [384, 384+d).
-// Softmax: row max as four partial maxima of three-input max; exp2 on the MUFU unit (a build
-// knob moves a share of column pairs to ex2_fma on the FMA pipe; measured
-// slower here, so off).
+// Softmax: row max as four partial maxima of three-input max; exp2 on the
+// MUFU unit (moving a share of the exponentials to a polynomial on the FMA
+// pipe measured slower: the softmax warps are issue-bound, not MUFU-bound).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -55,14 +55,8 @@ using namespace ptx;
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = 128;          // sequence keys per block
-#ifndef MODA_FWD_KSTAGES
-#define MODA_FWD_KSTAGES 3
-#endif
-#ifndef MODA_FWD_VSTAGES
-#define MODA_FWD_VSTAGES 3
-#endif
-constexpr int kKStages = MODA_FWD_KSTAGES;   // K ring: a stage frees when S_i is done
-constexpr int kVStages = MODA_FWD_VSTAGES;   // V ring: a stage frees when PV_i is done
+constexpr int kKStages = 3;      // K ring: a stage frees when S_i is done
+constexpr int kVStages = 3;      // V ring: a stage frees when PV_i is done
 constexpr int kSoftmaxWarps = 8;             // warps 2..9
 constexpr int kVWarp = 2 + kSoftmaxWarps;    // V producer
 constexpr int kThreads = 32 * (kVWarp + 1);
@@ -71,28 +65,6 @@ constexpr uint32_t kSlabBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBufs = 3;            // S / P buffers in TMEM
 constexpr uint32_t kColO = 384;      // O accumulator after the three S buffers
-#ifndef MODA_FWD_OFFSET
-#define MODA_FWD_OFFSET 0            // cycles the rows-16..31 softmax warps start late
-#endif
-#ifndef MODA_FWD_SWEXP
-#define MODA_FWD_SWEXP 0             // of every 4 column pairs, this many use ex2_fma
-#endif
-
-// Optional hand-off timeline of CTA 0 (clock64 per event and block), only in
-// builds with -DMODA_TRACE; read back with moda_trace_copy_fwd().
-#ifdef MODA_TRACE
-constexpr int kTraceSlots = 16, kTraceIters = 96;
-__device__ long long g_trace_fwd[kTraceSlots * kTraceIters];
-#define MODA_TRF(slot, it)                                                  \
-    do {                                                                    \
-        if (blockIdx.x == 0 && (it) >= 0 && (it) < kTraceIters)             \
-            g_trace_fwd[(slot) * kTraceIters + (it)] = clock64();           \
-    } while (0)
-#else
-#define MODA_TRF(slot, it) \
-    do {                   \
-    } while (0)
-#endif
 
 struct FwdArgs {
     TmaMap tq, tk, tv, tkd, tvd;
@@ -271,7 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         // The whole warp runs this loop converged, so descriptors and waits
         // are warp-uniform; elect.sync picks the lane that issues each MMA
         // and commit.
-        const bool tl = lane == 0;                    // trace lane
         const uint32_t id_seq = idesc_bf16(128, BN, false, false);
         const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
         const uint32_t id_pv = idesc_bf16(128, D, false, true);
@@ -284,10 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         auto issue_s = [&](int j, int i, const FwdTile& T) -> bool {
             const int st = j % kKStages;
             const int sb = j % kSBufs;
-            if (tl) MODA_TRF(0, j);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kKFull + st], (j / kKStages) & 1, a.status,
                                                    abort_flag))) return false;
-            if (tl) MODA_TRF(1, j);
             tc_fence_after();
             const uint64_t kd0 = desc_kmajor_sw128(smem_u32(sK + st * Lay::kTile));
             const uint32_t id = i < T.n_seq ? id_seq : id_dep;
@@ -297,7 +266,6 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 umma_ss_elect(tmem + sb * 128, qd0 + off, kd0 + off, id, kk > 0 ? 1u : 0u);
             }
             umma_commit_elect(&bars[kSFull + sb]);
-            if (tl) MODA_TRF(2, j);
             return true;
         };
         // O += P(j) V_j with P read from TMEM buffer j % 3; the tile's first
@@ -307,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             const int sb = j % kSBufs;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kPReady + sb], (j / kSBufs) & 1, a.status,
                                                    abort_flag))) return false;
-            if (tl) MODA_TRF(4, j);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status,
                                                    abort_flag))) return false;
             tc_fence_after();
@@ -324,7 +291,6 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                                   (i > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit_elect(&bars[kVEmpty + st]);
-            if (tl) MODA_TRF(3, j);
             return true;
         };
         // Two score tiles run ahead of the softmax.  S(i+2) goes in before
@@ -367,8 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         const int g = row_real ? r / a.Tq : 0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
         const int c0 = half * 64;                     // first S column this thread holds
-        const bool tr = r == 0 && half == 0;          // trace threads
-        const bool tr2 = r == 32 && half == 0;        // quarter 1: the MMA warp's sub-partition
         const float sl2 = a.scale_log2;
         bool ok = true;
         int j0 = 0, kt = 0;
@@ -382,13 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             for (int i = 0; i < nb; ++i) {
                 const int j = j0 + i;                     // running block count: ring phases
                 const int sb = j % kSBufs;
-                if (tr) MODA_TRF(5, j);
                 // every wait result is made warp-uniform: the shuffles and the
                 // .sync.aligned TMEM accesses below need the whole warp
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + sb], (j / kSBufs) & 1, a.status,
                                                        abort_flag))) { ok = false; break; }
-                if (tr) MODA_TRF(6, j);
-                if (tr2) MODA_TRF(12, j);
                 tc_fence_after();
                 const uint32_t s_addr = lane_base + sb * 128;
                 if (i >= n_seq) {
@@ -417,7 +378,6 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 tmem_ld16x2_32<64>(s_addr + 32, sr + 32);  // columns c0+32 .. c0+63
                 tmem_wait_ld();
                 reg_fence<64>(sr);
-                if (tr) MODA_TRF(7, j);
                 // masks: invisible scores become -inf (p = 0)
                 if (i < n_seq) {
                     const int kb = i * BN + c0;
@@ -457,14 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     for (int c = 0; c < 32; ++c) {
                         const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -m);
                         const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m);
-                        float p0, p1;
-                        if ((c & 3) < 4 - MODA_FWD_SWEXP) {     // MUFU
-                            p0 = ex2(x0);
-                            p1 = ex2(x1);
-                        } else {                                 // FMA pipe
-                            p0 = ex2_fma(x0);
-                            p1 = ex2_fma(x1);
-                        }
+                        const float p0 = ex2(x0);
+                        const float p1 = ex2(x1);
                         rs4[c & 3] += p0 + p1;
                         pk[c] = pack_bf16(p0, p1);
                     }
@@ -477,10 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                 // overflow too) does the warp take the block max, rescale O and
                 // l to the new reference and recompute P.  The first block sets m.
                 if (i == 0) m = block_max();
-                if (tr) MODA_TRF(8, j);
-                if (tr2) MODA_TRF(13, j);
                 float rs = exp_block();
-                if (tr) MODA_TRF(9, j);
                 if (i > 0 && __any_sync(0xffffffffu, !(rs <= kLazyLimit))) {
                     const float m_new = fmaxf(m, block_max());
                     // O must hold P_{i-1} V_{i-1} before it is rescaled: wait for
@@ -510,18 +461,14 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     rs = exp_block();
                 }
                 l += rs;
-                if (tr) MODA_TRF(10, j);
-                if (tr2) MODA_TRF(14, j);
                 // P columns c0/2 .. c0/2+31 (bf16 pairs) over the S columns this
                 // warp has already read (its own loads completed above)
                 __syncwarp();
                 tmem_st16x2_32<32>(s_addr, pk);
                 tmem_wait_st();
-                if (tr) MODA_TRF(11, j);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[kPReady + sb]);
-                if (tr2) MODA_TRF(15, j);
             }
             // ---------------------------------------------------- epilogue ------
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFinal], kt & 1, a.status, abort_flag));
@@ -594,11 +541,9 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
         a.tvd = a.tv;
     }
     const uint32_t smem = Layout<D>::kDynSmem;
-    e = cudaFuncSetAttribute(moda_fwd_sm100_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    e = set_max_dynamic_smem(reinterpret_cast<const void*>(moda_fwd_sm100_kernel<D, true>), (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(moda_fwd_sm100_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    e = set_max_dynamic_smem(reinterpret_cast<const void*>(moda_fwd_sm100_kernel<D, false>), (int)smem);
     if (e != cudaSuccess) return e;
     // Short tiles (on average fewer than 64 key blocks): one persistent CTA per
     // SM walks its share, so tile start-up and epilogue overlap the previous
@@ -619,12 +564,6 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
 
 }  // namespace
 
-#ifdef MODA_TRACE
-extern "C" int moda_trace_copy_fwd(long long* host, int n) {
-    const int cnt = n < kTraceSlots * kTraceIters ? n : kTraceSlots * kTraceIters;
-    return cudaMemcpyFromSymbol(host, g_trace_fwd, cnt * sizeof(long long)) == cudaSuccess ? cnt : -1;
-}
-#endif
 
 cudaError_t launch_fwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, void* O, float* LSE,

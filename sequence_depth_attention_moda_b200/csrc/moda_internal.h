@@ -88,4 +88,8 @@ struct TmaMap { alignas(64) unsigned char bytes[128]; };
 cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t rows,
                              uint64_t outer, uint32_t box_rows, uint32_t box_outer);
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) for `func` on the current
+// device, done once per (device, function): later calls only look it up.
+cudaError_t set_max_dynamic_smem(const void* func, int bytes);
+
 }  // namespace moda

@@ -346,27 +346,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x computed on the FMA pipe (offloads the MUFU unit, which is the other
-// limit of a softmax tile).  Range reduction x = n + f with n = rint(x) taken
-// from the low mantissa bits of x + 1.5*2^23 and f in [-0.5, 0.5]; 2^f by a
-// degree-4 polynomial fitted for this library (Lawson-weighted least squares
-// for relative error on [-0.5, 0.5]; max relative error 2.7e-6 in fp32
-// Horner form); 2^n by adding n to the exponent field.  x < -125 returns 0.
-constexpr float kExp2C0 = 0.9999992847442627f, kExp2C1 = 0.6931218504905701f,
-                kExp2C2 = 0.240247443318367f, kExp2C3 = 0.055917806923389435f,
-                kExp2C4 = 0.009570068679749966f;
-__device__ __forceinline__ float ex2_fma(float x) {
-    const float xc = fmaxf(x, -125.0f);
-    const float r = xc + 12582912.0f;
-    const float f = xc - (r - 12582912.0f);
-    float q = fmaf(kExp2C4, f, kExp2C3);
-    q = fmaf(q, f, kExp2C2);
-    q = fmaf(q, f, kExp2C1);
-    q = fmaf(q, f, kExp2C0);
-    const float y = __int_as_float(__float_as_int(q) + (__float_as_int(r) << 23));
-    return x < -125.0f ? 0.0f : y;
-}
-
 // max(a, b, c) in one instruction (three-input form of max.f32).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;

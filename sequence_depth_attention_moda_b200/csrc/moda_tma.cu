@@ -1,11 +1,15 @@
-// moda_tma.cu -- host-side construction of TMA tensor maps.  The driver entry
-// point cuTensorMapEncodeTiled is fetched through the runtime, so the library
-// does not link libcuda directly.
+// moda_tma.cu -- host-side launch set-up shared by the kernels: TMA tensor
+// maps (memoised) and the per-device dynamic shared-memory attribute.  The
+// driver entry point cuTensorMapEncodeTiled is fetched through the runtime,
+// so the library does not link libcuda directly.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstring>
 #include <mutex>
+#include <tuple>
+#include <unordered_map>
+#include <vector>
 
 #include "moda_internal.h"
 
@@ -35,8 +39,33 @@ EncodeTiledFn encode_fn() {
 
 static_assert(sizeof(TmaMap) == sizeof(CUtensorMap), "TmaMap must hold a CUtensorMap");
 
-cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t rows,
-                             uint64_t outer, uint32_t box_rows, uint32_t box_outer) {
+namespace {
+
+// Encoding a tensor map is a pure function of its arguments, so results are
+// memoised: repeated calls on the same buffers (every training step, every
+// decoding token) skip the driver call.  The table is cleared when it fills.
+struct MapKey {
+    uint64_t base, d, rows, outer;
+    uint32_t box_rows, box_outer;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && d == o.d && rows == o.rows && outer == o.outer &&
+               box_rows == o.box_rows && box_outer == o.box_outer;
+    }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey& k) const {
+        uint64_t h = k.base * 0x9E3779B97F4A7C15ull;
+        for (uint64_t v : {k.d, k.rows, k.outer, uint64_t(k.box_rows) << 32 | k.box_outer})
+            h = (h ^ v) * 0x100000001B3ull;
+        return static_cast<size_t>(h ^ (h >> 29));
+    }
+};
+constexpr size_t kMapCacheEntries = 1024;
+std::mutex g_map_mutex;
+std::unordered_map<MapKey, TmaMap, MapKeyHash> g_map_cache;
+
+cudaError_t encode_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t rows, uint64_t outer,
+                           uint32_t box_rows, uint32_t box_outer) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     CUtensorMap map;
@@ -52,6 +81,42 @@ cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     std::memcpy(out->bytes, &map, sizeof(map));
     return cudaSuccess;
+}
+
+std::mutex g_attr_mutex;
+std::vector<std::tuple<int, const void*, int>> g_attr_done;
+
+}  // namespace
+
+cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t rows,
+                             uint64_t outer, uint32_t box_rows, uint32_t box_outer) {
+    const MapKey key{reinterpret_cast<uint64_t>(base), d, rows, outer, box_rows, box_outer};
+    {
+        std::lock_guard<std::mutex> lk(g_map_mutex);
+        auto it = g_map_cache.find(key);
+        if (it != g_map_cache.end()) {
+            *out = it->second;
+            return cudaSuccess;
+        }
+    }
+    cudaError_t e = encode_3d_bf16(out, base, d, rows, outer, box_rows, box_outer);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_map_mutex);
+    if (g_map_cache.size() >= kMapCacheEntries) g_map_cache.clear();
+    g_map_cache.emplace(key, *out);
+    return cudaSuccess;
+}
+
+cudaError_t set_max_dynamic_smem(const void* func, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_attr_mutex);
+    for (const auto& t : g_attr_done)
+        if (std::get<0>(t) == dev && std::get<1>(t) == func && std::get<2>(t) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) g_attr_done.emplace_back(dev, func, bytes);
+    return e;
 }
 
 }  // namespace moda
