@@ -58,7 +58,43 @@ def parse_args():
                          "G x L x C sweep, L = 0 twins); one JSON line, one GPU")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decoding path (one JSON line; small device footprint)")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="start the ranks as for a run and report them (gloo, no GPU work)")
     return ap.parse_args()
+
+
+def launch_ranks(args) -> None:
+    """`--gpus N` (N > 1) outside torchrun: run this script again under
+    torch.distributed.run with N ranks on this node, one per GPU, and exit
+    with its status.  Under torchrun (WORLD_SIZE set) this does nothing."""
+    if args.gpus <= 1 or "WORLD_SIZE" in os.environ:
+        return
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__),
+           *sys.argv[1:]]
+    sys.exit(subprocess.call(cmd))
+
+
+def run_launch_check(args):
+    """Every rank joins a gloo group and reports its rank; rank 0 prints one
+    JSON line with the ranks seen (the launch path without any GPU work)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    seen = [rank]
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        out = [None] * world
+        torch.distributed.all_gather_object(out, rank)
+        seen = sorted(out)
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "n_gpus": world, "ranks": seen,
+                          "parallelism": f"dp{world}" if world > 1 else "single"}), flush=True)
 
 
 # ------------------------------------------------------------------ helpers --
@@ -388,6 +424,115 @@ def cpu_baseline_sample(w: I.Workload, x):
                       f"{dt:.1f} s"}
 
 
+def _rows_rate(lib, w: I.Workload, x, rows, cores: int):
+    """Oracle time of the sampled query rows (b, h, t) of workload w, run
+    on `cores` host threads (the row entry point releases the GIL).  Returns
+    (seconds, FLOPs of those rows)."""
+    import concurrent.futures as cf
+    import oracle
+    G, L = w.G, w.L
+    f64 = {}
+
+    def kv(b, hk):
+        if (b, hk) not in f64:
+            f64[(b, hk)] = (x["K"][b, hk].double().numpy(), x["V"][b, hk].double().numpy())
+        return f64[(b, hk)]
+
+    jobs = []
+    for (b, h, t) in rows:
+        K, V = kv(b, h // G)
+        Kd = x["Kd_layer"][:, b, h // G, t].double().numpy() if L else np.zeros((0, w.d))
+        Vd = x["Vd_layer"][:, b, h // G, t].double().numpy() if L else np.zeros((0, w.d))
+        jobs.append((x["Q"][b, h, t].double().numpy(), K[:t + 1], V[:t + 1], Kd, Vd))
+    flops = sum(4.0 * w.d * (t + 1 + L) for (_, _, t) in rows)
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        list(ex.map(lambda a: oracle.row(*a, lib=lib), jobs))
+    return time.perf_counter() - t0, flops
+
+
+def cpu_baselines_per_config(x_c2):
+    """The oracle, as it stands, on every workload of the benchmark, each on
+    a bounded sample (a few seconds of host time in all): the tiny fp32
+    workload in full; the 1.5B layer and the training shape on one (b, hk)
+    slice, forward + backward; the T = 64K forward and the G x L sweep on
+    sampled query rows.  Rates are FLOPs of the sample / its time; for the
+    sampled workloads `est_s` is the whole workload's time at that rate
+    (extrapolated)."""
+    import oracle
+    from moda_cases import slice_workload, token_major, f64
+    lib = oracle.load_library()
+    cores = oracle.threads(lib)
+    out = {}
+
+    def slice_rate(w, x, backward):
+        ws, xs = slice_workload(w, x, 0, 0)
+        Kd, Vd = token_major(xs, ws)
+        a = [f64(xs["Q"]), f64(xs["K"]), f64(xs["V"]), f64(Kd), f64(Vd)]
+        t0 = time.perf_counter()
+        oracle.fwd(*a, lib=lib)
+        if backward:
+            oracle.bwd(*a, f64(xs["dO"]), lib=lib)
+        dt = time.perf_counter() - t0
+        fl = ws.fwd_flops() * ((1 + BWD_FACTOR) if backward else 1)
+        return dt, fl, ws
+
+    def entry(w, dt, fl, total, sample, extrapolated, threads):
+        rate = fl / dt
+        return {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                "sample": sample, "sample_s": round(dt, 6), "extrapolated": extrapolated,
+                "est_s": round(total / rate, 4)}
+
+    w = I.TINY_FP32.with_(backward=True)
+    x = I.make_inputs(w, device="cpu")
+    Kd, Vd = token_major(x, w)
+    a = [f64(x["Q"]), f64(x["K"]), f64(x["V"]), f64(Kd), f64(Vd)]
+    reps = 50
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.fwd(*a, lib=lib)
+    dt = (time.perf_counter() - t0) / reps
+    out[w.name] = entry(w, dt, w.fwd_flops(), w.fwd_flops(),
+                        f"the whole forward, fp64 (mean of {reps} runs)", False, cores)
+
+    w = WORKLOAD
+    dt, fl, ws = slice_rate(w, x_c2, True)
+    out[w.name] = entry(w, dt, fl, w.fwd_flops() * (1 + BWD_FACTOR),
+                        f"one (b,hk) slice (B=1, Hq={ws.Hq}, Hk=1), forward + backward", True, cores)
+
+    w = I.TRAIN_FWD_BWD
+    x = I.make_inputs(w.with_(B=1, Hq=w.G, Hk=1), device="cpu")
+    dt, fl, ws = slice_rate(w.with_(B=1, Hq=w.G, Hk=1), x, True)
+    out[w.name] = entry(w, dt, fl, w.fwd_flops() * (1 + BWD_FACTOR),
+                        f"one (b,hk) slice (B=1, Hq={w.G}, Hk=1), forward + backward", True, cores)
+    del x
+
+    w = LONG
+    x = I.make_inputs(w.with_(Hq=w.G, Hk=1), device="cpu", grad_out=False)
+    rng = np.random.default_rng(11)
+    rows = [(0, int(rng.integers(w.G)), int(t)) for t in np.linspace(0, w.T - 1, 128).astype(int)]
+    dt, fl = _rows_rate(lib, w.with_(Hq=w.G, Hk=1), x, rows, cores)
+    out[w.name] = entry(w, dt, fl, w.fwd_flops(), "128 query rows, t evenly spread over 0..T-1, forward (row entry point)",
+                        True, cores)
+    del x
+
+    tot_fl = tot_dt = tot_all = 0.0
+    for G in (1, 2, 4, 8):
+        for L in (1, 8, 32, 64):
+            w = I.Workload(f"sweep_G{G}_L{L}", B=1, Hq=G, Hk=1, d=128, T=8192, L=L, C=64, seed=7)
+            x = I.make_inputs(w, device="cpu", grad_out=False)
+            rows = [(0, int(rng.integers(G)), int(t)) for t in np.linspace(0, w.T - 1, 32).astype(int)]
+            dt, fl = _rows_rate(lib, w, x, rows, cores)
+            tot_fl += fl
+            tot_dt += dt
+            tot_all += 3 * w.with_(Hq=4 * G, Hk=4).fwd_flops()     # three C values, same work
+            del x
+    out["depth_group_sweep"] = entry(None, tot_dt, tot_fl, tot_all,
+                                     "32 query rows of each (G, L) point (C does not change the work), "
+                                     "forward (row entry point)", True, cores)
+    return out
+
+
 def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -470,6 +615,14 @@ def run_ours(args):
         torch.cuda.empty_cache()
         extra["decode_T32k"] = decode_measure(I.DECODE_T32K, rank, world, peaks, max(10, args.steps // 2))
         torch.cuda.empty_cache()
+        # the training-shaped step and the G x L x C sweep, one kernel call at a
+        # time against max(FLOPs / peak, bytes / bandwidth) (fewer runs each)
+        flush = torch.empty(256 << 20, device="cuda", dtype=torch.uint8)
+        extra["train_T4k_L48"] = config_measure(I.TRAIN_FWD_BWD, peaks, flush, runs=5)
+        torch.cuda.empty_cache()
+        extra["depth_group_sweep"] = sweep_summary(peaks, flush, runs=5)
+        del flush
+        torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_e2e:
@@ -478,9 +631,10 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e, 3),
                "pipeline": "upload / compute / read-back on three streams, two buffer sets"}
 
-    cpu = None
+    cpu = cpu_all = None
     if world == 1 and rank == 0 and not args.no_cpu:
         cpu = cpu_baseline_sample(w, x)
+        cpu_all = cpu_baselines_per_config({k: v.cpu() for k, v in x.items()})
 
     if rank == 0:
         line = {
@@ -497,7 +651,8 @@ def run_ours(args):
             "roofline": roofline, "roofline_other_kernels": roofline_others,
             "roofline_repack": roofline_repack,
             "gpu_launches": r.launches_per_step() * args.steps,
-            "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu, **extra,
+            "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu,
+            "cpu_baseline_per_config": cpu_all, **extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -627,6 +782,25 @@ def config_measure(w: I.Workload, peaks, flush: torch.Tensor, runs: int = 20, tw
     return out
 
 
+def sweep_summary(peaks, flush, runs: int = 5):
+    """The G x L x C sweep's forward against its attainable time: worst and
+    median fraction over the 48 points, and the G = 1 and G = 8 points at
+    L = 64, C = 64."""
+    rows = []
+    seen_g = set()
+    for w in I.depth_group_sweep():
+        rows.append(config_measure(w, peaks, flush, runs=runs, twin=w.G not in seen_g))
+        seen_g.add(w.G)
+    fr = sorted(r["fwd"]["frac_of_attainable"] for r in rows)
+    pick = {r["workload"]: r for r in rows}
+    worst = min(rows, key=lambda r: r["fwd"]["frac_of_attainable"])
+    return {"points": len(rows), "runs": runs,
+            "fwd_frac_of_attainable_worst": fr[0], "worst_point": worst["workload"],
+            "fwd_frac_of_attainable_median": round(float(np.median(fr)), 4),
+            "G1_L64_C64": pick["sweep_G1_L64_C64"]["fwd"], "G8_L64_C64": pick["sweep_G8_L64_C64"]["fwd"],
+            "L0_fwd_ms": {f"G{r['Hq'] // r['Hk']}": r["L0_fwd_ms"] for r in rows if "L0_fwd_ms" in r}}
+
+
 def run_configs(args):
     """Every workload's kernels against their rooflines (one GPU)."""
     torch.cuda.set_device(0)
@@ -662,7 +836,10 @@ def run_decode_only(args):
 
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    launch_ranks(args)
+    if args.launch_check:
+        run_launch_check(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.decode_only:
         run_decode_only(args)

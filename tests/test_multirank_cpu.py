@@ -51,3 +51,22 @@ def test_two_gloo_ranks_time_max_and_distinct_batches():
     from sequence_depth_attention_moda_b200 import inputs as I
     assert abs(v0 - 2 * I.TINY_FP32.fwd_flops() / 5e-3 / 1e12) < 1e-12
     assert q0 != q1                            # different batches per rank
+
+
+@pytest.mark.timeout(300)
+def test_bench_gpus_flag_starts_one_rank_per_gpu():
+    """`python bench.py --gpus 2` outside torchrun starts two ranks itself
+    (torch.distributed.run on this node); both join one group and rank 0
+    reports them (gloo, no GPU work)."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--launch-check"],
+                         capture_output=True, text=True, timeout=240, env=env, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    rep = json.loads(lines[0])
+    assert rep["n_gpus"] == 2 and rep["ranks"] == [0, 1] and rep["parallelism"] == "dp2"
