@@ -178,6 +178,35 @@ def traffic_from_profile(kernel: str, kernel_src: str, table: str = "dram_traffi
     return int(m.group(1)) if cur == m.group(2) else None
 
 
+def kernel_work(w: I.Workload, stored_ds: bool):
+    """(algorithmic FLOPs, bytes each kernel must move) per launch of the
+    forward and of the backward's dK/dV and dQ kernels.  FLOPs: the forward's
+    4*B*Hq*d*(T(T+1)/2 + T*L); the backward's five matmuls over [seq | depth]
+    split as dK/dV = S^T, dP^T, dV, dK over the sequence keys and dQ = dQ over
+    all keys plus S, dP, dK_d, dV_d over the depth rows (recomputation is not
+    counted).  Bytes: every input read once and every output written once;
+    with stored dS, the dK/dV kernel writes and the dQ kernel reads the 16 KB
+    dS tiles (128 query rows x 64 keys) the causal mask needs."""
+    e = 2
+    mm_seq = 2.0 * w.B * w.Hq * w.d * (w.T * (w.T + 1) / 2)
+    mm_dep = 2.0 * w.B * w.Hq * w.d * (w.T * w.L)
+    q = w.B * w.Hq * w.T * w.d * e
+    kv = w.B * w.Hk * w.T * w.d * e
+    dep = w.B * w.Hk * w.T * w.L * w.d * e
+    rows = w.B * w.Hq * w.T * 4
+    ds = 0
+    if stored_ds:
+        Tq = 128 // w.G
+        n_qt, n_kb = -(-w.T // Tq), -(-w.T // 64)
+        per_head = sum(min(n_kb, (min(Tq * (qt + 1), w.T) - 1) // 64 + 1) if w.causal else n_kb
+                       for qt in range(n_qt))
+        ds = w.B * w.Hk * per_head * 16384
+    return {"fwd": (w.fwd_flops(), q + 2 * kv + 2 * dep + q + rows),
+            "dkdv": (4 * mm_seq, 2 * kv + 2 * q + 2 * rows + 2 * kv + ds),
+            "dq": ((mm_seq + mm_dep) + 4 * mm_dep,
+                   2 * q + 2 * rows + (ds + kv if stored_ds else 2 * kv) + 2 * dep + q + 2 * dep)}
+
+
 # --------------------------------------------------------------- our arm ----
 class Runner:
     """Device buffers and the four C-ABI calls of one step."""
@@ -195,8 +224,10 @@ class Runner:
         self.Vd = torch.empty_like(self.Kd) if w.L else None
         self.O = torch.empty_like(x["Q"])
         self.LSE = torch.empty(w.B, w.Hq, w.T, device=dev, dtype=torch.float32)
+        self.stored_ds = False
         if backward:
-            self.nws = moda.moda_workspace_size(self.sh, True)
+            self.nws = moda.moda_workspace_size(self.sh, 1)
+            self.stored_ds = self.nws > moda.moda_workspace_size(self.sh, 2)
             self.ws = torch.empty(max(self.nws, 16), device=dev, dtype=torch.uint8)
             self.dQ = torch.empty_like(x["Q"])
             self.dK = torch.empty_like(x["K"])
@@ -558,31 +589,35 @@ def run_ours(args):
     value = job_value(flops_step, ms, world)
     per_gpu = value / world
 
-    # Roofline of the dominant kernel (largest mean duration).  Algorithmic
-    # FLOPs per kernel: the backward's five matmuls over [seq | depth] keys
-    # (2.5x the forward) split as dkdv = S^T, dP^T, dV, dK over the sequence
-    # keys and dq = dQ over all keys plus S, dP, dK, dV over the depth keys;
-    # dq's recomputation of the sequence S and dP is not counted.
-    mm_seq = 2.0 * w.B * w.Hq * w.d * (w.T * (w.T + 1) / 2)
-    mm_dep = 2.0 * w.B * w.Hq * w.d * (w.T * w.L)
-    algo = {"fwd": w.fwd_flops(), "dkdv": 4 * mm_seq, "dq": (mm_seq + mm_dep) + 4 * mm_dep}
+    # Roofline of the dominant kernel (largest mean duration) and of the
+    # others: each against max(algorithmic FLOPs / tensor peak, bytes it must
+    # move / HBM bandwidth) (kernel_work).
+    work = kernel_work(w, stored_ds=r.stored_ds)
     names = {"fwd": "moda_fwd_sm100_kernel", "dkdv": "dkdv_kernel", "dq": "dq_kernel"}
     srcs = {"fwd": "moda_fwd_sm100.cu", "dkdv": "moda_bwd_sm100.cu", "dq": "moda_bwd_sm100.cu"}
-    dom = max(algo, key=lambda k: calls[k])
+    dom = max(names, key=lambda k: calls[k])
 
     def roof(k):
-        ach = algo[k] / (calls[k] * 1e-3) / 1e12
+        flops, nbytes = work[k]
+        t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
         src = os.path.join(ROOT, "sequence_depth_attention_moda_b200", "csrc", srcs[k])
-        return {"kernel": names[k], "bound": "tensor", "achieved": round(ach, 1),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(ach / peaks["bf16_tflops"], 4),
-                "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                "traffic": traffic_from_profile(names[k], src),
-                "mean_ms": round(calls[k], 4), "algorithmic_flops": algo[k]}
+        out = {"kernel": names[k], "mean_ms": round(calls[k], 4), "algorithmic_flops": flops,
+               "algorithmic_bytes": nbytes, "traffic": traffic_from_profile(names[k], src)}
+        if t_tensor >= t_hbm:
+            ach = flops / (calls[k] * 1e-3) / 1e12
+            out.update(bound="tensor", achieved=round(ach, 1), peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                       frac=round(ach / peaks["bf16_tflops"], 4),
+                       peak_source=f"{peaks['source']} bf16 dense (burst)")
+        else:
+            ach = nbytes / (calls[k] * 1e-3) / 1e9
+            out.update(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm_gbs"], unit="GB/s",
+                       frac=round(ach / peaks["hbm_gbs"], 4), peak_source=f"{peaks['source']} copy bandwidth")
+        return out
 
     roofline = roof(dom)
     roofline["per_kernel_ms"] = {k: round(v, 4) for k, v in calls.items()}
-    roofline_others = {k: roof(k) for k in algo if k != dom}
+    roofline_others = {k: roof(k) for k in names if k != dom}
     rep_bytes = 2 * 2 * w.B * w.Hk * w.T * w.L * w.d * 2
     rep_ach = rep_bytes / (calls["repack"] * 1e-3) / 1e9
     roofline_repack = {"kernel": "repack_vec16_kernel (x2)", "bound": "hbm", "achieved": round(rep_ach, 1),

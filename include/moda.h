@@ -108,9 +108,17 @@ typedef struct moda_shape {
 } moda_shape;
 
 /*
- * Bytes of workspace moda_fwd (for_bwd = 0) or moda_bwd (for_bwd = 1) needs
- * for this shape; 0 means ws may be NULL.  Returns (size_t)-1 for a shape
- * that the corresponding call would reject.
+ * Bytes of workspace for this shape:
+ *   for_bwd = 0   moda_fwd (0: ws may be NULL);
+ *   for_bwd = 1   moda_bwd at its fastest: the row statistics D plus, for
+ *                 bf16 with d = 128, G in {1, 2, 4, 8} and at most 16 GiB of
+ *                 them, the stored score gradients dS (16 KB per 128 query
+ *                 rows x 64 keys), which the dQ kernel then reads instead of
+ *                 recomputing the scores;
+ *   for_bwd = 2   the least moda_bwd accepts: D only (4 bytes per query row,
+ *                 rounded up to 256); the dQ kernel then recomputes S and dP.
+ * Returns (size_t)-1 for a shape the corresponding call would reject or an
+ * unknown for_bwd.
  */
 size_t moda_workspace_size(const moda_shape* shape, int for_bwd);
 
@@ -152,8 +160,13 @@ moda_status moda_fwd(const moda_shape* shape,
  *   O, LSE            the outputs of moda_fwd for the same inputs
  *   dO                incoming gradient [B, Hq, T, d]
  *   dQ, dK, dV, dKd, dVd   outputs (fully overwritten; dKd/dVd may be NULL if L = 0)
- *   ws, ws_bytes      workspace of at least moda_workspace_size(shape, 1) bytes
- * Deterministic: no floating-point atomics; repeated calls give identical bits.
+ *   ws, ws_bytes      workspace: at least moda_workspace_size(shape, 2) bytes;
+ *                     with moda_workspace_size(shape, 1) bytes or more the
+ *                     faster stored-dS path runs (the two paths round dS the
+ *                     same way but compute it in different kernels, so their
+ *                     results may differ in the last bits)
+ * Deterministic: no floating-point atomics; repeated calls with the same
+ * ws_bytes give identical bits.
  */
 moda_status moda_bwd(const moda_shape* shape,
                      const void* Q, const void* K, const void* V,

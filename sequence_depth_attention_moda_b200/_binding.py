@@ -174,8 +174,10 @@ def _check(rc: int, where: str):
         raise MoDAError(rc, where, detail)
 
 
-def moda_workspace_size(shape: moda_shape, for_bwd: bool) -> int:
-    n = load().moda_workspace_size(ctypes.byref(shape), 1 if for_bwd else 0)
+def moda_workspace_size(shape: moda_shape, for_bwd) -> int:
+    """for_bwd: 0/False forward, 1/True backward at its fastest, 2 the least
+    the backward accepts."""
+    n = load().moda_workspace_size(ctypes.byref(shape), int(for_bwd))
     if n == ctypes.c_size_t(-1).value:
         _check(load().moda_fwd(ctypes.byref(shape), *([None] * 7), None, 0, None), "moda_workspace_size")
     return int(n)

@@ -152,8 +152,10 @@ extern "C" {
 size_t moda_workspace_size(const moda_shape* shape, int for_bwd) {
     Problem p;
     if (validate(shape, &p) != MODA_OK) return static_cast<size_t>(-1);
+    if (for_bwd < 0 || for_bwd > 2) return static_cast<size_t>(-1);
     if (!for_bwd) return 0;
-    return bwd_workspace_bytes(p);
+    if (for_bwd == 2) return bwd_workspace_bytes(p);
+    return bwd_workspace_bytes(p) + bwd_ds_bytes(p);
 }
 
 moda_status moda_repack_depth(const moda_shape* shape, const void* src, void* dst,
@@ -215,7 +217,7 @@ moda_status moda_bwd(const moda_shape* shape, const void* Q, const void* K, cons
     phase_mark(0, s);
     cudaError_t e =
         p.elem_bytes == 2
-            ? launch_bwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, s)
+            ? launch_bwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, ws, ws_bytes, s)
             : launch_bwd_simt(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, s);
     return e == cudaSuccess ? MODA_OK : cuda_fail(e, "backward launch");
 }

@@ -33,6 +33,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <cmath>
+
 #include "moda_internal.h"
 #include "moda_ptx.cuh"
 
@@ -99,9 +101,55 @@ struct DkdvArgs {
     __nv_bfloat16* dV;
     unsigned int* status;
     int B, Hq, Hk, T, G, n_kt, n_qb;     // n_qb counts 64-row query blocks
+    int band;                            // (b, KV head) pairs per band (banded_item)
     int causal;
     float scale, scale_log2;
+    // Stored dS (nullptr: not stored): the tiles the dq kernel reads instead
+    // of recomputing S and dP; see store_ds_tile.
+    unsigned char* dS;
+    int n_qt, n_kb, tq_log2;             // dq query tiles (Tq = 1 << tq_log2 tokens), 64-key blocks
 };
+
+// Stored dS tiles.  Tile (bh, qt, kb) holds dS = P * (dP - D) (unscaled, bf16)
+// for the 128 rows of dq query tile qt (row r = g * Tq + t - qt * Tq, as in the
+// forward's tile) and the 64 keys of key block kb, laid out byte for byte as
+// the dq kernel's shared-memory A operand: MN-major with 128-byte swizzle,
+// two 8 KB slabs (rows 0-63 and 64-127), key k of the block at byte k * 128
+// of each slab, the 16-byte chunk of rows 8c .. 8c + 7 at chunk position
+// c ^ (k & 7).  Tiles are 16 KB, at ((bh * n_qt + qt) * n_kb + kb) * 16 KB.
+constexpr uint32_t kDsTileBytes = 128 * 64 * 2;
+
+// One dkdv math thread's 32 dS values (16 packed bf16 pairs in dk: key `key`,
+// head g, tokens t_first .. t_first + 31) into their tiles.  Needs Tq >= 16
+// (a power of two): the 32 tokens fall in one or two query tiles, each piece
+// a run of whole 16-byte chunks.  Keys past T get zeros; tiles past the last
+// key block or query tile are skipped.
+__device__ __forceinline__ void store_ds_tile(const DkdvArgs& a, int bh, int g, int key, int t_first,
+                                              const uint32_t* dk) {
+    const int kb = key >> 6, k = key & 63;
+    if (kb >= a.n_kb) return;
+    const bool live = key < a.T;
+    const int Tq = 1 << a.tq_log2;
+    const int per = Tq < 32 ? Tq : 32;            // tokens of one piece (16 or 32)
+#pragma unroll
+    for (int pc = 0; pc < 2; ++pc) {
+        if (pc * per >= 32) break;
+        const int t = t_first + pc * per;
+        const int qt = t >> a.tq_log2;
+        if (qt >= a.n_qt) break;
+        const int r0 = g * Tq + (t - (qt << a.tq_log2));
+        unsigned char* row = a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + kb) * kDsTileBytes +
+                             (r0 >> 6) * 8192 + k * 128;
+        const int cbase = (r0 & 63) >> 3;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (i * 8 >= per) break;
+            const int e = pc * 8 + 4 * i;            // first packed pair of the chunk (pc > 0 only if per = 16)
+            const uint4 v = live ? make_uint4(dk[e], dk[e + 1], dk[e + 2], dk[e + 3]) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(row + (((cbase + i) ^ (k & 7)) << 4)) = v;
+        }
+    }
+}
 
 constexpr int kKvBQ = 64;               // query rows per iteration
 constexpr int kKvStages = 3;            // Q/dO ring depth
@@ -142,8 +190,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nbh = a.B * a.Hk;
-    const int kt = static_cast<int>(blockIdx.x) / nbh;     // small kt = most work: first
-    const int bh = static_cast<int>(blockIdx.x) % nbh;
+    int kt, bh;                                             // small kt = most work: first
+    banded_item(static_cast<int>(blockIdx.x), a.n_kt, nbh, a.band, &kt, &bh);
     const int b = bh / a.Hk;
     const int hk = bh - b * a.Hk;
     const int qb0 = a.causal ? kt * (BN / kKvBQ) : 0;      // first query block that sees the keys
@@ -352,6 +400,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             __syncwarp();
             tmem_st16x2_16<16>(lane_base + buf * 64, pk);
             tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
+            if (a.dS) store_ds_tile(a, bh, g, k, tq0 + c0, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -409,7 +458,10 @@ struct DqArgs {
     unsigned int* status;
     int B, Hq, Hk, T, L, G, Tq, n_qt, dep_rows;
     int causal, win_lo;
+    int band;                            // (b, KV head) pairs per band (banded_item)
     float scale, scale_log2;
+    const unsigned char* dS;             // stored dS tiles (store_ds_tile), kStored only
+    int n_kb;                            // 64-key blocks per head
 };
 
 constexpr int kDqBN = 64;            // rows per key / depth block
@@ -438,7 +490,11 @@ enum { kB_QFull = 0, kB_KVFull = 1, kB_KVEmpty = 1 + kDqStages, kB_SFull = 1 + 2
 
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDKd = 384, kColDVd = 448;
 
-template <int D>
+// kStored: the sequence part reads the dS tiles the dK/dV kernel stored
+// (dQ += dS K straight from shared memory, no recomputation of S and dP, no
+// math); the tile's depth blocks come first and run as before.  Otherwise
+// every block recomputes S and dP, sequence blocks first.
+template <int D, bool kStored>
 __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__ DqArgs a) {
     using Lay = DqLayout<D>;
     extern __shared__ unsigned char smem_raw[];
@@ -451,8 +507,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nbh = a.B * a.Hk;
-    const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / nbh;
-    const int bh = static_cast<int>(blockIdx.x) % nbh;
+    int outer, bh;
+    banded_item(static_cast<int>(blockIdx.x), a.n_qt, nbh, a.band, &outer, &bh);
+    const int qt = a.n_qt - 1 - outer;                  // longest query tiles first
     const int b = bh / a.Hk;
     const int hk = bh - b * a.Hk;
     const int t0 = qt * a.Tq;
@@ -462,6 +519,10 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const int dep_total = a.L > 0 ? (t_end - t0) * a.L : 0;
     const int n_dep = (dep_total + a.dep_rows - 1) / a.dep_rows;
     const int nb = n_seq + n_dep;
+    // Block i of the tile, in the order of the variant.
+    auto is_dep = [&](int i) { return kStored ? i < n_dep : i >= n_seq; };
+    auto seq_idx = [&](int i) { return kStored ? i - n_dep : i; };
+    auto dep_idx = [&](int i) { return kStored ? i : i - n_seq; };
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kB_QFull], 1);
@@ -506,6 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             prefetch_tmap(&a.tq); prefetch_tmap(&a.tdo); prefetch_tmap(&a.tk); prefetch_tmap(&a.tv);
             if (a.L > 0) { prefetch_tmap(&a.tkd); prefetch_tmap(&a.tvd); }
             const uint32_t q_bytes = Lay::kSlabs * 128u * a.Tq * a.G;
+            const uint64_t once = policy_evict_first();
             mbar_arrive_expect_tx(&bars[kB_QFull], 2 * q_bytes);
             for (int s = 0; s < Lay::kSlabs; ++s) {
                 tma_load_3d(smem + Lay::kQ + s * kSlabBytes, &a.tq, &bars[kB_QFull], s * 64, t0, b * a.Hq + hk * a.G);
@@ -519,15 +581,33 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     break;
                 unsigned char* dk = smem + Lay::kK + st * Lay::kKTile;
                 unsigned char* dv = smem + Lay::kV + st * Lay::kKTile;
-                const bool seq = i < n_seq;
-                const int row0 = seq ? i * kDqBN : t0 * a.L + (i - n_seq) * a.dep_rows;
+                const bool seq = !is_dep(i);
+                const int row0 = seq ? seq_idx(i) * kDqBN : t0 * a.L + dep_idx(i) * a.dep_rows;
                 const uint32_t bytes = Lay::kSlabs * 128u * (seq ? kDqBN : a.dep_rows);
+                if (kStored && seq) {
+                    // K tile by TMA into the K slot, the stored dS tile (16 KB,
+                    // already in operand layout) by one bulk copy into the V slot
+                    static_assert(!kStored || Lay::kKTile == kDsTileBytes, "dS tile must fill the V slot");
+                    const unsigned char* tile =
+                        a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + seq_idx(i)) * kDsTileBytes;
+                    mbar_arrive_expect_tx(&bars[kB_KVFull + st], bytes + kDsTileBytes);
+                    for (int s = 0; s < Lay::kSlabs; ++s)
+                        tma_load_3d(dk + s * kDqSlab, &a.tk, &bars[kB_KVFull + st], s * 64, row0, bh);
+                    bulk_load_hint(dv, tile, kDsTileBytes, &bars[kB_KVFull + st], once);
+                    issued = i + 1;
+                    continue;
+                }
                 const void* mk = seq ? static_cast<const void*>(&a.tk) : static_cast<const void*>(&a.tkd);
                 const void* mv = seq ? static_cast<const void*>(&a.tv) : static_cast<const void*>(&a.tvd);
                 mbar_arrive_expect_tx(&bars[kB_KVFull + st], 2 * bytes);
                 for (int s = 0; s < Lay::kSlabs; ++s) {
-                    tma_load_3d(dk + s * kDqSlab, mk, &bars[kB_KVFull + st], s * 64, row0, bh);
-                    tma_load_3d(dv + s * kDqSlab, mv, &bars[kB_KVFull + st], s * 64, row0, bh);
+                    if (seq) {
+                        tma_load_3d(dk + s * kDqSlab, mk, &bars[kB_KVFull + st], s * 64, row0, bh);
+                        tma_load_3d(dv + s * kDqSlab, mv, &bars[kB_KVFull + st], s * 64, row0, bh);
+                    } else {   // depth tiles are read exactly once
+                        tma_load_3d_hint(dk + s * kDqSlab, mk, &bars[kB_KVFull + st], s * 64, row0, bh, once);
+                        tma_load_3d_hint(dv + s * kDqSlab, mv, &bars[kB_KVFull + st], s * 64, row0, bh, once);
+                    }
                 }
                 issued = i + 1;
             }
@@ -559,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 const int buf = j & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag))) return false;
                 tc_fence_after();
-                const uint32_t id = j < n_seq ? id_seq : id_dep;
+                const uint32_t id = is_dep(j) ? id_dep : id_seq;
                 const uint64_t kd = desc_kmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile));
                 const uint64_t vd = desc_kmajor_sw128(smem_u32(smem + Lay::kV + st * Lay::kKTile));
 #pragma unroll
@@ -578,8 +658,10 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 return true;
             };
             if (warp == 6) {
+                // kStored: only the depth blocks (blocks 0 .. n_dep-1) need S and dP
+                const int n_sdp = kStored ? n_dep : nb;
                 bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag));
-                for (int j = 0; ok && j < nb; ++j) {
+                for (int j = 0; ok && j < n_sdp; ++j) {
                     // buffer j & 1 last held dS(j-2), which dQ(j-2) reads: wait
                     // until that has completed (its K/V-stage release)
                     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVEmpty + (j - 2) % kDqStages],
@@ -589,10 +671,27 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 }
             } else {
                 bool ok = true;
+                const uint32_t id_dqs = idesc_bf16(128, D, true, true);   // A = stored dS, MN-major
                 for (int i = 0; ok && i < nb; ++i) {
                     const int st = i % kDqStages;
                     const int buf = i & 1;
-                    const bool seq = i < n_seq;
+                    const bool seq = !is_dep(i);
+                    if (kStored && seq) {
+                        // dQ += dS K: A = the dS tile in the V slot (two 64-row
+                        // slabs 8 KB apart; 16 keys = 2048 B per K step), B = the
+                        // K tile, MN-major
+                        if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVFull + st], (i / kDqStages) & 1,
+                                                               a.status, abort_flag))) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a_addr = smem_u32(smem + Lay::kV + st * Lay::kKTile);
+                        const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
+#pragma unroll
+                        for (int kk = 0; kk < kDqBN / 16; ++kk)
+                            umma_ss_elect(tmem + kColDQ, desc_mnmajor_sw128(a_addr + kk * 2048, 8192),
+                                          kmn + kk * (2048 >> 4), id_dqs, (i > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit_elect(&bars[kB_KVEmpty + st]);
+                        continue;
+                    }
                     const int n = seq ? kDqBN : a.dep_rows;
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
                     tc_fence_after();
@@ -675,9 +774,10 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
 
         bool ok = true;
         int jd = 0;
-        for (int i = 0; i < nb; ++i) {
+        const int n_math = kStored ? n_dep : nb;      // kStored: depth blocks only (blocks 0 .. n_dep-1)
+        for (int i = 0; i < n_math; ++i) {
             const int buf = i & 1;
-            const bool seq = i < n_seq;
+            const bool seq = !is_dep(i);
             if (!mbar_wait(&bars[kB_SFull + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t s[32], dp[32], dsk[16], pk[16];
@@ -689,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             int lo = 0, hi = kDqBN, kb = 0;
             const int lim = a.causal ? t_row : a.T - 1;   // last visible sequence key
             if (seq) {
-                kb = i * kDqBN;
+                kb = seq_idx(i) * kDqBN;
             } else {
                 const int base = t_row * a.L - (t0 * a.L + jd * a.dep_rows);
                 lo = base + a.win_lo;
@@ -794,12 +894,30 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     }
 }
 
+// The stored-dS backward: d = 128, G in {1, 2, 4, 8} (Tq = 128 / G >= 16, a
+// power of two, so a dK/dV thread's 32 queries fall in whole chunks of one or
+// two dq tiles), and at most this many bytes of tiles.
+constexpr double kMaxStoredDsBytes = 16.0 * 1024 * 1024 * 1024;
+
+int log2_exact(int x) {
+    int l = 0;
+    while ((1 << l) < x) ++l;
+    return (1 << l) == x ? l : -1;
+}
+
 template <int D>
 cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void* V,
                      const void* Kd, const void* Vd, const void* O, const float* LSE,
                      const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
-                     float* Dws, cudaStream_t stream) {
+                     void* ws, size_t ws_bytes, cudaStream_t stream) {
     cudaError_t e;
+    float* Dws = static_cast<float*>(ws);
+    const size_t ds_bytes = bwd_ds_bytes(p);
+    const bool stored = ds_bytes > 0 && ws_bytes >= bwd_workspace_bytes(p) + ds_bytes;
+    unsigned char* ds_tiles = stored ? static_cast<unsigned char*>(ws) + bwd_workspace_bytes(p) : nullptr;
+    const int Tq = BM / p.G;
+    const int n_qt = (p.T + Tq - 1) / Tq;
+    const int n_kb = (p.T + kDqBN - 1) / kDqBN;
     // 1. D = rowsum(dO * O)
     const long long nrows = (long long)p.B * p.Hq * p.T;
     constexpr int kRowsPerBlock = 8 * (32 / (D / 8));
@@ -819,6 +937,11 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     A.dK = static_cast<__nv_bfloat16*>(dK);
     A.dV = static_cast<__nv_bfloat16*>(dV);
     A.status = device_status_word();
+    A.band = l2_band(p.B * p.Hk, 2.0 * p.G * p.T * D * 2);   // Q and dO of one group
+    A.dS = ds_tiles;
+    A.n_qt = n_qt;
+    A.n_kb = n_kb;
+    A.tq_log2 = stored ? log2_exact(Tq) : 0;
     if ((e = make_tma_3d_bf16(&A.tk, K, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&A.tv, V, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&A.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
@@ -848,6 +971,9 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     B.dKd = static_cast<__nv_bfloat16*>(dKd);
     B.dVd = static_cast<__nv_bfloat16*>(dVd);
     B.status = device_status_word();
+    B.band = l2_band(p.B * p.Hk, 2.0 * p.T * D * 2);          // K and V of one head
+    B.dS = ds_tiles;
+    B.n_kb = n_kb;
     if ((e = make_tma_3d_bf16(&B.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&B.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&B.tk, K, D, p.T, (uint64_t)p.B * p.Hk, kDqBN, 1)) != cudaSuccess) return e;
@@ -862,10 +988,23 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     }
     {
         const uint32_t smem = DqLayout<D>::kDynSmem;
-        if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dq_kernel<D>), (int)smem)) != cudaSuccess)
-            return e;
         const long long grid = (long long)p.B * p.Hk * B.n_qt;
-        dq_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(B);
+        bool launched = false;
+        if constexpr (D == 128) {
+            if (stored) {
+                if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dq_kernel<D, true>), (int)smem)) !=
+                    cudaSuccess)
+                    return e;
+                dq_kernel<D, true><<<(unsigned)grid, kThreads, smem, stream>>>(B);
+                launched = true;
+            }
+        }
+        if (!launched) {
+            if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dq_kernel<D, false>), (int)smem)) !=
+                cudaSuccess)
+                return e;
+            dq_kernel<D, false><<<(unsigned)grid, kThreads, smem, stream>>>(B);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         phase_mark(3, stream);
     }
@@ -875,14 +1014,22 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
 }  // namespace
 
 
+size_t bwd_ds_bytes(const Problem& p) {
+    if (p.elem_bytes != 2 || p.d != 128 || !(p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8)) return 0;
+    const double Tq = BM / p.G;
+    const double tiles = double(p.B) * p.Hk * std::ceil(p.T / Tq) * std::ceil(p.T / double(kDqBN));
+    const double bytes = tiles * kDsTileBytes;
+    return bytes <= kMaxStoredDsBytes ? static_cast<size_t>(bytes) : 0;
+}
+
 cudaError_t launch_bwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, const void* O, const float* LSE,
                              const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
-                             float* Dws, cudaStream_t stream) {
+                             void* ws, size_t ws_bytes, cudaStream_t stream) {
     if (p.d == 128)
-        return launch_d<128>(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, stream);
+        return launch_d<128>(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, ws, ws_bytes, stream);
     if (p.d == 64)
-        return launch_d<64>(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, Dws, stream);
+        return launch_d<64>(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, ws, ws_bytes, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -74,20 +74,22 @@ struct FwdArgs {
     int B, Hq, Hk, T, L, G, Tq, n_qt, dep_rows;
     int causal;       // 0: every row sees keys 0..T-1
     int win_lo;       // first visible depth row of a token
-    int n_tiles;      // B * Hk * n_qt query tiles, longest first
+    int n_tiles;      // B * Hk * n_qt query tiles, longest first within a band of heads
+    int band;         // (b, KV head) pairs per band (banded_item)
     float scale_log2;
 };
 
-// Query tile `idx` of the longest-first order: the last query tiles of every
-// (b, hk) come first.  Blocks are n_seq key blocks, then the depth blocks.
+// Query tile `idx`: heads in bands (banded_item), and within a band the last
+// query tiles (the longest) of every (b, hk) first.  Blocks are n_seq key
+// blocks, then the depth blocks.
 struct FwdTile {
     int b, hk, bh, t0, t_end, n_seq, nb;
 };
 __device__ __forceinline__ FwdTile fwd_tile(const FwdArgs& a, int idx) {
-    const int nbh = a.B * a.Hk;
     FwdTile t;
-    const int qt = a.n_qt - 1 - idx / nbh;
-    t.bh = idx % nbh;
+    int outer;
+    banded_item(idx, a.n_qt, a.B * a.Hk, a.band, &outer, &t.bh);
+    const int qt = a.n_qt - 1 - outer;
     t.b = t.bh / a.Hk;
     t.hk = t.bh - t.b * a.Hk;
     t.t0 = qt * a.Tq;
@@ -191,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             unsigned char* ring = is_k ? sK : sV;
             const void* m_seq = is_k ? static_cast<const void*>(&a.tk) : static_cast<const void*>(&a.tv);
             const void* m_dep = is_k ? static_cast<const void*>(&a.tkd) : static_cast<const void*>(&a.tvd);
+            const uint64_t once = policy_evict_first();   // depth tiles are read exactly once
             prefetch_tmap(m_seq);
             if (a.L > 0) prefetch_tmap(m_dep);
             if (is_k) prefetch_tmap(&a.tq);
@@ -227,8 +230,12 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     const int row0 = seq ? i * BN : T.t0 * a.L + (i - T.n_seq) * a.dep_rows;
                     const uint32_t bytes = Lay::kSlabs * 128u * (seq ? BN : a.dep_rows);
                     mbar_arrive_expect_tx(&full[st], bytes);
-                    for (int s = 0; s < Lay::kSlabs; ++s)
-                        tma_load_3d(dst + s * kSlabBytes, seq ? m_seq : m_dep, &full[st], s * 64, row0, T.bh);
+                    for (int s = 0; s < Lay::kSlabs; ++s) {
+                        if (seq)
+                            tma_load_3d(dst + s * kSlabBytes, m_seq, &full[st], s * 64, row0, T.bh);
+                        else
+                            tma_load_3d_hint(dst + s * kSlabBytes, m_dep, &full[st], s * 64, row0, T.bh, once);
+                    }
                     issued = j + 1;
                 }
                 ++kt;
@@ -552,6 +559,7 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     const long long n_tiles = (long long)p.B * p.Hk * a.n_qt;
     if (n_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     a.n_tiles = static_cast<int>(n_tiles);
+    a.band = l2_band(p.B * p.Hk, 2.0 * p.T * D * 2);   // K and V of one head
     const long long seq_blocks = p.causal ? ((long long)p.T + BN - 1) / BN / 2 + 1 : ((long long)p.T + BN - 1) / BN;
     const long long avg_blocks = seq_blocks + ((long long)a.Tq * p.L + a.dep_rows - 1) / a.dep_rows;
     const long long sms = device_sm_count() > 0 ? device_sm_count() : 1;

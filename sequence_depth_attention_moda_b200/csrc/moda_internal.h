@@ -43,6 +43,34 @@ __host__ __device__ inline int snake_tile(int r, int c, int G) {
     return r * G + ((r & 1) ? G - 1 - c : c);
 }
 
+// Work item `idx` of a list of n_outer x nbh items, in bands of `band`
+// (b, KV head) pairs: every item of the first band's heads (outer index 0,
+// 1, ... for each head in turn), then the next band.  Items that run at the
+// same time then share the K/V (or Q/dO) of only a few heads, which stay in
+// L2 while the band lasts instead of being re-read from HBM for every outer
+// index.  With band >= nbh this is the plain outer-major order.
+__host__ __device__ inline void banded_item(int idx, int n_outer, int nbh, int band, int* outer,
+                                            int* bh) {
+    const int per_band = band * n_outer;
+    const int bi = idx / per_band;
+    const int local = idx - bi * per_band;
+    const int h0 = bi * band;
+    const int hb = nbh - h0 < band ? nbh - h0 : band;
+    *outer = local / hb;
+    *bh = h0 + (local - *outer * hb);
+}
+
+// Heads per band.  When every head's re-read operands (`bytes_per_head`
+// each) fit in half of the 126 MB L2 together, no banding (nbh: the plain
+// longest-first order over all heads keeps the best load balance); else as
+// many heads as fit in a 32 MB share, at least one.
+inline int l2_band(int nbh, double bytes_per_head) {
+    const double mib = 1024.0 * 1024.0;
+    if (bytes_per_head <= 0 || nbh * bytes_per_head <= 64.0 * mib) return nbh;
+    const int b = static_cast<int>(32.0 * mib / bytes_per_head);
+    return b < 1 ? 1 : (b > nbh ? nbh : b);
+}
+
 // Records the calling thread's k-th phase marker on `stream`, if one is set
 // (see moda_set_phase_events); a no-op otherwise.
 void phase_mark(int k, cudaStream_t stream);
@@ -73,13 +101,20 @@ cudaError_t launch_bwd_simt(const Problem& p, const void* Q, const void* K, cons
 cudaError_t launch_fwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, void* O, float* LSE,
                              cudaStream_t stream);
+// ws holds D = rowsum(dO * O) (bwd_workspace_bytes) and, when ws_bytes also
+// covers bwd_ds_bytes after it, the stored dS tiles; otherwise the dQ kernel
+// recomputes S and dP.
 cudaError_t launch_bwd_sm100(const Problem& p, const void* Q, const void* K, const void* V,
                              const void* Kd, const void* Vd, const void* O, const float* LSE,
                              const void* dO, void* dQ, void* dK, void* dV, void* dKd, void* dVd,
-                             float* Dws, cudaStream_t stream);
+                             void* ws, size_t ws_bytes, cudaStream_t stream);
 
-// Workspace bytes the backward needs: D = rowsum(dO * O), fp32 [B, Hq, T].
+// Workspace bytes the backward needs at least: D = rowsum(dO * O), fp32
+// [B, Hq, T], rounded up to 256 bytes.
 size_t bwd_workspace_bytes(const Problem& p);
+// Bytes of stored dS tiles the faster backward uses on top of that (0 when it
+// does not apply to this shape).
+size_t bwd_ds_bytes(const Problem& p);
 
 // ---- TMA descriptors (moda_tma.cu) -------------------------------------------
 // A 3-D bf16 tensor map over a row-major [outer, rows, d] tensor, box

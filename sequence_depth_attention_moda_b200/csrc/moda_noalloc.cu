@@ -95,12 +95,14 @@ extern "C" moda_status moda_bwd_noalloc(const moda_shape* shape, const void* Q, 
     float* scratch = nullptr;
     if ((st = scratch_for_current_device(&scratch)) != MODA_OK) return st;
     // D rows need no clearing: the first kernel of the call writes every row
-    // of [0, B*Hq*T) before any later kernel reads it.
+    // of [0, B*Hq*T) before any later kernel reads it.  Only the D rows are
+    // offered, so the dQ kernel recomputes S and dP (no stored dS tiles).
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     phase_mark(0, s);
     cudaError_t e =
         p.elem_bytes == 2
-            ? launch_bwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, scratch, s)
+            ? launch_bwd_sm100(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, scratch,
+                               bwd_workspace_bytes(p), s)
             : launch_bwd_simt(p, Q, K, V, Kd, Vd, O, LSE, dO, dQ, dK, dV, dKd, dVd, scratch, s);
     if (e != cudaSuccess) {
         char msg[160];

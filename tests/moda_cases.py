@@ -49,12 +49,15 @@ class Guarded:
     def __init__(self):
         self.items = []
 
-    def empty(self, name: str, shape, dtype, device) -> torch.Tensor:
+    def empty(self, name: str, shape, dtype, device, output: bool = True) -> torch.Tensor:
+        """A guarded tensor; an output (not a workspace) also starts as NaN
+        and must be fully written."""
         n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
         raw = torch.full((2 * GUARD_BYTES + n,), GUARD_BYTE, dtype=torch.uint8, device=device)
         view = raw[GUARD_BYTES:GUARD_BYTES + n].view(dtype).view(*shape)
-        view.fill_(float("nan"))
-        self.items.append((name, raw, n, view))
+        if output:
+            view.fill_(float("nan"))
+        self.items.append((name, raw, n, view if output else None))
         return view
 
     def like(self, name: str, t: torch.Tensor) -> torch.Tensor:
@@ -67,7 +70,8 @@ class Guarded:
             head, tail = raw[:GUARD_BYTES], raw[GUARD_BYTES + n:]
             assert bool((head == GUARD_BYTE).all()), f"{name}: bytes written before the tensor"
             assert bool((tail == GUARD_BYTE).all()), f"{name}: bytes written past the end of the tensor"
-            assert not bool(torch.isnan(view).any()), f"{name}: elements left unwritten"
+            if view is not None:
+                assert not bool(torch.isnan(view).any()), f"{name}: elements left unwritten"
 
 
 def shape_of(w: Workload, layout=moda.MODA_DEPTH_FLAT, C=None):
@@ -78,10 +82,12 @@ def shape_of(w: Workload, layout=moda.MODA_DEPTH_FLAT, C=None):
 
 
 def run_gpu(w: Workload, x: Dict[str, torch.Tensor], backward=None, layout=moda.MODA_DEPTH_FLAT,
-            C=None, null_depth_if_empty=True):
+            C=None, null_depth_if_empty=True, ws_mode: int = 1):
     """Repack the depth cache, run the forward (and backward) on the current
-    stream; returns a dict of device tensors.  Every output is guarded
-    (``Guarded``) and checked before returning."""
+    stream; returns a dict of device tensors.  Every output (and the
+    backward's workspace) is guarded (``Guarded``) and checked before
+    returning.  ws_mode: the backward's workspace, moda_workspace_size(shape,
+    ws_mode) bytes (1: the fastest path, 2: the least it accepts)."""
     sh = shape_of(w, layout, C)
     dev = x["Q"].device
     dt = x["Q"].dtype
@@ -100,8 +106,8 @@ def run_gpu(w: Workload, x: Dict[str, torch.Tensor], backward=None, layout=moda.
     moda.moda_fwd(sh, x["Q"], x["K"], x["V"], Kd, Vd, O, LSE)
     out["O"], out["LSE"] = O, LSE
     if backward if backward is not None else w.backward:
-        nws = moda.moda_workspace_size(sh, True)
-        ws = torch.empty(max(nws, 16), device=dev, dtype=torch.uint8)
+        nws = moda.moda_workspace_size(sh, ws_mode)
+        ws = gd.empty("workspace", (max(nws, 16),), torch.uint8, dev, output=False)
         dQ = gd.like("dQ", x["Q"])
         dK = gd.like("dK", x["K"])
         dV = gd.like("dV", x["V"])

@@ -87,7 +87,7 @@ def test_fwd_rejects_null_and_misaligned(lib):
 
 def test_bwd_rejects_small_workspace(lib):
     sh = moda.make_shape(1, 4, 2, 64, 128, 2, 16)
-    need = lib.moda_workspace_size(ctypes.byref(sh), 1)
+    need = lib.moda_workspace_size(ctypes.byref(sh), 2)
     assert need == 4 * 4 * 64  # fp32 D = rowsum(dO * O), [B, Hq, T], 256-byte rounded
     rc = lib.moda_bwd(ctypes.byref(sh), *([FAKE] * 13), FAKE, need - 1, None)
     assert rc == 4
@@ -95,12 +95,31 @@ def test_bwd_rejects_small_workspace(lib):
     assert rc == 4
 
 
+def ws(lib, sh, mode):
+    return lib.moda_workspace_size(ctypes.byref(sh), mode)
+
+
 def test_workspace_sizes(lib):
     sh = moda.make_shape(2, 16, 4, 4096, 128, 16, 64)
-    assert lib.moda_workspace_size(ctypes.byref(sh), 0) == 0
-    assert lib.moda_workspace_size(ctypes.byref(sh), 1) == 2 * 16 * 4096 * 4
+    d_rows = 2 * 16 * 4096 * 4                     # D: one fp32 per query row
+    # stored dS: one 16 KB tile per (b, hk, 128-row query tile of G=4 heads x
+    # 32 tokens, 64-key block)
+    tiles = 2 * 4 * (4096 // 32) * (4096 // 64)
+    assert ws(lib, sh, 0) == 0
+    assert ws(lib, sh, 2) == d_rows
+    assert ws(lib, sh, 1) == d_rows + tiles * 16384
+    # ragged T: whole tiles, D rounded up to 256 bytes
+    sh = moda.make_shape(1, 8, 1, 1000, 128, 3, 0)  # G = 8: 16 tokens per query tile
+    assert ws(lib, sh, 2) == (8 * 1000 * 4 + 255) // 256 * 256
+    assert ws(lib, sh, 1) == ws(lib, sh, 2) + (-(-1000 // 16)) * (-(-1000 // 64)) * 16384
+    # no stored dS: G not in {1, 2, 4, 8}, d = 64, fp32, or more than 16 GiB of tiles
+    for s in (moda.make_shape(1, 6, 2, 300, 128, 2, 0), moda.make_shape(1, 4, 2, 300, 64, 2, 0),
+              moda.make_shape(1, 4, 2, 300, 128, 2, 0, moda.MODA_FP32),
+              moda.make_shape(1, 16, 4, 65536, 128, 32, 64)):
+        assert ws(lib, s, 1) == ws(lib, s, 2) > 0
     bad = moda.make_shape(2, 16, 5, 4096, 128, 16, 64)
-    assert lib.moda_workspace_size(ctypes.byref(bad), 1) == ctypes.c_size_t(-1).value
+    assert ws(lib, bad, 1) == ctypes.c_size_t(-1).value
+    assert ws(lib, moda.make_shape(1, 4, 2, 64, 128, 2, 0), 3) == ctypes.c_size_t(-1).value
 
 
 def test_empty_problems_are_noops(lib):

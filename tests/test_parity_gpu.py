@@ -223,12 +223,49 @@ def test_bwd_deterministic():
         assert torch.equal(a[k], b[k]), k
 
 
+# (B, Hq, Hk, d, T, L, causal, window): every G the stored-dS backward takes
+# (1, 2, 4, 8), ragged T, the modes; G = 3 and d = 64 fall back to recomputing
+BOTH_PATHS = [
+    (1, 4, 4, 128, 300, 5, True, 0),      # G = 1: 128 tokens per query tile
+    (2, 4, 2, 128, 257, 3, True, 0),      # G = 2
+    (1, 8, 2, 128, 513, 16, True, 0),     # G = 4
+    (1, 16, 2, 128, 200, 6, True, 0),     # G = 8: 16 tokens per query tile
+    (1, 8, 2, 128, 300, 8, False, 3),     # non-causal, depth window
+    (1, 8, 1, 128, 129, 0, True, 0),      # L = 0, ragged last tile of 128 tokens
+    (1, 6, 2, 128, 100, 5, True, 0),      # G = 3: no stored path
+    (1, 8, 2, 64, 200, 4, True, 0),       # d = 64: no stored path
+]
+
+
+@pytest.mark.parametrize("case", BOTH_PATHS, ids=lambda c: "B%d_Hq%d_Hk%d_d%d_T%d_L%d_c%d_w%d" % c)
+def test_bwd_stored_and_recomputed_paths(case):
+    """The backward with its full workspace (dS stored by the dK/dV kernel,
+    read by the dQ kernel) and with the least workspace (dQ kernel
+    recomputes S and dP): both match the oracle, the workspace guards hold,
+    and each is bitwise repeatable."""
+    B, Hq, Hk, d, T, L, causal, window = case
+    w = small_w(B, Hq, Hk, d, T, L, backward=True).with_(causal=causal, window=window)
+    x = I.make_inputs(w, device=DEV)
+    ref = oracle_bwd_full(w, x)
+    for mode in (1, 2):
+        out = run_gpu(w, x, ws_mode=mode)
+        for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), ref):
+            if out[name] is None:
+                assert r.size == 0
+                continue
+            assert_grad_close(f64(out[name]), r, f"ws_mode {mode} {name}")
+        again = run_gpu(w, x, ws_mode=mode)
+        for name in ("dQ", "dK", "dV", "dKd", "dVd"):
+            if out[name] is not None:
+                assert torch.equal(out[name], again[name]), f"ws_mode {mode} {name} not repeatable"
+
+
 def test_bwd_workspace_error_on_device():
     w = small_w(1, 4, 2, 128, 64, 2, backward=True)
     x = I.make_inputs(w, device=DEV)
     out = run_gpu(w, x, backward=False)
     sh = moda.make_shape(w.B, w.Hq, w.Hk, w.T, w.d, w.L, w.C)
-    need = moda.moda_workspace_size(sh, True)
+    need = moda.moda_workspace_size(sh, 2)
     ws = torch.empty(need, device=DEV, dtype=torch.uint8)
     g = {k: torch.empty_like(v) for k, v in (("dQ", x["Q"]), ("dK", x["K"]), ("dV", x["V"]),
                                             ("dKd", out["Kd"]), ("dVd", out["Vd"]))}

@@ -3,18 +3,20 @@ memory where they run it (a plugin whose host framework forbids allocation
 during execution, code replaying a fixed memory plan).  Its scratch is a fixed
 array inside the library instead of a caller workspace.
 
-It runs the same kernels as moda_bwd (the entry point that takes a workspace),
-so its results must be bit-identical to moda_bwd's, on two calls in a row with
+It runs the same kernels as moda_bwd given the least workspace moda_bwd
+accepts (moda_workspace_size(shape, 2): the dQ kernel recomputes S and dP), so
+its results must be bit-identical to those, on two calls in a row with
 different inputs (scratch contents left behind by the first call must not leak
-into the second), for the tensor-core bf16 path and the CUDA-core fp32 path.
-This file is collected last.
+into the second), for the tensor-core bf16 path and the CUDA-core fp32 path;
+and within the gradient tolerance of moda_bwd with its full workspace (the
+stored-dS path).  This file is collected last.
 """
 import pytest
 import torch
 
 import sequence_depth_attention_moda_b200 as moda
 from sequence_depth_attention_moda_b200 import inputs as I
-from moda_cases import Guarded, run_gpu, shape_of
+from moda_cases import Guarded, assert_grad_close, f64, run_gpu, shape_of
 
 pytestmark = pytest.mark.gpu
 
@@ -40,12 +42,14 @@ def test_noalloc_matches_workspace_backward_twice(w):
     for call, seed in enumerate((w.seed, w.seed + 101)):
         wc = w.with_(seed=seed)
         x = I.make_inputs(wc, device="cuda")
-        ref = run_gpu(wc, x)                     # repack + forward + moda_bwd with a workspace
+        ref = run_gpu(wc, x, ws_mode=2)          # repack + forward + moda_bwd, least workspace
+        fast = run_gpu(wc, x, ws_mode=1)         # moda_bwd with its full workspace
         got = _grads_noalloc(wc, x, ref)
         torch.cuda.synchronize()
         moda.moda_check_status()
         for k in NAMES:
             assert torch.equal(got[k], ref[k]), f"call {call} {k}: differs from moda_bwd"
+            assert_grad_close(f64(got[k]), f64(fast[k]), f"call {call} {k} vs the stored-dS path")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
