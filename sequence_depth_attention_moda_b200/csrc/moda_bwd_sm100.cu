@@ -113,10 +113,11 @@ struct DkdvArgs {
 // Stored dS tiles.  Tile (bh, qt, kb) holds dS = P * (dP - D) (unscaled, bf16)
 // for the 128 rows of dq query tile qt (row r = g * Tq + t - qt * Tq, as in the
 // forward's tile) and the 64 keys of key block kb, laid out byte for byte as
-// the dq kernel's shared-memory A operand: MN-major with 128-byte swizzle,
-// two 8 KB slabs (rows 0-63 and 64-127), key k of the block at byte k * 128
-// of each slab, the 16-byte chunk of rows 8c .. 8c + 7 at chunk position
-// c ^ (k & 7).  Tiles are 16 KB, at ((bh * n_qt + qt) * n_kb + kb) * 16 KB.
+// the dq kernel's shared-memory A operand, MN-major without swizzle: the 16
+// bytes of rows 8c .. 8c + 7 for key k at byte c * 1024 + k * 16.  A dK/dV
+// thread holds one key and 32 consecutive rows, so the 16 keys of a half warp
+// write 256 contiguous bytes per store.  Tiles are 16 KB, at
+// ((bh * n_qt + qt) * n_kb + kb) * 16 KB.
 constexpr uint32_t kDsTileBytes = 128 * 64 * 2;
 
 // One dkdv math thread's 32 dS values (16 packed bf16 pairs in dk: key `key`,
@@ -138,15 +139,14 @@ __device__ __forceinline__ void store_ds_tile(const DkdvArgs& a, int bh, int g, 
         const int qt = t >> a.tq_log2;
         if (qt >= a.n_qt) break;
         const int r0 = g * Tq + (t - (qt << a.tq_log2));
-        unsigned char* row = a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + kb) * kDsTileBytes +
-                             (r0 >> 6) * 8192 + k * 128;
-        const int cbase = (r0 & 63) >> 3;
+        unsigned char* base = a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + kb) * kDsTileBytes +
+                              (r0 >> 3) * 1024 + k * 16;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             if (i * 8 >= per) break;
             const int e = pc * 8 + 4 * i;            // first packed pair of the chunk (pc > 0 only if per = 16)
             const uint4 v = live ? make_uint4(dk[e], dk[e + 1], dk[e + 2], dk[e + 3]) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(row + (((cbase + i) ^ (k & 7)) << 4)) = v;
+            *reinterpret_cast<uint4*>(base + i * 1024) = v;
         }
     }
 }
@@ -677,9 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     const int buf = i & 1;
                     const bool seq = !is_dep(i);
                     if (kStored && seq) {
-                        // dQ += dS K: A = the dS tile in the V slot (two 64-row
-                        // slabs 8 KB apart; 16 keys = 2048 B per K step), B = the
-                        // K tile, MN-major
+                        // dQ += dS K: A = the dS tile in the V slot (MN-major,
+                        // no swizzle: 8 keys 128 B apart, 8 rows 1024 B apart; 16
+                        // keys = 256 B per K step), B = the K tile, MN-major
                         if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVFull + st], (i / kDqStages) & 1,
                                                                a.status, abort_flag))) { ok = false; break; }
                         tc_fence_after();
@@ -687,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                         const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
 #pragma unroll
                         for (int kk = 0; kk < kDqBN / 16; ++kk)
-                            umma_ss_elect(tmem + kColDQ, desc_mnmajor_sw128(a_addr + kk * 2048, 8192),
+                            umma_ss_elect(tmem + kColDQ, desc_mnmajor_noswizzle(a_addr + kk * 256, 128, 1024),
                                           kmn + kk * (2048 >> 4), id_dqs, (i > 0 || kk > 0) ? 1u : 0u);
                         umma_commit_elect(&bars[kB_KVEmpty + st]);
                         continue;

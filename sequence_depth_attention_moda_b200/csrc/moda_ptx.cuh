@@ -359,6 +359,19 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t 
     return desc;
 }
 
+// MN-major operand without swizzle: core matrices of 8 K rows x 16 bytes (8
+// MN elements) stored as 128 contiguous bytes; the next core matrix along K
+// lbo_bytes further, along MN sbo_bytes further.  Advancing K by 16 elements
+// (two core matrices) adds 2 * lbo_bytes to the address.
+__device__ __forceinline__ uint64_t desc_mnmajor_noswizzle(uint32_t saddr, uint32_t lbo_bytes,
+                                                           uint32_t sbo_bytes) {
+    uint64_t desc = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    desc |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    desc |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    desc |= static_cast<uint64_t>(1u) << 46;                // descriptor version; swizzle 0 = none
+    return desc;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                                   // D = f32
