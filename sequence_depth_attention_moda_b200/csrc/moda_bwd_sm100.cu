@@ -465,7 +465,7 @@ struct DqArgs {
 };
 
 constexpr int kDqBN = 64;            // rows per key / depth block
-constexpr int kDqStages = 3;         // K/V ring depth
+constexpr int kDqStages = 4;         // K/V ring depth (stored dS: K + dS tile per stage)
 constexpr uint32_t kDqSlab = 64 * 128;   // 64 rows x 64 bf16
 
 template <int D>
