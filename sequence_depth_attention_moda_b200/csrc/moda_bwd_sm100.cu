@@ -48,7 +48,8 @@ constexpr int BN = 128;
 constexpr int kThreads = 352;            // dq: warp 0 TMA, warps 1 and 6 MMA, warps 2..5 and 7..10 math
 constexpr int kMathThreads = 256;
 constexpr int kKvMathWarps = 8;          // dkdv: warps 2..9, two per TMEM lane quarter
-constexpr int kKvThreads = 64 + 32 * kKvMathWarps;
+constexpr int kKvGradWarp = 2 + kKvMathWarps;   // dkdv: issuer of dV and dK (warp 10)
+constexpr int kKvThreads = 32 * (kKvGradWarp + 1);
 constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -292,8 +293,12 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             for (int it = max(0, issued - kKvStages); it < issued; ++it)
                 mbar_wait(&bars[kA_QFull + it % kKvStages], (it / kKvStages) & 1, a.status, abort_flag);
         }
-    } else if (warp == 1) {
-        // whole warp, converged: warp-uniform waits, one elected lane issues
+    } else if (warp == 1 || warp == kKvGradWarp) {
+        // Two issuers on different sub-partitions: warp 1 the score products
+        // S^T, dP^T, warp kKvGradWarp the gradient products dV, dK (issuing a
+        // tcgen05.mma costs its warp tens of cycles, more while math warps
+        // share the sub-partition).  Each runs converged: warp-uniform waits,
+        // one elected lane issues; a commit tracks only its own warp's MMAs.
         {
             const uint32_t id_s = idesc_bf16(128, kKvBQ, false, false);
             const uint32_t id_g = idesc_bf16(128, D, false, true);
@@ -327,24 +332,36 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 umma_commit_elect(&bars[kA_SFull + buf]);
                 return true;
             };
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag)) && (n_it == 0 || issue_s(0));
-            for (int it = 0; ok && it < n_it; ++it) {
-                if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
-                const int st = it % kKvStages;
-                const int buf = it & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
-                tc_fence_after();
-                const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
-                const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
-#pragma unroll
-                for (int kk = 0; kk < kKvBQ / 16; ++kk) {
-                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts_elect(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, acc);
-                    umma_ts_elect(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g, acc);
+            if (warp == 1) {
+                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag));
+                for (int it = 0; ok && it < n_it; ++it) {
+                    // buffer it & 1 held P^T / dS^T of iteration it - 2, read by
+                    // its dV / dK products: wait for their completion (the
+                    // Q/dO-stage release of that iteration)
+                    if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + (it - 2) % kKvStages],
+                                                                      ((it - 2) / kKvStages) & 1, a.status,
+                                                                      abort_flag))) { ok = false; break; }
+                    if (!issue_s(it)) { ok = false; break; }
                 }
-                umma_commit_elect(&bars[kA_QEmpty + st]);
+            } else {
+                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag));
+                for (int it = 0; ok && it < n_it; ++it) {
+                    const int st = it % kKvStages;
+                    const int buf = it & 1;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
+                    const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
+#pragma unroll
+                    for (int kk = 0; kk < kKvBQ / 16; ++kk) {
+                        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                        umma_ts_elect(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, acc);
+                        umma_ts_elect(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g, acc);
+                    }
+                    umma_commit_elect(&bars[kA_QEmpty + st]);
+                }
+                umma_commit_elect(&bars[kA_Final]);
             }
-            umma_commit_elect(&bars[kA_Final]);
         }
     } else {
         // Math warps 2..9: two per TMEM lane quarter, each on 16 key rows;
@@ -700,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     // (kk % 2) * 8 of the buffer (each math half packs its 32 keys
                     // into the first 16 of its own 32 columns)
                     if (n == kDqBN) {
-    #pragma unroll
+#pragma unroll
                         for (int kk = 0; kk < kDqBN / 16; ++kk)
                             umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
                                     kmn + kk * (2048 >> 4), id_dq, (i > 0 || kk > 0) ? 1u : 0u);
@@ -710,7 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                                     kmn + kk * (2048 >> 4), id_dq, (i > 0 || kk > 0) ? 1u : 0u);
                     }
                     if (!seq) {
-    #pragma unroll
+#pragma unroll
                         for (int kk = 0; kk < BM / 16; ++kk) {
                             umma_ss_elect(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
                                     desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);

@@ -16,18 +16,19 @@
 // group, and the depth rows of the tile's Tq tokens are one contiguous range
 // [t0*L, (t0+Tq)*L) of the token-major depth tensor.
 //
-// CTA roles (352 threads):
+// CTA roles (384 threads):
 //   warp 0      TMA producer of Q (once) and of the K (or K_depth) tiles;
 //   warp 10     TMA producer of the V (or V_depth) tiles.  K and V have rings
 //               of their own: a K stage frees as soon as S_i = Q K_i^T is
 //               done, a V stage only when O += P_i V_i is, so the next K
 //               tiles stream in while PV still holds older V tiles.
-//   warp 1      TMEM allocator and MMA issuer (one thread):
-//               S_i = Q K_i^T into one of three TMEM S buffers, and
-//               O += P_i V_i with P read from TMEM; S_{i+2} is issued
-//               before PV_i, so two score tiles are always ahead of the
-//               softmax and the tensor pipe's issue-to-completion latency
-//               (hundreds of cycles) is off the softmax's critical path.
+//   warp 11     score-MMA issuer: S_i = Q K_i^T into one of three TMEM S
+//               buffers, up to three blocks ahead of the PV products, so
+//               score tiles are ready before the softmax needs them and the
+//               tensor pipe's issue-to-completion latency (hundreds of
+//               cycles) is off the softmax's critical path.
+//   warp 1      TMEM allocator and PV-MMA issuer: O += P_i V_i with P read
+//               from TMEM.  The two issuers sit on different sub-partitions.
 //   warps 2..9  softmax, two warps per TMEM lane quarter (16 rows each) and
 //               two threads per tile row: with the 16x32bx2 TMEM shapes,
 //               thread t < 16 holds columns [0, 64) of its row and thread
@@ -59,7 +60,8 @@ constexpr int kKStages = 3;      // K ring: a stage frees when S_i is done
 constexpr int kVStages = 3;      // V ring: a stage frees when PV_i is done
 constexpr int kSoftmaxWarps = 8;             // warps 2..9
 constexpr int kVWarp = 2 + kSoftmaxWarps;    // V producer
-constexpr int kThreads = 32 * (kVWarp + 1);
+constexpr int kSWarp = kVWarp + 1;           // score-MMA issuer (sub-partition 3)
+constexpr int kThreads = 32 * (kSWarp + 1);
 constexpr float kLazyLimit = 1024.0f;     // largest half-row sum of p kept without a rescale
 constexpr uint32_t kSlabBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
@@ -119,6 +121,7 @@ enum { kQFull = 0, kKFull = 1, kVFull = kKFull + kKStages, kVEmpty = kVFull + kV
        kSFull = kVEmpty + kVStages, kPReady = kSFull + kSBufs, kOFinal = kPReady + kSBufs,
        kOFree = kOFinal + 1, kNumBars = kOFree + 1 };
 static_assert(kKStages == kSBufs, "a K stage is released by the score barrier of its S buffer");
+static_assert(kVStages == kSBufs, "an S buffer is free again at the V-stage release of its PV");
 
 // kPersist: CTAs walk several tiles (grid = SM count); otherwise each CTA
 // takes exactly tile blockIdx.x and the tile loops compile away.
@@ -245,11 +248,15 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             for (int i = max(0, issued - nst); i < issued; ++i)
                 mbar_wait(&full[i % nst], (i / nst) & 1, a.status, abort_flag);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer --
-        // The whole warp runs this loop converged, so descriptors and waits
-        // are warp-uniform; elect.sync picks the lane that issues each MMA
-        // and commit.
+    } else if (warp == 1 || warp == kSWarp) {
+        // ------------------------------------------------------ MMA issuers -
+        // Two warps issue: warp kSWarp the score products S(j), warp 1 the
+        // PV(j) products.  Issuing a tcgen05.mma costs its warp tens of
+        // cycles, and every wait and commit more while a softmax warp shares
+        // the sub-partition; one warp issuing both products was the forward's
+        // bound, so the two streams now run on two sub-partitions.  Each warp
+        // runs its loop converged (warp-uniform waits, elect.sync picks the
+        // issuing lane); a commit tracks only its own warp's MMAs.
         const uint32_t id_seq = idesc_bf16(128, BN, false, false);
         const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
         const uint32_t id_pv = idesc_bf16(128, D, false, true);
@@ -257,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         // the 14-bit address field (shared addresses stay < 256 KB).
         const uint64_t qd0 = desc_kmajor_sw128(smem_u32(sQ));
         // S(j) = Q K_j^T into buffer j % 3 (i: the block's index in its tile).
-        // The buffer last held P(j-3), read by PV(j-3), which is issued before
-        // S(j) (in-order pipe).
+        // The buffer last held P(j-3), read by PV(j-3): the caller waits for
+        // that product's completion (its V-stage release) first.
         auto issue_s = [&](int j, int i, const FwdTile& T) -> bool {
             const int st = j % kKStages;
             const int sb = j % kSBufs;
@@ -300,33 +307,41 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             umma_commit_elect(&bars[kVEmpty + st]);
             return true;
         };
-        // Two score tiles run ahead of the softmax.  S(i+2) goes in before
-        // PV(i): its buffer held P(i-1), whose PV(i-1) is already in the
-        // (in-order) pipe, so it never waits for P(i); each issue blocks
-        // until the shallow MMA queue has room, so this order is what keeps
-        // the next scores ready when the softmax needs them.
+        // The score issuer runs up to three blocks ahead of the PV issuer
+        // (three S buffers), so two score tiles are ready before the softmax
+        // needs them.
         bool ok = true;
         int j0 = 0, kt = 0;
+        const bool s_role = warp == kSWarp;
         for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
             const int tile = tile_of(rnd);
             if (tile >= a.n_tiles) continue;
             const FwdTile T = fwd_tile(a, tile);
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], kt & 1, a.status, abort_flag));
-            if (ok) ok = issue_s(j0, 0, T);
-            if (ok && T.nb > 1) ok = issue_s(j0 + 1, 1, T);
-            for (int i = 0; ok && i < T.nb; ++i) {
-                if (i + 2 < T.nb && !issue_s(j0 + i + 2, i + 2, T)) { ok = false; break; }
-                // the tile's first PV overwrites O: the softmax warps must have
-                // read the previous tile's O out
-                if (i == 0 && kt > 0 &&
-                    !__all_sync(0xffffffffu, mbar_wait(&bars[kOFree], (kt - 1) & 1, a.status, abort_flag))) {
-                    ok = false;
-                    break;
+            if (s_role) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], kt & 1, a.status, abort_flag));
+                for (int i = 0; ok && i < T.nb; ++i) {
+                    const int j = j0 + i;
+                    // buffer j % 3 held P(j-3): PV(j-3) must have completed
+                    if (j >= kSBufs &&
+                        !__all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + (j - kSBufs) % kVStages],
+                                                           ((j - kSBufs) / kVStages) & 1, a.status,
+                                                           abort_flag))) { ok = false; break; }
+                    if (!issue_s(j, i, T)) { ok = false; break; }
                 }
-                if (i == 0) tc_fence_after();
-                if (!issue_pv(j0 + i, i, T)) { ok = false; break; }
+            } else {
+                for (int i = 0; ok && i < T.nb; ++i) {
+                    // the tile's first PV overwrites O: the softmax warps must
+                    // have read the previous tile's O out
+                    if (i == 0 && kt > 0 &&
+                        !__all_sync(0xffffffffu, mbar_wait(&bars[kOFree], (kt - 1) & 1, a.status, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    if (i == 0) tc_fence_after();
+                    if (!issue_pv(j0 + i, i, T)) { ok = false; break; }
+                }
+                umma_commit_elect(&bars[kOFinal]);
             }
-            umma_commit_elect(&bars[kOFinal]);
             j0 += T.nb;
             ++kt;
         }
