@@ -713,6 +713,19 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
+                    // depth block: the gradient products first, so their
+                    // completion (which the math warps wait for before the next
+                    // depth block) does not queue behind this block's dQ
+                    if (!seq) {
+#pragma unroll
+                        for (int kk = 0; kk < BM / 16; ++kk) {
+                            umma_ss_elect(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
+                                    desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                            umma_ss_elect(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
+                                    desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit_elect(&bars[kB_DDFull]);
+                    }
                     // dS of keys [16kk, 16kk + 16) sits at column (kk / 2) * 32 +
                     // (kk % 2) * 8 of the buffer (each math half packs its 32 keys
                     // into the first 16 of its own 32 columns)
@@ -725,16 +738,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                         for (int kk = 0; kk < n / 16; ++kk)
                             umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
                                     kmn + kk * (2048 >> 4), id_dq, (i > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    if (!seq) {
-#pragma unroll
-                        for (int kk = 0; kk < BM / 16; ++kk) {
-                            umma_ss_elect(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
-                                    desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
-                            umma_ss_elect(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
-                                    desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit_elect(&bars[kB_DDFull]);
                     }
                     umma_commit_elect(&bars[kB_KVEmpty + st]);
                 }
@@ -767,13 +770,18 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         // so for each depth row the four warps of a half store 128 consecutive
         // d values (64 contiguous bytes per warp) straight to global memory;
         // the half takes depth rows [c0, c0 + 32) of the block.
-        auto depth_epilogue = [&](int jd) {
-            uint32_t xk[32], xv[32];
+        // The accumulators are read into registers (epi_load) before the next
+        // depth block's gradient MMAs may overwrite them, and written out
+        // (epi_store) after this thread's P-ready arrive, so the global stores
+        // are off the serial chain MMA -> read-out -> next block's MMA.
+        auto epi_load = [&](uint32_t* xk, uint32_t* xv) {
             tmem_ld32(lane_base + kColDKd + c0, xk);
             tmem_ld32(lane_base + kColDVd + c0, xv);
             tmem_wait_ld();
             reg_fence<32>(xk);
             reg_fence<32>(xv);
+        };
+        auto epi_store = [&](int jd, const uint32_t* xk, const uint32_t* xv) {
             if (r < D) {
                 const int row0 = jd * a.dep_rows + c0;
                 const int nvalid = min(a.dep_rows, dep_total - jd * a.dep_rows) - c0;
@@ -847,13 +855,14 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             // packed dS of keys [c0, c0 + 32) into columns [c0, c0 + 16): inside
             // this half's own score columns, which only it reads
             tmem_st16(lane_base + kColS + buf * 64 + c0, dsk);
+            uint32_t xk[32], xv[32];                      // depth gradients of block jd - 1
             if (!seq) {
                 // the previous depth block's MMAs are done before its staging
                 // tiles and TMEM columns are reused
                 if (jd >= 1) {
                     if (!mbar_wait(&bars[kB_DDFull], (jd - 1) & 1, a.status, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    depth_epilogue(jd - 1);
+                    epi_load(xk, xv);
                 }
                 // row r of the [q][depth] staging tiles, 128-byte swizzle;
                 // this half's depth columns are 16-byte chunks 4*half .. 4*half+3
@@ -866,16 +875,21 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                         make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
                 }
                 fence_proxy_async_smem();
-                ++jd;
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[kB_PReady + buf]);
+            if (!seq) {
+                if (jd >= 1) epi_store(jd - 1, xk, xv);
+                ++jd;
+            }
         }
         if (ok && n_dep > 0) {
             if (mbar_wait(&bars[kB_DDFull], (n_dep - 1) & 1, a.status, abort_flag)) {
                 tc_fence_after();
-                depth_epilogue(n_dep - 1);
+                uint32_t xk[32], xv[32];
+                epi_load(xk, xv);
+                epi_store(n_dep - 1, xk, xv);
             } else {
                 ok = false;
             }
