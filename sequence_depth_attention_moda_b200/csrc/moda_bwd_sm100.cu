@@ -49,7 +49,8 @@ constexpr int kThreads = 352;            // dq: warp 0 TMA, warps 1 and 6 MMA, w
 constexpr int kMathThreads = 256;
 constexpr int kKvMathWarps = 8;          // dkdv: warps 2..9, two per TMEM lane quarter
 constexpr int kKvGradWarp = 2 + kKvMathWarps;   // dkdv: issuer of dV and dK (warp 10)
-constexpr int kKvThreads = 32 * (kKvGradWarp + 1);
+constexpr int kKvStoreWarp0 = kKvGradWarp + 1;  // dkdv: warps 11..14 store dS (one per lane quarter)
+constexpr int kKvThreads = 32 * (kKvStoreWarp0 + 4);
 constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -106,7 +107,7 @@ struct DkdvArgs {
     int causal;
     float scale, scale_log2;
     // Stored dS (nullptr: not stored): the tiles the dq kernel reads instead
-    // of recomputing S and dP; see store_ds_tile.
+    // of recomputing S and dP; see store_ds_row.
     unsigned char* dS;
     int n_qt, n_kb, tq_log2;             // dq query tiles (Tq = 1 << tq_log2 tokens), 64-key blocks
 };
@@ -115,40 +116,34 @@ struct DkdvArgs {
 // for the 128 rows of dq query tile qt (row r = g * Tq + t - qt * Tq, as in the
 // forward's tile) and the 64 keys of key block kb, laid out byte for byte as
 // the dq kernel's shared-memory A operand, MN-major without swizzle: the 16
-// bytes of rows 8c .. 8c + 7 for key k at byte c * 1024 + k * 16.  A dK/dV
-// thread holds one key and 32 consecutive rows, so the 16 keys of a half warp
-// write 256 contiguous bytes per store.  Tiles are 16 KB, at
-// ((bh * n_qt + qt) * n_kb + kb) * 16 KB.
+// bytes of rows 8c .. 8c + 7 for key k at byte c * 1024 + k * 16.  The dK/dV
+// kernel's store warps hold one key row each (a warp: 32 consecutive keys),
+// so every store instruction writes 512 contiguous bytes.  Tiles are 16 KB,
+// at ((bh * n_qt + qt) * n_kb + kb) * 16 KB.
 constexpr uint32_t kDsTileBytes = 128 * 64 * 2;
 
-// One dkdv math thread's 32 dS values (16 packed bf16 pairs in dk: key `key`,
-// head g, tokens t_first .. t_first + 31) into their tiles.  Needs Tq >= 16
-// (a power of two): the 32 tokens fall in one or two query tiles, each piece
-// a run of whole 16-byte chunks.  Keys past T get zeros; tiles past the last
-// key block or query tile are skipped.
-__device__ __forceinline__ void store_ds_tile(const DkdvArgs& a, int bh, int g, int key, int t_first,
-                                              const uint32_t* dk) {
+// One key row's dS for the 64 queries of a query block (32 packed bf16 pairs
+// in v: head g, tokens t0 .. t0 + 63) into the tiles: 8 chunks of 8 tokens,
+// each inside one query tile (Tq >= 16 is a multiple of 8).  Keys past T get
+// zeros; tiles past the last key block or query tile are skipped.
+__device__ __forceinline__ void store_ds_row(const DkdvArgs& a, int bh, int g, int key, int t0,
+                                             const uint32_t* v) {
     const int kb = key >> 6, k = key & 63;
     if (kb >= a.n_kb) return;
     const bool live = key < a.T;
     const int Tq = 1 << a.tq_log2;
-    const int per = Tq < 32 ? Tq : 32;            // tokens of one piece (16 or 32)
 #pragma unroll
-    for (int pc = 0; pc < 2; ++pc) {
-        if (pc * per >= 32) break;
-        const int t = t_first + pc * per;
+    for (int j = 0; j < 8; ++j) {
+        const int t = t0 + 8 * j;
         const int qt = t >> a.tq_log2;
         if (qt >= a.n_qt) break;
-        const int r0 = g * Tq + (t - (qt << a.tq_log2));
-        unsigned char* base = a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + kb) * kDsTileBytes +
-                              (r0 >> 3) * 1024 + k * 16;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (i * 8 >= per) break;
-            const int e = pc * 8 + 4 * i;            // first packed pair of the chunk (pc > 0 only if per = 16)
-            const uint4 v = live ? make_uint4(dk[e], dk[e + 1], dk[e + 2], dk[e + 3]) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(base + i * 1024) = v;
-        }
+        const int r = g * Tq + (t - (qt << a.tq_log2));
+        unsigned char* dst = a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + kb) * kDsTileBytes +
+                             (r >> 3) * 1024 + k * 16;
+        // streaming store (evict first): the tiles are read once, by the dQ
+        // kernel, and must not push the Q / dO tiles this kernel re-reads out of L2
+        __stcs(reinterpret_cast<uint4*>(dst),
+               live ? make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]) : make_uint4(0, 0, 0, 0));
     }
 }
 
@@ -176,7 +171,8 @@ struct DkdvLayout {
 };
 
 enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 1 + kKvStages, kA_SFull = 1 + 2 * kKvStages,
-       kA_PReady = 3 + 2 * kKvStages, kA_Final = 5 + 2 * kKvStages, kA_NumBars = 6 + 2 * kKvStages };
+       kA_PReady = 3 + 2 * kKvStages, kA_Final = 5 + 2 * kKvStages, kA_DSRead = 6 + 2 * kKvStages,
+       kA_NumBars = 8 + 2 * kKvStages };
 
 template <int D>
 __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_constant__ DkdvArgs a) {
@@ -210,6 +206,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             mbar_init(&bars[kA_PReady + s], kKvMathWarps);   // one arrive per math warp
         }
         mbar_init(&bars[kA_Final], 1);
+        for (int s = 0; s < 2; ++s) mbar_init(&bars[kA_DSRead + s], 4);   // one arrive per store warp
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -341,6 +338,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + (it - 2) % kKvStages],
                                                                       ((it - 2) / kKvStages) & 1, a.status,
                                                                       abort_flag))) { ok = false; break; }
+                    // ... and, with stored dS, for the store warps to have read it
+                    if (it >= 2 && a.dS &&
+                        !__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSRead + (it & 1)], ((it - 2) >> 1) & 1,
+                                                           a.status, abort_flag))) { ok = false; break; }
                     if (!issue_s(it)) { ok = false; break; }
                 }
             } else {
@@ -361,6 +362,33 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     umma_commit_elect(&bars[kA_QEmpty + st]);
                 }
                 umma_commit_elect(&bars[kA_Final]);
+            }
+        }
+    } else if (warp >= kKvStoreWarp0) {
+        // Store warps (stored dS only): once the math warps have written an
+        // iteration's dS^T into TMEM (P-ready), each reads its lane quarter's
+        // 32 key rows x 64 packed queries, releases the buffer for the next
+        // score products (DSRead) and writes the rows into the dQ kernel's
+        // tiles -- off the math warps' path.
+        if (a.dS) {
+            const int quarter = warp & 3;
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            const int k = kt * BN + quarter * 32 + lane;
+            for (int it = 0; it < n_it; ++it) {
+                const int g = it / nqb;
+                const int qb = qb0 + (it - g * nqb);
+                const int buf = it & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status,
+                                                       abort_flag))) break;
+                tc_fence_after();
+                uint32_t v[32];
+                tmem_ld32(lane_base + 128 + buf * 64, v);
+                tmem_wait_ld();
+                reg_fence<32>(v);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kA_DSRead + buf]);
+                store_ds_row(a, bh, g, k, qb * kKvBQ, v);
             }
         }
     } else {
@@ -417,7 +445,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             __syncwarp();
             tmem_st16x2_16<16>(lane_base + buf * 64, pk);
             tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
-            if (a.dS) store_ds_tile(a, bh, g, k, tq0 + c0, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -477,7 +504,7 @@ struct DqArgs {
     int causal, win_lo;
     int band;                            // (b, KV head) pairs per band (banded_item)
     float scale, scale_log2;
-    const unsigned char* dS;             // stored dS tiles (store_ds_tile), kStored only
+    const unsigned char* dS;             // stored dS tiles (written by the dK/dV kernel), kStored only
     int n_kb;                            // 64-key blocks per head
 };
 
