@@ -78,6 +78,7 @@ struct FwdArgs {
     int win_lo;       // first visible depth row of a token
     int n_tiles;      // B * Hk * n_qt query tiles, longest first within a band of heads
     int band;         // (b, KV head) pairs per band (banded_item)
+    int tok_major;    // query tile rows token-major (r = t * G + g), else head-major (r = g * Tq + t)
     float scale_log2;
 };
 
@@ -214,9 +215,13 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     if (kt > 0 && !mbar_wait(&bars[kSFull + (j - 1) % kSBufs], ((j - 1) / kSBufs) & 1,
                                              a.status, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(&bars[kQFull], q_bytes);
-                    for (int s = 0; s < Lay::kSlabs; ++s)
-                        tma_load_3d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, T.t0,
-                                    T.b * a.Hq + T.hk * a.G);
+                    for (int s = 0; s < Lay::kSlabs; ++s) {
+                        if (a.tok_major)
+                            tma_load_4d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, 0, T.t0, T.bh);
+                        else
+                            tma_load_3d(sQ + s * kSlabBytes, &a.tq, &bars[kQFull], s * 64, T.t0,
+                                        T.b * a.Hq + T.hk * a.G);
+                    }
                     ++nq;
                 }
                 for (int i = 0; i < T.nb; ++i, ++j) {
@@ -352,7 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
         const int half = lane >> 4;                   // column half of the row
         const int r = quarter * 32 + sub * 16 + (lane & 15);   // tile row
         const bool row_real = r < R;
-        const int g = row_real ? r / a.Tq : 0;
+        // the row's head and token offset within the tile
+        const int g = row_real ? (a.tok_major ? r % a.G : r / a.Tq) : 0;
+        const int t_off = row_real ? (a.tok_major ? r / a.G : r - g * a.Tq) : 0;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
         const int c0 = half * 64;                     // first S column this thread holds
         const float sl2 = a.scale_log2;
@@ -363,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
             if (tile >= a.n_tiles) continue;
             const FwdTile T = fwd_tile(a, tile);
             const int t0 = T.t0, n_seq = T.n_seq, nb = T.nb;
-            const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
+            const int t_row = t0 + t_off;
             float m = -INFINITY, l = 0.0f;                // l: this half's share of the row sum
             for (int i = 0; i < nb; ++i) {
                 const int j = j0 + i;                     // running block count: ring phases
@@ -551,7 +558,20 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     a.LSE = LSE;
     a.status = device_status_word();
     cudaError_t e;
-    if ((e = make_tma_3d_bf16(&a.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, a.Tq, p.G)) != cudaSuccess) return e;
+    // Query tile token-major: a 4-D view of Q as (d, head g, token, b * Hk + hk)
+    // with byte strides (T * d * 2, d * 2, G * T * d * 2): the box (64, G, Tq, 1)
+    // lands as rows t * G + g.  Each warp's rows then cover few tokens, so
+    // most depth blocks hold none of a warp's visible depth rows and the
+    // warp skips them.  Head-major (a 3-D box) if the driver declines the view.
+    {
+        const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.G, (uint64_t)p.T, (uint64_t)p.B * p.Hk};
+        const uint64_t strides[3] = {(uint64_t)p.T * D * 2, (uint64_t)D * 2, (uint64_t)p.G * p.T * D * 2};
+        const uint32_t box[4] = {64, (uint32_t)p.G, (uint32_t)a.Tq, 1};
+        a.tok_major = make_tma_4d_bf16(&a.tq, Q, dims, strides, box) == cudaSuccess ? 1 : 0;
+    }
+    if (!a.tok_major &&
+        (e = make_tma_3d_bf16(&a.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, a.Tq, p.G)) != cudaSuccess)
+        return e;
     if ((e = make_tma_3d_bf16(&a.tk, K, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&a.tv, V, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
     if (p.L > 0) {

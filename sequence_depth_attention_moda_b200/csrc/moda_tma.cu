@@ -107,6 +107,24 @@ cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t
     return cudaSuccess;
 }
 
+cudaError_t make_tma_4d_bf16(TmaMap* out, const void* base, const uint64_t dims[4],
+                             const uint64_t strides_bytes[3], const uint32_t box[4]) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof(map));
+    const cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+    const cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+    const cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+    const cuuint32_t estride[4] = {1, 1, 1, 1};
+    CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gd, gs, bx,
+                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    std::memcpy(out->bytes, &map, sizeof(map));
+    return cudaSuccess;
+}
+
 cudaError_t set_max_dynamic_smem(const void* func, int bytes) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
