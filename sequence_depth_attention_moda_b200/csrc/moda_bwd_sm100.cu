@@ -20,11 +20,14 @@
 //              S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and dS^T written
 //              back to TMEM as bf16, then dV += P^T dO and dK += dS^T Q with
 //              the A operand read from TMEM.  The group's G heads are all
-//              iterated inside the CTA, so dK/dV are complete sums.
+//              iterated inside the CTA, so dK/dV are complete sums.  With the
+//              full workspace, store warps also write every dS^T row into
+//              the dq kernel's operand tiles (stored dS).
 //  3. dq:      one CTA per 128-row query tile (G heads x 128/G tokens, as in
-//              the forward).  S = Q K^T, dP = dO V^T, dQ += dS K over the
-//              causal sequence blocks and then the tile's depth blocks.  For
-//              a depth block, P' and dS' (bf16) are also staged in shared
+//              the forward).  Sequence blocks: dQ += dS K, dS either read
+//              from the stored tiles (no S, dP, exponentials) or recomputed
+//              from S = Q K^T and dP = dO V^T.  Depth blocks: S', dP' and
+//              dS' recomputed, P' and dS' (bf16) also staged in shared
 //              memory, and the token-local depth gradients come out as
 //              dKd^T = Q^T dS' and dVd^T = dO^T P' (M = d, N = depth rows):
 //              each depth row belongs to exactly one query tile, so these
