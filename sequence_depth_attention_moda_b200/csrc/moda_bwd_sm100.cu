@@ -173,9 +173,16 @@ struct DkdvLayout {
     static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
 };
 
+// Per S/dP buffer b (iteration it uses b = it & 1): SFull / DPFull (S^T /
+// dP^T products done), PReady / DSReady (P^T / dS^T written over them by the
+// math warps), SFree (dV product done: the S columns may be overwritten),
+// DSRead (store warps hold the dS^T rows).  The Q/dO stage release QEmpty
+// follows the dK product, the last reader of the stage and of dS^T.
 enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 1 + kKvStages, kA_SFull = 1 + 2 * kKvStages,
-       kA_PReady = 3 + 2 * kKvStages, kA_Final = 5 + 2 * kKvStages, kA_DSRead = 6 + 2 * kKvStages,
-       kA_NumBars = 8 + 2 * kKvStages };
+       kA_DPFull = 3 + 2 * kKvStages, kA_PReady = 5 + 2 * kKvStages, kA_DSReady = 7 + 2 * kKvStages,
+       kA_SFree = 9 + 2 * kKvStages, kA_Final = 11 + 2 * kKvStages, kA_DSRead = 12 + 2 * kKvStages,
+       kA_NumBars = 14 + 2 * kKvStages };
+static_assert(kA_NumBars * 8 + 8 <= 256, "dK/dV barriers, TMEM address and abort flag fit the barrier area");
 
 template <int D>
 __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_constant__ DkdvArgs a) {
@@ -206,7 +213,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[kA_SFull + s], 1);
+            mbar_init(&bars[kA_DPFull + s], 1);
             mbar_init(&bars[kA_PReady + s], kKvMathWarps);   // one arrive per math warp
+            mbar_init(&bars[kA_DSReady + s], kKvMathWarps);
+            mbar_init(&bars[kA_SFree + s], 1);
         }
         mbar_init(&bars[kA_Final], 1);
         for (int s = 0; s < 2; ++s) mbar_init(&bars[kA_DSRead + s], 4);   // one arrive per store warp
@@ -242,6 +252,21 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             }
         }
         const float inv_scale = 1.0f / a.scale;
+        // LSE and D of a query block are read one iteration ahead, so their
+        // global-load latency overlaps the wait for the stage to free up
+        float nl[2], nd[2];
+        auto fetch_stats = [&](int it) {
+            const int g = it / nqb;
+            const int qb = qb0 + (it - g * nqb);
+            const size_t qrow0 = static_cast<size_t>(b * a.Hq + hk * a.G + g) * a.T;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int t = qb * kKvBQ + lane + 32 * h2;
+                nl[h2] = t < a.T ? a.LSE[qrow0 + t] : INFINITY;   // rows past T: p = 0
+                nd[h2] = t < a.T ? a.Drow[qrow0 + t] : 0.0f;
+            }
+        };
+        if (n_it > 0) fetch_stats(0);
         int issued = 0;
         for (int it = 0; it < n_it; ++it) {
             const int st = it % kKvStages;
@@ -252,20 +277,17 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             const int g = it / nqb;
             const int qb = qb0 + (it - g * nqb);
             const int qh = b * a.Hq + hk * a.G + g;
+            float cl[2] = {nl[0], nl[1]}, cd[2] = {nd[0], nd[1]};
+            if (it + 1 < n_it) fetch_stats(it + 1);
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int rr = lane + 32 * h2;                 // query row of the block
-                const int t = qb * kKvBQ + rr;
-                const size_t qrow = static_cast<size_t>(qh) * a.T + t;
-                float lh = -INFINITY, ll = 0.0f, dh = 0.0f, dl = 0.0f;   // rows past T: p = 0
-                if (t < a.T) {
-                    const float bl = -a.LSE[qrow] * inv_scale;
-                    const float bd = -a.Drow[qrow];
-                    lh = __bfloat162float(__float2bfloat16_rn(bl));
-                    ll = bl - lh;
-                    dh = __bfloat162float(__float2bfloat16_rn(bd));
-                    dl = bd - dh;
-                }
+                const float bl = -cl[h2] * inv_scale;
+                const float bd = -cd[h2];
+                const float lh = __bfloat162float(__float2bfloat16_rn(bl));
+                const float ll = bl == -INFINITY ? 0.0f : bl - lh;
+                const float dh = __bfloat162float(__float2bfloat16_rn(bd));
+                const float dl = bd - dh;
                 const uint32_t o0 = rr * 128 + ((0 ^ (rr & 7)) << 4);
                 const uint32_t o1 = rr * 128 + ((1 ^ (rr & 7)) << 4);
                 unsigned char* al = smem + Lay::kAL + st * kKvSlab;
@@ -295,73 +317,85 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         }
     } else if (warp == 1 || warp == kKvGradWarp) {
         // Two issuers on different sub-partitions: warp 1 the score products
-        // S^T, dP^T, warp kKvGradWarp the gradient products dV, dK (issuing a
-        // tcgen05.mma costs its warp tens of cycles, more while math warps
-        // share the sub-partition).  Each runs converged: warp-uniform waits,
-        // one elected lane issues; a commit tracks only its own warp's MMAs.
+        // S^T, dP^T, warp kKvGradWarp the gradient products dV, dK.  Each runs
+        // converged: warp-uniform waits, one elected lane issues; a commit
+        // tracks only its own warp's MMAs.  The two halves of an iteration
+        // are chained separately -- S^T -> P^T -> dV and dP^T -> dS^T -> dK --
+        // so the math warps start on P while dP^T is still computing, and dV
+        // runs while they compute dS.
         {
             const uint32_t id_s = idesc_bf16(128, kKvBQ, false, false);
             const uint32_t id_g = idesc_bf16(128, D, false, true);
             const uint64_t kd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kK));
             const uint64_t vd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kV));
             const uint64_t ad0 = desc_kmajor_sw128(smem_u32(smem + Lay::kAA));
-            // S^T(j) = K Q_j^T - LSE/scale and dP^T(j) = V dO_j^T - D into buffer j & 1.
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % kKvStages;
-                const int buf = j & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_QFull + st], (j / kKvStages) & 1, a.status, abort_flag))) return false;
-                tc_fence_after();
-                const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
-                const uint64_t dd = desc_kmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile));
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
-                    const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                    umma_ss_elect(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
-                }
-                umma_ss_elect(tmem + buf * 64, ad0, desc_kmajor_sw128(smem_u32(smem + Lay::kAL + st * kKvSlab)),
-                              id_s, 1u);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
-                    const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                    umma_ss_elect(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
-                }
-                umma_ss_elect(tmem + 128 + buf * 64, ad0,
-                              desc_kmajor_sw128(smem_u32(smem + Lay::kAD + st * kKvSlab)), id_s, 1u);
-                umma_commit_elect(&bars[kA_SFull + buf]);
-                return true;
-            };
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag));
             if (warp == 1) {
-                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag));
-                for (int it = 0; ok && it < n_it; ++it) {
-                    // buffer it & 1 held P^T / dS^T of iteration it - 2, read by
-                    // its dV / dK products: wait for their completion (the
-                    // Q/dO-stage release of that iteration)
-                    if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + (it - 2) % kKvStages],
-                                                                      ((it - 2) / kKvStages) & 1, a.status,
-                                                                      abort_flag))) { ok = false; break; }
-                    // ... and, with stored dS, for the store warps to have read it
-                    if (it >= 2 && a.dS &&
-                        !__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSRead + (it & 1)], ((it - 2) >> 1) & 1,
-                                                           a.status, abort_flag))) { ok = false; break; }
-                    if (!issue_s(it)) { ok = false; break; }
-                }
-            } else {
-                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag));
                 for (int it = 0; ok && it < n_it; ++it) {
                     const int st = it % kKvStages;
                     const int buf = it & 1;
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_QFull + st], (it / kKvStages) & 1, a.status,
+                                                           abort_flag))) { ok = false; break; }
+                    // S^T(it) = K Q^T - LSE/scale into the S columns of buffer
+                    // buf, which held P^T(it-2): its dV product must be done
+                    if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFree + buf], ((it - 2) >> 1) & 1,
+                                                                      a.status, abort_flag))) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
+                    const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
+                    const uint64_t dd = desc_kmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile));
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                        const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
+                        umma_ss_elect(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_ss_elect(tmem + buf * 64, ad0, desc_kmajor_sw128(smem_u32(smem + Lay::kAL + st * kKvSlab)),
+                                  id_s, 1u);
+                    umma_commit_elect(&bars[kA_SFull + buf]);
+                    // dP^T(it) = V dO^T - D over dS^T(it-2): its dK product must be
+                    // done (the stage release of it-2) and, with stored dS, the
+                    // store warps must have read it
+                    if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + (it - 2) % kKvStages],
+                                                                      ((it - 2) / kKvStages) & 1, a.status,
+                                                                      abort_flag))) { ok = false; break; }
+                    if (it >= 2 && a.dS &&
+                        !__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSRead + buf], ((it - 2) >> 1) & 1,
+                                                           a.status, abort_flag))) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                        const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
+                        umma_ss_elect(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_ss_elect(tmem + 128 + buf * 64, ad0,
+                                  desc_kmajor_sw128(smem_u32(smem + Lay::kAD + st * kKvSlab)), id_s, 1u);
+                    umma_commit_elect(&bars[kA_DPFull + buf]);
+                }
+            } else {
+                for (int it = 0; ok && it < n_it; ++it) {
+                    const int st = it % kKvStages;
+                    const int buf = it & 1;
+                    const uint32_t acc0 = it > 0 ? 1u : 0u;
+                    // dV += P^T dO (A: P^T from TMEM), then release the S columns
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status,
+                                                           abort_flag))) { ok = false; break; }
+                    tc_fence_after();
                     const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
 #pragma unroll
-                    for (int kk = 0; kk < kKvBQ / 16; ++kk) {
-                        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                        umma_ts_elect(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, acc);
-                        umma_ts_elect(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g, acc);
-                    }
+                    for (int kk = 0; kk < kKvBQ / 16; ++kk)
+                        umma_ts_elect(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g,
+                                      kk > 0 ? 1u : acc0);
+                    umma_commit_elect(&bars[kA_SFree + buf]);
+                    // dK += dS^T Q, then release the Q/dO stage (and dS^T)
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSReady + buf], (it >> 1) & 1, a.status,
+                                                           abort_flag))) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
+#pragma unroll
+                    for (int kk = 0; kk < kKvBQ / 16; ++kk)
+                        umma_ts_elect(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g,
+                                      kk > 0 ? 1u : acc0);
                     umma_commit_elect(&bars[kA_QEmpty + st]);
                 }
                 umma_commit_elect(&bars[kA_Final]);
@@ -369,7 +403,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         }
     } else if (warp >= kKvStoreWarp0) {
         // Store warps (stored dS only): once the math warps have written an
-        // iteration's dS^T into TMEM (P-ready), each reads its lane quarter's
+        // iteration's dS^T into TMEM (DSReady), each reads its lane quarter's
         // 32 key rows x 64 packed queries, releases the buffer for the next
         // score products (DSRead) and writes the rows into the dQ kernel's
         // tiles -- off the math warps' path.
@@ -381,7 +415,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 const int g = it / nqb;
                 const int qb = qb0 + (it - g * nqb);
                 const int buf = it & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status,
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSReady + buf], (it >> 1) & 1, a.status,
                                                        abort_flag))) break;
                 tc_fence_after();
                 uint32_t v[32];
@@ -408,9 +442,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         const float sl2 = a.scale_log2;
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
-            const int g = it / nqb;
-            const int qb = qb0 + (it - g * nqb);
+            const int qb = qb0 + it % nqb;
             const int buf = it & 1;
+            // P^T = 2^(scale*log2(e) * (s - LSE/scale)) once S^T is in
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status,
                                                    abort_flag))) { ok = false; break; }
             tc_fence_after();
@@ -418,40 +452,45 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             const bool diag = a.causal && tq0 < kt * BN + BN;   // some key after some query
             uint32_t s[32], dp[32], pk[16], dk[16];
             tmem_ld16x2_32<32>(lane_base + buf * 64, s);          // s - LSE/scale
-            tmem_ld16x2_32<32>(lane_base + 128 + buf * 64, dp);   // dP - D
             tmem_wait_ld();
             reg_fence<32>(s);
-            reg_fence<32>(dp);
             if (!diag) {                   // every column visible (CTA-uniform branch)
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float p0 = ex2(__uint_as_float(s[e]) * sl2);
-                    const float p1 = ex2(__uint_as_float(s[e + 1]) * sl2);
-                    pk[e / 2] = pack_bf16(p0, p1);
-                    dk[e / 2] = pack_bf16(p0 * __uint_as_float(dp[e]), p1 * __uint_as_float(dp[e + 1]));
-                }
+                for (int e = 0; e < 32; ++e) s[e] = __float_as_uint(ex2(__uint_as_float(s[e]) * sl2));
             } else {
                 // visible columns c >= k - tq0; a select, no branch per element
                 // (masked: score -inf, so P = dS = 0)
                 const int vlo = k - tq0 - c0;
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float s0 = e >= vlo ? __uint_as_float(s[e]) : -INFINITY;
-                    const float s1 = e + 1 >= vlo ? __uint_as_float(s[e + 1]) : -INFINITY;
-                    const float p0 = ex2(s0 * sl2);
-                    const float p1 = ex2(s1 * sl2);
-                    pk[e / 2] = pack_bf16(p0, p1);
-                    dk[e / 2] = pack_bf16(p0 * __uint_as_float(dp[e]), p1 * __uint_as_float(dp[e + 1]));
-                }
+                for (int e = 0; e < 32; ++e)
+                    s[e] = __float_as_uint(ex2((e >= vlo ? __uint_as_float(s[e]) : -INFINITY) * sl2));
             }
-            // P^T and dS^T (bf16 pairs) over the columns this warp has read
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) pk[e / 2] = pack_bf16(__uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+            // P^T (bf16 pairs) over the S columns this warp has read
             __syncwarp();
             tmem_st16x2_16<16>(lane_base + buf * 64, pk);
-            tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kA_PReady + buf]);
+            // dS^T = P^T * (dP^T - D) once dP^T is in
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DPFull + buf], (it >> 1) & 1, a.status,
+                                                   abort_flag))) { ok = false; break; }
+            tc_fence_after();
+            tmem_ld16x2_32<32>(lane_base + 128 + buf * 64, dp);   // dP - D
+            tmem_wait_ld();
+            reg_fence<32>(dp);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2)
+                dk[e / 2] = pack_bf16(__uint_as_float(s[e]) * __uint_as_float(dp[e]),
+                                      __uint_as_float(s[e + 1]) * __uint_as_float(dp[e + 1]));
+            __syncwarp();
+            tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kA_DSReady + buf]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_Final], 0, a.status, abort_flag));
         if (ok) {
