@@ -151,8 +151,16 @@ __device__ __forceinline__ void store_ds_row(const DkdvArgs& a, int bh, int g, i
 }
 
 constexpr int kKvBQ = 64;               // query rows per iteration
-constexpr int kKvStages = 3;            // Q/dO ring depth
+constexpr int kKvStages = 4;            // Q/dO ring depth
 constexpr uint32_t kKvSlab = 64 * 128;
+// Bias tiles: K = 16 (one MMA step), K-major without swizzle.  Core matrices
+// of 8 rows x 16 bytes; element (row r, k) at (r / 8) * 256 + (k / 8) * 128 +
+// (r % 8) * 16 + (k % 8) * 2, so the K-adjacent core matrix is 128 B further
+// and the next 8-row group 256 B further.
+constexpr uint32_t kBiasLbo = 128, kBiasSbo = 256;
+__host__ __device__ constexpr uint32_t bias_chunk(int r, int c) {   // 16-byte chunk c (k = 8c .. 8c + 7) of row r
+    return (r >> 3) * kBiasSbo + c * kBiasLbo + (r & 7) * 16;
+}
 
 template <int D>
 struct DkdvLayout {
@@ -163,12 +171,12 @@ struct DkdvLayout {
     static constexpr uint32_t kV = kKTile;
     static constexpr uint32_t kQ = 2 * kKTile;                  // kKvStages stages
     static constexpr uint32_t kDO = kQ + kKvStages * kQTile;    // kKvStages stages
-    // bias rows of each stage (64 query rows x 128 B, 128-byte swizzle; only
-    // the first 32 B of a row are read): LSE / scale, then D
+    // bias tiles of each stage (64 query rows x K = 16): LSE / scale, then D
+    static constexpr uint32_t kBiasQ = 64 * 32;
     static constexpr uint32_t kAL = kDO + kKvStages * kQTile;
-    static constexpr uint32_t kAD = kAL + kKvStages * kKvSlab;
-    static constexpr uint32_t kAA = kAD + kKvStages * kKvSlab;  // key-side (1, 1, 0, ...) rows, 128 x 128 B
-    static constexpr uint32_t kBar = kAA + kSlabBytes;
+    static constexpr uint32_t kAD = kAL + kKvStages * kBiasQ;
+    static constexpr uint32_t kAA = kAD + kKvStages * kBiasQ;   // key-side (1, 1, 0, ...) rows, 128 x K = 16
+    static constexpr uint32_t kBar = kAA + 128 * 32;
     static constexpr uint32_t kBytes = kBar + 256;
     static constexpr uint32_t kDynSmem = kBytes + 1024 > 120u * 1024 ? kBytes + 1024 : 120u * 1024;
 };
@@ -223,12 +231,16 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    // key-side bias rows: elements 0 and 1 are 1.0, the rest of the first 32 B
-    // zero (16-byte chunks c = 0, 1 of row r sit at chunk c ^ (r & 7))
+    // key-side bias rows: elements 0 and 1 are 1.0, the rest zero; in the
+    // query-side tiles the second chunk (k = 8 .. 15) of every row stays zero
     for (int i = threadIdx.x; i < 2 * BN; i += kKvThreads) {
         const int r = i >> 1, c = i & 1;
-        *reinterpret_cast<uint4*>(smem + Lay::kAA + r * 128 + ((c ^ (r & 7)) << 4)) =
+        *reinterpret_cast<uint4*>(smem + Lay::kAA + bias_chunk(r, c)) =
             c == 0 ? make_uint4(pack_bf16(1.0f, 1.0f), 0u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int i = threadIdx.x; i < 2 * kKvStages * kKvBQ; i += kKvThreads) {
+        const int r = i % kKvBQ, t = i / kKvBQ;          // t: tile (AL, AD of each stage)
+        *reinterpret_cast<uint4*>(smem + Lay::kAL + t * Lay::kBiasQ + bias_chunk(r, 1)) = make_uint4(0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
     if (warp == 1) {
@@ -288,14 +300,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 const float ll = bl == -INFINITY ? 0.0f : bl - lh;
                 const float dh = __bfloat162float(__float2bfloat16_rn(bd));
                 const float dl = bd - dh;
-                const uint32_t o0 = rr * 128 + ((0 ^ (rr & 7)) << 4);
-                const uint32_t o1 = rr * 128 + ((1 ^ (rr & 7)) << 4);
-                unsigned char* al = smem + Lay::kAL + st * kKvSlab;
-                unsigned char* ad = smem + Lay::kAD + st * kKvSlab;
-                *reinterpret_cast<uint4*>(al + o0) = make_uint4(pack_bf16(lh, ll), 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(al + o1) = make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(ad + o0) = make_uint4(pack_bf16(dh, dl), 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(ad + o1) = make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t o0 = bias_chunk(rr, 0);
+                *reinterpret_cast<uint4*>(smem + Lay::kAL + st * Lay::kBiasQ + o0) = make_uint4(pack_bf16(lh, ll), 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(smem + Lay::kAD + st * Lay::kBiasQ + o0) = make_uint4(pack_bf16(dh, dl), 0u, 0u, 0u);
             }
             fence_proxy_async_smem();   // generic writes -> the tensor core's reads
             __syncwarp();
@@ -317,29 +324,33 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         }
     } else if (warp == 1 || warp == kKvGradWarp) {
         // Two issuers on different sub-partitions: warp 1 the score products
-        // S^T, dP^T, warp kKvGradWarp the gradient products dV, dK.  Each runs
-        // converged: warp-uniform waits, one elected lane issues; a commit
-        // tracks only its own warp's MMAs.  The two halves of an iteration
-        // are chained separately -- S^T -> P^T -> dV and dP^T -> dS^T -> dK --
-        // so the math warps start on P while dP^T is still computing, and dV
-        // runs while they compute dS.
-        {
+        // S^T, dP^T, warp kKvGradWarp the gradient products dV, dK.  One
+        // elected thread of each runs the loop; a commit tracks only its own
+        // thread's MMAs.  The two halves of an iteration are chained
+        // separately -- S^T -> P^T -> dV and dP^T -> dS^T -> dK -- so the math
+        // warps start on P while dP^T is still computing, and dV runs while
+        // they compute dS.
+        if (elect_one()) {
             const uint32_t id_s = idesc_bf16(128, kKvBQ, false, false);
             const uint32_t id_g = idesc_bf16(128, D, false, true);
             const uint64_t kd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kK));
             const uint64_t vd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kV));
-            const uint64_t ad0 = desc_kmajor_sw128(smem_u32(smem + Lay::kAA));
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag));
+            const uint64_t ad0 = desc_noswizzle(smem_u32(smem + Lay::kAA), kBiasLbo, kBiasSbo);
+            bool ok = mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
             if (warp == 1) {
                 for (int it = 0; ok && it < n_it; ++it) {
                     const int st = it % kKvStages;
                     const int buf = it & 1;
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_QFull + st], (it / kKvStages) & 1, a.status,
-                                                           abort_flag))) { ok = false; break; }
+                    if (!mbar_wait(&bars[kA_QFull + st], (it / kKvStages) & 1, a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     // S^T(it) = K Q^T - LSE/scale into the S columns of buffer
                     // buf, which held P^T(it-2): its dV product must be done
-                    if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFree + buf], ((it - 2) >> 1) & 1,
-                                                                      a.status, abort_flag))) { ok = false; break; }
+                    if (it >= 2 && !mbar_wait(&bars[kA_SFree + buf], ((it - 2) >> 1) & 1, a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
                     const uint64_t dd = desc_kmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile));
@@ -347,30 +358,34 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                         const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                        umma_ss_elect(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
+                        umma_ss(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
                     }
-                    umma_ss_elect(tmem + buf * 64, ad0, desc_kmajor_sw128(smem_u32(smem + Lay::kAL + st * kKvSlab)),
-                                  id_s, 1u);
-                    umma_commit_elect(&bars[kA_SFull + buf]);
+                    umma_ss(tmem + buf * 64, ad0,
+                            desc_noswizzle(smem_u32(smem + Lay::kAL + st * Lay::kBiasQ), kBiasLbo, kBiasSbo), id_s, 1u);
+                    umma_commit(&bars[kA_SFull + buf]);
                     // dP^T(it) = V dO^T - D over dS^T(it-2): its dK product must be
                     // done (the stage release of it-2) and, with stored dS, the
                     // store warps must have read it
-                    if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + (it - 2) % kKvStages],
-                                                                      ((it - 2) / kKvStages) & 1, a.status,
-                                                                      abort_flag))) { ok = false; break; }
+                    if (it >= 2 && !mbar_wait(&bars[kA_QEmpty + (it - 2) % kKvStages], ((it - 2) / kKvStages) & 1,
+                                              a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     if (it >= 2 && a.dS &&
-                        !__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSRead + buf], ((it - 2) >> 1) & 1,
-                                                           a.status, abort_flag))) { ok = false; break; }
+                        !mbar_wait(&bars[kA_DSRead + buf], ((it - 2) >> 1) & 1, a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                         const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                        umma_ss_elect(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
+                        umma_ss(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
                     }
-                    umma_ss_elect(tmem + 128 + buf * 64, ad0,
-                                  desc_kmajor_sw128(smem_u32(smem + Lay::kAD + st * kKvSlab)), id_s, 1u);
-                    umma_commit_elect(&bars[kA_DPFull + buf]);
+                    umma_ss(tmem + 128 + buf * 64, ad0,
+                            desc_noswizzle(smem_u32(smem + Lay::kAD + st * Lay::kBiasQ), kBiasLbo, kBiasSbo), id_s, 1u);
+                    umma_commit(&bars[kA_DPFull + buf]);
                 }
             } else {
                 for (int it = 0; ok && it < n_it; ++it) {
@@ -378,29 +393,33 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                     const int buf = it & 1;
                     const uint32_t acc0 = it > 0 ? 1u : 0u;
                     // dV += P^T dO (A: P^T from TMEM), then release the S columns
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status,
-                                                           abort_flag))) { ok = false; break; }
+                    if (!mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
 #pragma unroll
                     for (int kk = 0; kk < kKvBQ / 16; ++kk)
-                        umma_ts_elect(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g,
-                                      kk > 0 ? 1u : acc0);
-                    umma_commit_elect(&bars[kA_SFree + buf]);
+                        umma_ts(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, kk > 0 ? 1u : acc0);
+                    umma_commit(&bars[kA_SFree + buf]);
                     // dK += dS^T Q, then release the Q/dO stage (and dS^T)
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSReady + buf], (it >> 1) & 1, a.status,
-                                                           abort_flag))) { ok = false; break; }
+                    if (!mbar_wait(&bars[kA_DSReady + buf], (it >> 1) & 1, a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
 #pragma unroll
                     for (int kk = 0; kk < kKvBQ / 16; ++kk)
-                        umma_ts_elect(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g,
-                                      kk > 0 ? 1u : acc0);
-                    umma_commit_elect(&bars[kA_QEmpty + st]);
+                        umma_ts(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g,
+                                kk > 0 ? 1u : acc0);
+                    umma_commit(&bars[kA_QEmpty + st]);
                 }
-                umma_commit_elect(&bars[kA_Final]);
+                umma_commit(&bars[kA_Final]);
             }
         }
+        __syncwarp();
     } else if (warp >= kKvStoreWarp0) {
         // Store warps (stored dS only): once the math warps have written an
         // iteration's dS^T into TMEM (DSReady), each reads its lane quarter's

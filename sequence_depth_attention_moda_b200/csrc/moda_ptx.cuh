@@ -198,6 +198,21 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
         : "memory");
 }
 
+// True in exactly one lane of a converged warp (elect.sync).  An MMA issuer
+// runs its whole loop -- barrier waits, MMAs, commits -- in that one thread:
+// a wait on a completed barrier and an MMA issue cost about half as much as
+// their warp-collective forms below, and the issue path sits between the
+// tensor pipe's batches.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t e;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(e));
+    return e != 0;
+}
+
 // Warp-collective issue: every lane of a converged warp calls these with the
 // same (warp-uniform) operands; elect.sync picks the one lane that issues.
 __device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -380,6 +395,13 @@ __device__ __forceinline__ uint64_t desc_mnmajor_noswizzle(uint32_t saddr, uint3
     desc |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     desc |= static_cast<uint64_t>(1u) << 46;                // descriptor version; swizzle 0 = none
     return desc;
+}
+
+// Either major-ness without swizzle (the instruction descriptor says which):
+// core matrices of 8 rows x 16 bytes, the next one along K lbo_bytes further,
+// the next 8-row group along M/N sbo_bytes further.
+__device__ __forceinline__ uint64_t desc_noswizzle(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return desc_mnmajor_noswizzle(saddr, lbo_bytes, sbo_bytes);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
