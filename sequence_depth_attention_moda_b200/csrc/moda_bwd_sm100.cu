@@ -724,10 +724,10 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         // ------------------------------------------------------ MMA issuers -
         // Two warps on different sub-partitions share the issue work: warp 6
         // the score products S(j), dP(j); warp 1 dQ(i) and the depth
-        // gradients.  Each runs converged (warp-uniform waits, one elected
-        // lane issues); a commit tracks only its own warp's MMAs, and the
-        // waits below order every TMEM reuse across the two.
-        {
+        // gradients.  One elected thread of each runs the loop; a commit
+        // tracks only its own thread's MMAs, and the waits below order every
+        // TMEM reuse across the two.
+        if (elect_one()) {
             const uint32_t id_seq = idesc_bf16(128, kDqBN, false, false);
             const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
             const uint32_t id_dq = idesc_bf16(128, D, false, true);
@@ -742,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             auto issue_s = [&](int j) -> bool {
                 const int st = j % kDqStages;
                 const int buf = j & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag))) return false;
+                if (!mbar_wait(&bars[kB_KVFull + st], (j / kDqStages) & 1, a.status, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t id = is_dep(j) ? id_dep : id_seq;
                 const uint64_t kd = desc_kmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile));
@@ -751,27 +751,29 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t offq = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                     const uint64_t offk = ((kk >> 2) * kDqSlab + (kk & 3) * 32) >> 4;
-                    umma_ss_elect(tmem + kColS + buf * 64, qd0 + offq, kd + offk, id, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + kColS + buf * 64, qd0 + offq, kd + offk, id, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t offq = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
                     const uint64_t offk = ((kk >> 2) * kDqSlab + (kk & 3) * 32) >> 4;
-                    umma_ss_elect(tmem + kColDP + buf * 64, dod0 + offq, vd + offk, id, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + kColDP + buf * 64, dod0 + offq, vd + offk, id, kk > 0 ? 1u : 0u);
                 }
-                umma_commit_elect(&bars[kB_SFull + buf]);
+                umma_commit(&bars[kB_SFull + buf]);
                 return true;
             };
             if (warp == 6) {
                 // kStored: only the depth blocks (blocks 0 .. n_dep-1) need S and dP
                 const int n_sdp = kStored ? n_dep : nb;
-                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag));
+                bool ok = mbar_wait(&bars[kB_QFull], 0, a.status, abort_flag);
                 for (int j = 0; ok && j < n_sdp; ++j) {
                     // buffer j & 1 last held dS(j-2), which dQ(j-2) reads: wait
                     // until that has completed (its K/V-stage release)
-                    if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVEmpty + (j - 2) % kDqStages],
-                                                                     ((j - 2) / kDqStages) & 1, a.status,
-                                                                     abort_flag))) { ok = false; break; }
+                    if (j >= 2 && !mbar_wait(&bars[kB_KVEmpty + (j - 2) % kDqStages], ((j - 2) / kDqStages) & 1,
+                                             a.status, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     if (!issue_s(j)) { ok = false; break; }
                 }
             } else {
@@ -785,20 +787,22 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                         // dQ += dS K: A = the dS tile in the V slot (MN-major,
                         // no swizzle: 8 keys 128 B apart, 8 rows 1024 B apart; 16
                         // keys = 256 B per K step), B = the K tile, MN-major
-                        if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_KVFull + st], (i / kDqStages) & 1,
-                                                               a.status, abort_flag))) { ok = false; break; }
+                        if (!mbar_wait(&bars[kB_KVFull + st], (i / kDqStages) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after();
                         const uint32_t a_addr = smem_u32(smem + Lay::kV + st * Lay::kKTile);
                         const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
 #pragma unroll
                         for (int kk = 0; kk < kDqBN / 16; ++kk)
-                            umma_ss_elect(tmem + kColDQ, desc_mnmajor_noswizzle(a_addr + kk * 256, 128, 1024),
-                                          kmn + kk * (2048 >> 4), id_dqs, (i > 0 || kk > 0) ? 1u : 0u);
-                        umma_commit_elect(&bars[kB_KVEmpty + st]);
+                            umma_ss(tmem + kColDQ, desc_mnmajor_noswizzle(a_addr + kk * 256, 128, 1024),
+                                    kmn + kk * (2048 >> 4), id_dqs, (i > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&bars[kB_KVEmpty + st]);
                         continue;
                     }
                     const int n = seq ? kDqBN : a.dep_rows;
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag))) { ok = false; break; }
+                    if (!mbar_wait(&bars[kB_PReady + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
                     // depth block: the gradient products first, so their
@@ -807,12 +811,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     if (!seq) {
 #pragma unroll
                         for (int kk = 0; kk < BM / 16; ++kk) {
-                            umma_ss_elect(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
+                            umma_ss(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
                                     desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
-                            umma_ss_elect(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
+                            umma_ss(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
                                     desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
                         }
-                        umma_commit_elect(&bars[kB_DDFull]);
+                        umma_commit(&bars[kB_DDFull]);
                     }
                     // dS of keys [16kk, 16kk + 16) sits at column (kk / 2) * 32 +
                     // (kk % 2) * 8 of the buffer (each math half packs its 32 keys
@@ -820,18 +824,19 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     if (n == kDqBN) {
 #pragma unroll
                         for (int kk = 0; kk < kDqBN / 16; ++kk)
-                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+                            umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
                                     kmn + kk * (2048 >> 4), id_dq, (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
                         for (int kk = 0; kk < n / 16; ++kk)
-                            umma_ts_elect(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+                            umma_ts(tmem + kColDQ, tmem + kColS + buf * 64 + (kk >> 1) * 32 + (kk & 1) * 8,
                                     kmn + kk * (2048 >> 4), id_dq, (i > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit_elect(&bars[kB_KVEmpty + st]);
+                    umma_commit(&bars[kB_KVEmpty + st]);
                 }
-                umma_commit_elect(&bars[kB_Final]);
+                umma_commit(&bars[kB_Final]);
             }
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------------ math --------
         // Warps 2..5 and 7..10: two per TMEM lane quarter (they share its

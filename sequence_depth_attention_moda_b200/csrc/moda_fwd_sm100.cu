@@ -256,100 +256,100 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
     } else if (warp == 1 || warp == kSWarp) {
         // ------------------------------------------------------ MMA issuers -
         // Two warps issue: warp kSWarp the score products S(j), warp 1 the
-        // PV(j) products.  Issuing a tcgen05.mma costs its warp tens of
-        // cycles, and every wait and commit more while a softmax warp shares
-        // the sub-partition; one warp issuing both products was the forward's
-        // bound, so the two streams now run on two sub-partitions.  Each warp
-        // runs its loop converged (warp-uniform waits, elect.sync picks the
-        // issuing lane); a commit tracks only its own warp's MMAs.
-        const uint32_t id_seq = idesc_bf16(128, BN, false, false);
-        const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
-        const uint32_t id_pv = idesc_bf16(128, D, false, true);
-        // Descriptors are built once; a K step adds its byte offset / 16 to
-        // the 14-bit address field (shared addresses stay < 256 KB).
-        const uint64_t qd0 = desc_kmajor_sw128(smem_u32(sQ));
-        // S(j) = Q K_j^T into buffer j % 3 (i: the block's index in its tile).
-        // The buffer last held P(j-3), read by PV(j-3): the caller waits for
-        // that product's completion (its V-stage release) first.
-        auto issue_s = [&](int j, int i, const FwdTile& T) -> bool {
-            const int st = j % kKStages;
-            const int sb = j % kSBufs;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kKFull + st], (j / kKStages) & 1, a.status,
-                                                   abort_flag))) return false;
-            tc_fence_after();
-            const uint64_t kd0 = desc_kmajor_sw128(smem_u32(sK + st * Lay::kTile));
-            const uint32_t id = i < T.n_seq ? id_seq : id_dep;
+        // PV(j) products, on two sub-partitions.  One elected thread of each
+        // runs the whole loop (waits, MMAs, commits): an MMA issue blocks until
+        // the tensor pipe takes it, so the issue path's own cost is pipe idle
+        // time, and single-thread waits and issues cost about half of the
+        // warp-collective forms.  A commit tracks only its own thread's MMAs.
+        if (elect_one()) {
+            const uint32_t id_seq = idesc_bf16(128, BN, false, false);
+            const uint32_t id_dep = idesc_bf16(128, a.dep_rows, false, false);
+            const uint32_t id_pv = idesc_bf16(128, D, false, true);
+            // Descriptors are built once; a K step adds its byte offset / 16 to
+            // the 14-bit address field (shared addresses stay < 256 KB).
+            const uint64_t qd0 = desc_kmajor_sw128(smem_u32(sQ));
+            // S(j) = Q K_j^T into buffer j % 3 (i: the block's index in its tile).
+            // The buffer last held P(j-3), read by PV(j-3): the caller waits for
+            // that product's completion (its V-stage release) first.
+            auto issue_s = [&](int j, int i, const FwdTile& T) -> bool {
+                const int st = j % kKStages;
+                const int sb = j % kSBufs;
+                if (!mbar_wait(&bars[kKFull + st], (j / kKStages) & 1, a.status, abort_flag)) return false;
+                tc_fence_after();
+                const uint64_t kd0 = desc_kmajor_sw128(smem_u32(sK + st * Lay::kTile));
+                const uint32_t id = i < T.n_seq ? id_seq : id_dep;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t off = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
-                umma_ss_elect(tmem + sb * 128, qd0 + off, kd0 + off, id, kk > 0 ? 1u : 0u);
-            }
-            umma_commit_elect(&bars[kSFull + sb]);
-            return true;
-        };
-        // O += P(j) V_j with P read from TMEM buffer j % 3; the tile's first
-        // block overwrites O.
-        auto issue_pv = [&](int j, int i, const FwdTile& T) -> bool {
-            const int st = j % kVStages;
-            const int sb = j % kSBufs;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kPReady + sb], (j / kSBufs) & 1, a.status,
-                                                   abort_flag))) return false;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status,
-                                                   abort_flag))) return false;
-            tc_fence_after();
-            const int krows = i < T.n_seq ? BN : a.dep_rows;
-            const uint64_t vd0 = desc_mnmajor_sw128(smem_u32(sV + st * Lay::kTile), kSlabBytes);
-            if (krows == BN) {
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_ts_elect(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
-                                  (i > 0 || kk > 0) ? 1u : 0u);
-            } else {
-                for (int kk = 0; kk < krows / 16; ++kk)
-                    umma_ts_elect(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
-                                  (i > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit_elect(&bars[kVEmpty + st]);
-            return true;
-        };
-        // The score issuer runs up to three blocks ahead of the PV issuer
-        // (three S buffers), so two score tiles are ready before the softmax
-        // needs them.
-        bool ok = true;
-        int j0 = 0, kt = 0;
-        const bool s_role = warp == kSWarp;
-        for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
-            const int tile = tile_of(rnd);
-            if (tile >= a.n_tiles) continue;
-            const FwdTile T = fwd_tile(a, tile);
-            if (s_role) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], kt & 1, a.status, abort_flag));
-                for (int i = 0; ok && i < T.nb; ++i) {
-                    const int j = j0 + i;
-                    // buffer j % 3 held P(j-3): PV(j-3) must have completed
-                    if (j >= kSBufs &&
-                        !__all_sync(0xffffffffu, mbar_wait(&bars[kVEmpty + (j - kSBufs) % kVStages],
-                                                           ((j - kSBufs) / kVStages) & 1, a.status,
-                                                           abort_flag))) { ok = false; break; }
-                    if (!issue_s(j, i, T)) { ok = false; break; }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + sb * 128, qd0 + off, kd0 + off, id, kk > 0 ? 1u : 0u);
                 }
-            } else {
-                for (int i = 0; ok && i < T.nb; ++i) {
-                    // the tile's first PV overwrites O: the softmax warps must
-                    // have read the previous tile's O out
-                    if (i == 0 && kt > 0 &&
-                        !__all_sync(0xffffffffu, mbar_wait(&bars[kOFree], (kt - 1) & 1, a.status, abort_flag))) {
-                        ok = false;
-                        break;
+                umma_commit(&bars[kSFull + sb]);
+                return true;
+            };
+            // O += P(j) V_j with P read from TMEM buffer j % 3; the tile's first
+            // block overwrites O.
+            auto issue_pv = [&](int j, int i, const FwdTile& T) -> bool {
+                const int st = j % kVStages;
+                const int sb = j % kSBufs;
+                if (!mbar_wait(&bars[kPReady + sb], (j / kSBufs) & 1, a.status, abort_flag)) return false;
+                if (!mbar_wait(&bars[kVFull + st], (j / kVStages) & 1, a.status, abort_flag)) return false;
+                tc_fence_after();
+                const int krows = i < T.n_seq ? BN : a.dep_rows;
+                const uint64_t vd0 = desc_mnmajor_sw128(smem_u32(sV + st * Lay::kTile), kSlabBytes);
+                if (krows == BN) {
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
+                                (i > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    for (int kk = 0; kk < krows / 16; ++kk)
+                        umma_ts(tmem + kColO, tmem + sb * 128 + kk * 8, vd0 + kk * (2048 >> 4), id_pv,
+                                (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&bars[kVEmpty + st]);
+                return true;
+            };
+            // The score issuer runs up to three blocks ahead of the PV issuer
+            // (three S buffers), so two score tiles are ready before the softmax
+            // needs them.
+            bool ok = true;
+            int j0 = 0, kt = 0;
+            const bool s_role = warp == kSWarp;
+            for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+                const int tile = tile_of(rnd);
+                if (tile >= a.n_tiles) continue;
+                const FwdTile T = fwd_tile(a, tile);
+                if (s_role) {
+                    ok = mbar_wait(&bars[kQFull], kt & 1, a.status, abort_flag);
+                    for (int i = 0; ok && i < T.nb; ++i) {
+                        const int j = j0 + i;
+                        // buffer j % 3 held P(j-3): PV(j-3) must have completed
+                        if (j >= kSBufs && !mbar_wait(&bars[kVEmpty + (j - kSBufs) % kVStages],
+                                                      ((j - kSBufs) / kVStages) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!issue_s(j, i, T)) { ok = false; break; }
                     }
-                    if (i == 0) tc_fence_after();
-                    if (!issue_pv(j0 + i, i, T)) { ok = false; break; }
+                } else {
+                    for (int i = 0; ok && i < T.nb; ++i) {
+                        // the tile's first PV overwrites O: the softmax warps must
+                        // have read the previous tile's O out
+                        if (i == 0 && kt > 0 &&
+                            !mbar_wait(&bars[kOFree], (kt - 1) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (i == 0) tc_fence_after();
+                        if (!issue_pv(j0 + i, i, T)) { ok = false; break; }
+                    }
+                    umma_commit(&bars[kOFinal]);
                 }
-                umma_commit_elect(&bars[kOFinal]);
+                j0 += T.nb;
+                ++kt;
             }
-            j0 += T.nb;
-            ++kt;
         }
+        __syncwarp();
     } else if (warp >= 2 && warp < 2 + kSoftmaxWarps) {
         // ------------------------------------------------------ softmax -----
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
