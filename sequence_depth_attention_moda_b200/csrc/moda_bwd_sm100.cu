@@ -807,14 +807,34 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     const uint64_t kmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kK + st * Lay::kKTile), kDqSlab);
                     // depth block: the gradient products first, so their
                     // completion (which the math warps wait for before the next
-                    // depth block) does not queue behind this block's dQ
+                    // depth block) does not queue behind this block's dQ.  Their
+                    // K dimension is the tile's query rows, and P', dS' are zero
+                    // outside the rows of the block's own tokens (each query
+                    // row sees only its own token's depth rows), so only the
+                    // 16-row K steps that hold such rows are issued.
                     if (!seq) {
+                        const int r0 = dep_idx(i) * a.dep_rows;
+                        const int tok_lo = r0 / a.L;
+                        const int tok_hi = (min(r0 + a.dep_rows, dep_total) - 1) / a.L;
+                        uint32_t steps = 0xffu;
+                        if (a.G <= 8) {
+                            steps = 0;
+                            for (int g = 0, base = 0; g < a.G && base < R; ++g, base += a.Tq) {
+                                const int s0 = (base + tok_lo) >> 4;
+                                const int s1 = min(base + tok_hi, R - 1) >> 4;
+                                steps |= ((2u << s1) - 1u) & ~((1u << s0) - 1u);
+                            }
+                            if (steps == 0) steps = 1;   // (cannot happen) keep the accumulators defined
+                        }
+                        uint32_t acc = 0;
 #pragma unroll
                         for (int kk = 0; kk < BM / 16; ++kk) {
+                            if (!((steps >> kk) & 1u)) continue;
                             umma_ss(tmem + kColDKd, desc_mnmajor_sw128(q_addr + kk * 2048, kSlabBytes),
-                                    desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                                    desc_mnmajor_sw128(ds_addr + kk * 2048, kSlabBytes), id_dd, acc);
                             umma_ss(tmem + kColDVd, desc_mnmajor_sw128(do_addr + kk * 2048, kSlabBytes),
-                                    desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, kk > 0 ? 1u : 0u);
+                                    desc_mnmajor_sw128(p_addr + kk * 2048, kSlabBytes), id_dd, acc);
+                            acc = 1;
                         }
                         umma_commit(&bars[kB_DDFull]);
                     }
