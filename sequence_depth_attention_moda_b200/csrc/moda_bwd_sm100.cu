@@ -22,11 +22,14 @@
 //              the A operand read from TMEM.  The group's G heads are all
 //              iterated inside the CTA, so dK/dV are complete sums.  With the
 //              full workspace, store warps also write every dS^T row into
-//              the dq kernel's operand tiles (stored dS).
+//              the dq kernel's operand tiles (stored dS); the query blocks
+//              are then token-major (64 / G tokens of all G heads, row
+//              t * G + g), the dq tile's row order.
 //  3. dq:      one CTA per 128-row query tile (G heads x 128/G tokens, as in
-//              the forward).  Sequence blocks: dQ += dS K, dS either read
-//              from the stored tiles (no S, dP, exponentials) or recomputed
-//              from S = Q K^T and dP = dO V^T.  Depth blocks: S', dP' and
+//              the forward; token-major rows with stored dS).  Sequence
+//              blocks: dQ += dS K, dS either read from the stored tiles (no
+//              S, dP, exponentials) or recomputed from S = Q K^T and
+//              dP = dO V^T.  Depth blocks: S', dP' and
 //              dS' recomputed, P' and dS' (bf16) also staged in shared
 //              memory, and the token-local depth gradients come out as
 //              dKd^T = Q^T dS' and dVd^T = dO^T P' (M = d, N = depth rows):
@@ -113,11 +116,16 @@ struct DkdvArgs {
     // of recomputing S and dP; see store_ds_row.
     unsigned char* dS;
     int n_qt, n_kb, tq_log2;             // dq query tiles (Tq = 1 << tq_log2 tokens), 64-key blocks
+    // Token-major query blocks (kTok, with stored dS): block i holds tokens
+    // [i * TB, (i + 1) * TB), TB = 64 / G = 1 << tb_log2, of all G heads, row
+    // t * G + g (tq / tdo are 4-D head-strided maps); otherwise the blocks are
+    // 64 tokens of one head, head by head.
+    int tb_log2, g_log2, n_tb;
 };
 
 // Stored dS tiles.  Tile (bh, qt, kb) holds dS = P * (dP - D) (unscaled, bf16)
-// for the 128 rows of dq query tile qt (row r = g * Tq + t - qt * Tq, as in the
-// forward's tile) and the 64 keys of key block kb, laid out byte for byte as
+// for the 128 rows of dq query tile qt (token-major: row r = (t - qt * Tq) * G
+// + g, as in the forward's tile) and the 64 keys of key block kb, laid out byte for byte as
 // the dq kernel's shared-memory A operand, MN-major without swizzle: the 16
 // bytes of rows 8c .. 8c + 7 for key k at byte c * 1024 + k * 16.  The dK/dV
 // kernel's store warps hold one key row each (a warp: 32 consecutive keys),
@@ -125,27 +133,24 @@ struct DkdvArgs {
 // at ((bh * n_qt + qt) * n_kb + kb) * 16 KB.
 constexpr uint32_t kDsTileBytes = 128 * 64 * 2;
 
-// One key row's dS for the 64 queries of a query block (32 packed bf16 pairs
-// in v: head g, tokens t0 .. t0 + 63) into the tiles: 8 chunks of 8 tokens,
-// each inside one query tile (Tq >= 16 is a multiple of 8).  Keys past T get
-// zeros; tiles past the last key block or query tile are skipped.
-__device__ __forceinline__ void store_ds_row(const DkdvArgs& a, int bh, int g, int key, int t0,
-                                             const uint32_t* v) {
+// One key row's dS for the 64 rows of a token-major query block (32 packed
+// bf16 pairs in v: tokens t0 .. t0 + TB - 1 of all G heads, row t * G + g)
+// into the tiles: the block is 64 consecutive rows of one dq query tile (TB
+// divides Tq), so its 8 chunks of 8 rows go to 8 consecutive 1 KB row groups
+// of that tile.  Keys past T get zeros; key blocks past the last are skipped.
+__device__ __forceinline__ void store_ds_row(const DkdvArgs& a, int bh, int key, int t0, const uint32_t* v) {
     const int kb = key >> 6, k = key & 63;
     if (kb >= a.n_kb) return;
     const bool live = key < a.T;
-    const int Tq = 1 << a.tq_log2;
+    const int qt = t0 >> a.tq_log2;
+    const int r0 = (t0 - (qt << a.tq_log2)) << a.g_log2;   // first row of the block in the tile
+    unsigned char* dst = a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + kb) * kDsTileBytes +
+                         (r0 >> 3) * 1024 + k * 16;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const int t = t0 + 8 * j;
-        const int qt = t >> a.tq_log2;
-        if (qt >= a.n_qt) break;
-        const int r = g * Tq + (t - (qt << a.tq_log2));
-        unsigned char* dst = a.dS + (static_cast<size_t>(bh * a.n_qt + qt) * a.n_kb + kb) * kDsTileBytes +
-                             (r >> 3) * 1024 + k * 16;
         // streaming store (evict first): the tiles are read once, by the dQ
         // kernel, and must not push the Q / dO tiles this kernel re-reads out of L2
-        __stcs(reinterpret_cast<uint4*>(dst),
+        __stcs(reinterpret_cast<uint4*>(dst + j * 1024),
                live ? make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]) : make_uint4(0, 0, 0, 0));
     }
 }
@@ -192,7 +197,8 @@ enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 1 + kKvStages, kA_SFull = 1 + 2 
        kA_NumBars = 14 + 2 * kKvStages };
 static_assert(kA_NumBars * 8 + 8 <= 256, "dK/dV barriers, TMEM address and abort flag fit the barrier area");
 
-template <int D>
+// kTok: token-major query blocks (the stored-dS backward), see DkdvArgs.
+template <int D, bool kTok>
 __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_constant__ DkdvArgs a) {
     using Lay = DkdvLayout<D>;
     extern __shared__ unsigned char smem_raw[];
@@ -209,9 +215,22 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
     banded_item(static_cast<int>(blockIdx.x), a.n_kt, nbh, a.band, &kt, &bh);
     const int b = bh / a.Hk;
     const int hk = bh - b * a.Hk;
-    const int qb0 = a.causal ? kt * (BN / kKvBQ) : 0;      // first query block that sees the keys
+    // Iteration it -> query block: its first token tq0 and, head by head, its
+    // head g (token-major blocks hold all G heads).  Causal: the first block
+    // that sees the key tile is the one holding token kt * BN.
+    const int qb0 = a.causal ? kt * (BN / kKvBQ) : 0;
     const int nqb = a.n_qb - qb0;
-    const int n_it = a.G * nqb;
+    const int tb0 = a.causal ? (kt * BN) >> a.tb_log2 : 0;
+    const int n_it = kTok ? a.n_tb - tb0 : a.G * nqb;
+    auto block_of = [&](int it, int* g, int* tq0) {
+        if (kTok) {
+            *g = 0;
+            *tq0 = (tb0 + it) << a.tb_log2;
+        } else {
+            *g = it / nqb;
+            *tq0 = (qb0 + it - *g * nqb) * kKvBQ;
+        }
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[kA_KVFull], 1);
@@ -268,14 +287,16 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         // global-load latency overlaps the wait for the stage to free up
         float nl[2], nd[2];
         auto fetch_stats = [&](int it) {
-            const int g = it / nqb;
-            const int qb = qb0 + (it - g * nqb);
-            const size_t qrow0 = static_cast<size_t>(b * a.Hq + hk * a.G + g) * a.T;
+            int g, tq0;
+            block_of(it, &g, &tq0);
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
-                const int t = qb * kKvBQ + lane + 32 * h2;
-                nl[h2] = t < a.T ? a.LSE[qrow0 + t] : INFINITY;   // rows past T: p = 0
-                nd[h2] = t < a.T ? a.Drow[qrow0 + t] : 0.0f;
+                const int rr = lane + 32 * h2;                 // row of the block
+                const int gr = kTok ? (rr & (a.G - 1)) : g;
+                const int t = tq0 + (kTok ? rr >> a.g_log2 : rr);
+                const size_t qrow = static_cast<size_t>(b * a.Hq + hk * a.G + gr) * a.T + t;
+                nl[h2] = t < a.T ? a.LSE[qrow] : INFINITY;     // rows past T: p = 0
+                nd[h2] = t < a.T ? a.Drow[qrow] : 0.0f;
             }
         };
         if (n_it > 0) fetch_stats(0);
@@ -286,9 +307,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + st], ((it / kKvStages) - 1) & 1,
                                                    a.status, abort_flag)))
                 break;
-            const int g = it / nqb;
-            const int qb = qb0 + (it - g * nqb);
-            const int qh = b * a.Hq + hk * a.G + g;
+            int g, tq0;
+            block_of(it, &g, &tq0);
             float cl[2] = {nl[0], nl[1]}, cd[2] = {nd[0], nd[1]};
             if (it + 1 < n_it) fetch_stats(it + 1);
 #pragma unroll
@@ -309,10 +329,16 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[kA_QFull + st], 2 * Lay::kQTile);
                 for (int s = 0; s < Lay::kSlabs; ++s) {
-                    tma_load_3d(smem + Lay::kQ + st * Lay::kQTile + s * kKvSlab, &a.tq,
-                                &bars[kA_QFull + st], s * 64, qb * kKvBQ, qh);
-                    tma_load_3d(smem + Lay::kDO + st * Lay::kQTile + s * kKvSlab, &a.tdo,
-                                &bars[kA_QFull + st], s * 64, qb * kKvBQ, qh);
+                    unsigned char* dq_ = smem + Lay::kQ + st * Lay::kQTile + s * kKvSlab;
+                    unsigned char* ddo = smem + Lay::kDO + st * Lay::kQTile + s * kKvSlab;
+                    if (kTok) {   // box (64, G, TB, 1): rows t * G + g
+                        tma_load_4d(dq_, &a.tq, &bars[kA_QFull + st], s * 64, 0, tq0, bh);
+                        tma_load_4d(ddo, &a.tdo, &bars[kA_QFull + st], s * 64, 0, tq0, bh);
+                    } else {
+                        const int qh = b * a.Hq + hk * a.G + g;
+                        tma_load_3d(dq_, &a.tq, &bars[kA_QFull + st], s * 64, tq0, qh);
+                        tma_load_3d(ddo, &a.tdo, &bars[kA_QFull + st], s * 64, tq0, qh);
+                    }
                 }
             }
             issued = it + 1;
@@ -431,8 +457,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
             const int k = kt * BN + quarter * 32 + lane;
             for (int it = 0; it < n_it; ++it) {
-                const int g = it / nqb;
-                const int qb = qb0 + (it - g * nqb);
+                int g, tq0;
+                block_of(it, &g, &tq0);
                 const int buf = it & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSReady + buf], (it >> 1) & 1, a.status,
                                                        abort_flag))) break;
@@ -444,7 +470,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[kA_DSRead + buf]);
-                store_ds_row(a, bh, g, k, qb * kKvBQ, v);
+                store_ds_row(a, bh, k, tq0, v);
             }
         }
     } else {
@@ -461,13 +487,13 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         const float sl2 = a.scale_log2;
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
-            const int qb = qb0 + it % nqb;
+            int g, tq0;
+            block_of(it, &g, &tq0);
             const int buf = it & 1;
             // P^T = 2^(scale*log2(e) * (s - LSE/scale)) once S^T is in
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status,
                                                    abort_flag))) { ok = false; break; }
             tc_fence_after();
-            const int tq0 = qb * kKvBQ;
             const bool diag = a.causal && tq0 < kt * BN + BN;   // some key after some query
             uint32_t s[32], dp[32], pk[16], dk[16];
             tmem_ld16x2_32<32>(lane_base + buf * 64, s);          // s - LSE/scale
@@ -477,9 +503,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
 #pragma unroll
                 for (int e = 0; e < 32; ++e) s[e] = __float_as_uint(ex2(__uint_as_float(s[e]) * sl2));
             } else {
-                // visible columns c >= k - tq0; a select, no branch per element
-                // (masked: score -inf, so P = dS = 0)
-                const int vlo = k - tq0 - c0;
+                // visible columns: token >= k, i.e. c >= k - tq0 (head by head)
+                // or c >= (k - tq0) * G (token-major); a select, no branch per
+                // element (masked: score -inf, so P = dS = 0)
+                const int vlo = (kTok ? (k - tq0) * a.G : k - tq0) - c0;
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
                     s[e] = __float_as_uint(ex2((e >= vlo ? __uint_as_float(s[e]) : -INFINITY) * sl2));
@@ -567,6 +594,7 @@ struct DqArgs {
     float scale, scale_log2;
     const unsigned char* dS;             // stored dS tiles (written by the dK/dV kernel), kStored only
     int n_kb;                            // 64-key blocks per head
+    int g_log2;                          // kStored: G = 1 << g_log2
 };
 
 constexpr int kDqBN = 64;            // rows per key / depth block
@@ -675,8 +703,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             const uint64_t once = policy_evict_first();
             mbar_arrive_expect_tx(&bars[kB_QFull], 2 * q_bytes);
             for (int s = 0; s < Lay::kSlabs; ++s) {
-                tma_load_3d(smem + Lay::kQ + s * kSlabBytes, &a.tq, &bars[kB_QFull], s * 64, t0, b * a.Hq + hk * a.G);
-                tma_load_3d(smem + Lay::kDO + s * kSlabBytes, &a.tdo, &bars[kB_QFull], s * 64, t0, b * a.Hq + hk * a.G);
+                if (kStored) {   // token-major: box (64, G, Tq, 1) lands as rows t * G + g
+                    tma_load_4d(smem + Lay::kQ + s * kSlabBytes, &a.tq, &bars[kB_QFull], s * 64, 0, t0, bh);
+                    tma_load_4d(smem + Lay::kDO + s * kSlabBytes, &a.tdo, &bars[kB_QFull], s * 64, 0, t0, bh);
+                } else {
+                    tma_load_3d(smem + Lay::kQ + s * kSlabBytes, &a.tq, &bars[kB_QFull], s * 64, t0, b * a.Hq + hk * a.G);
+                    tma_load_3d(smem + Lay::kDO + s * kSlabBytes, &a.tdo, &bars[kB_QFull], s * 64, t0, b * a.Hq + hk * a.G);
+                }
             }
             int issued = 0;
             for (int i = 0; i < nb; ++i) {
@@ -817,7 +850,11 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                         const int tok_lo = r0 / a.L;
                         const int tok_hi = (min(r0 + a.dep_rows, dep_total) - 1) / a.L;
                         uint32_t steps = 0xffu;
-                        if (a.G <= 8) {
+                        if (kStored) {       // token-major: rows [tok_lo * G, (tok_hi + 1) * G)
+                            const int s0 = (tok_lo << a.g_log2) >> 4;
+                            const int s1 = (min((tok_hi + 1) << a.g_log2, R) - 1) >> 4;
+                            steps = ((2u << s1) - 1u) & ~((1u << s0) - 1u);
+                        } else if (a.G <= 8) {
                             steps = 0;
                             for (int g = 0, base = 0; g < a.G && base < R; ++g, base += a.Tq) {
                                 const int s0 = (base + tok_lo) >> 4;
@@ -861,14 +898,17 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         // ------------------------------------------------------ math --------
         // Warps 2..5 and 7..10: two per TMEM lane quarter (they share its
         // sub-partition and interleave).  Thread = query row r; the warp's
-        // half takes columns [c0, c0 + 32) of every 64-row block.
+        // half takes columns [c0, c0 + 32) of every 64-row block.  Rows are
+        // token-major with stored dS (r = t * G + g: a warp's 32 rows are
+        // 32 / G tokens, so most depth blocks hold none of its rows' depth
+        // rows and the warp skips them), head by head otherwise (r = g * Tq + t).
         const int quarter = warp & 3;
         const int half = warp >= 7 ? 1 : 0;
         const int c0 = 32 * half;
         const int r = quarter * 32 + lane;
         const bool row_real = r < R;
-        const int g = row_real ? r / a.Tq : 0;
-        const int t_row = row_real ? t0 + (r - g * a.Tq) : t0;
+        const int g = row_real ? (kStored ? r & (a.G - 1) : r / a.Tq) : 0;
+        const int t_row = row_real ? t0 + (kStored ? r >> a.g_log2 : r - g * a.Tq) : t0;
         const bool row_live = row_real && t_row < a.T;
         const size_t qrow = (static_cast<size_t>(b) * a.Hq + hk * a.G + g) * a.T + t_row;
         const float lse2 = row_live ? a.LSE[qrow] * kLog2e : INFINITY;
@@ -919,11 +959,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             if (!mbar_wait(&bars[kB_SFull + buf], (i >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t s[32], dp[32], dsk[16], pk[16];
-            tmem_ld32(lane_base + kColS + buf * 64 + c0, s);
-            tmem_ld32(lane_base + kColDP + buf * 64 + c0, dp);
-            tmem_wait_ld();
-            reg_fence<32>(s);
-            reg_fence<32>(dp);
             int lo = 0, hi = kDqBN, kb = 0;
             const int lim = a.causal ? t_row : a.T - 1;   // last visible sequence key
             if (seq) {
@@ -933,10 +968,25 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 lo = base + a.win_lo;
                 hi = min(base + a.L, a.dep_rows);
             }
+            // A depth block none of the warp's rows can see in its half of the
+            // columns (token-major rows): P' and dS' are exactly 0 there, written
+            // without loading or exponentiating.
+            const bool skip = kStored && !seq &&
+                              __all_sync(0xffffffffu, !row_live || max(lo, c0) >= min(hi, c0 + 32));
             const bool all_visible = seq && kb + c0 + 31 <= lim;
+            if (!skip) {
+                tmem_ld32(lane_base + kColS + buf * 64 + c0, s);
+                tmem_ld32(lane_base + kColDP + buf * 64 + c0, dp);
+                tmem_wait_ld();
+                reg_fence<32>(s);
+                reg_fence<32>(dp);
+            }
             // Masked entries get score -inf and dP 0 by selects (no branch per
             // element), so exp2 runs unconditionally and yields exactly 0.
-            if (all_visible) {
+            if (skip) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dsk[e] = pk[e] = 0u;
+            } else if (all_visible) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const float p0 = ex2(fmaf(__uint_as_float(s[e]), sl2, -lse2));
@@ -1057,9 +1107,24 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     cudaError_t e;
     float* Dws = static_cast<float*>(ws);
     const size_t ds_bytes = bwd_ds_bytes(p);
-    const bool stored = ds_bytes > 0 && ws_bytes >= bwd_workspace_bytes(p) + ds_bytes;
-    unsigned char* ds_tiles = stored ? static_cast<unsigned char*>(ws) + bwd_workspace_bytes(p) : nullptr;
+    bool stored = ds_bytes > 0 && ws_bytes >= bwd_workspace_bytes(p) + ds_bytes;
     const int Tq = BM / p.G;
+    // Stored dS runs both kernels on token-major query rows: Q and dO as
+    // (d, head g, token, b * Hk + hk) with byte strides (T * d * 2, d * 2,
+    // G * T * d * 2), whose boxes (64, G, tokens, 1) land as rows t * G + g.
+    // If the driver declines these views, the backward recomputes dS instead.
+    TmaMap q_kv, do_kv, q_dq, do_dq;
+    if (stored) {
+        const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.G, (uint64_t)p.T, (uint64_t)p.B * p.Hk};
+        const uint64_t strides[3] = {(uint64_t)p.T * D * 2, (uint64_t)D * 2, (uint64_t)p.G * p.T * D * 2};
+        const uint32_t box_kv[4] = {64, (uint32_t)p.G, (uint32_t)(kKvBQ / p.G), 1};
+        const uint32_t box_dq[4] = {64, (uint32_t)p.G, (uint32_t)Tq, 1};
+        stored = make_tma_4d_bf16(&q_kv, Q, dims, strides, box_kv) == cudaSuccess &&
+                 make_tma_4d_bf16(&do_kv, dO, dims, strides, box_kv) == cudaSuccess &&
+                 make_tma_4d_bf16(&q_dq, Q, dims, strides, box_dq) == cudaSuccess &&
+                 make_tma_4d_bf16(&do_dq, dO, dims, strides, box_dq) == cudaSuccess;
+    }
+    unsigned char* ds_tiles = stored ? static_cast<unsigned char*>(ws) + bwd_workspace_bytes(p) : nullptr;
     const int n_qt = (p.T + Tq - 1) / Tq;
     const int n_kb = (p.T + kDqBN - 1) / kDqBN;
     // 1. D = rowsum(dO * O)
@@ -1086,16 +1151,28 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     A.n_qt = n_qt;
     A.n_kb = n_kb;
     A.tq_log2 = stored ? log2_exact(Tq) : 0;
+    A.g_log2 = stored ? log2_exact(p.G) : 0;
+    A.tb_log2 = stored ? 6 - A.g_log2 : 0;
+    A.n_tb = stored ? (p.T + (1 << A.tb_log2) - 1) >> A.tb_log2 : 0;
     if ((e = make_tma_3d_bf16(&A.tk, K, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&A.tv, V, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
-    if ((e = make_tma_3d_bf16(&A.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
-    if ((e = make_tma_3d_bf16(&A.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
+    if (stored) {
+        A.tq = q_kv;
+        A.tdo = do_kv;
+    } else {
+        if ((e = make_tma_3d_bf16(&A.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
+        if ((e = make_tma_3d_bf16(&A.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, kKvBQ, 1)) != cudaSuccess) return e;
+    }
     {
         const uint32_t smem = DkdvLayout<D>::kDynSmem;
-        if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dkdv_kernel<D>), (int)smem)) != cudaSuccess)
-            return e;
+        const void* fn = stored ? reinterpret_cast<const void*>(dkdv_kernel<D, true>)
+                                : reinterpret_cast<const void*>(dkdv_kernel<D, false>);
+        if ((e = set_max_dynamic_smem(fn, (int)smem)) != cudaSuccess) return e;
         const long long grid = (long long)p.B * p.Hk * A.n_kt;
-        dkdv_kernel<D><<<(unsigned)grid, kKvThreads, smem, stream>>>(A);
+        if (stored)
+            dkdv_kernel<D, true><<<(unsigned)grid, kKvThreads, smem, stream>>>(A);
+        else
+            dkdv_kernel<D, false><<<(unsigned)grid, kKvThreads, smem, stream>>>(A);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         phase_mark(2, stream);
     }
@@ -1118,8 +1195,14 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     B.band = l2_band(p.B * p.Hk, 2.0 * p.T * D * 2);          // K and V of one head
     B.dS = ds_tiles;
     B.n_kb = n_kb;
-    if ((e = make_tma_3d_bf16(&B.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
-    if ((e = make_tma_3d_bf16(&B.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
+    B.g_log2 = stored ? log2_exact(p.G) : 0;
+    if (stored) {
+        B.tq = q_dq;
+        B.tdo = do_dq;
+    } else {
+        if ((e = make_tma_3d_bf16(&B.tq, Q, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
+        if ((e = make_tma_3d_bf16(&B.tdo, dO, D, p.T, (uint64_t)p.B * p.Hq, B.Tq, p.G)) != cudaSuccess) return e;
+    }
     if ((e = make_tma_3d_bf16(&B.tk, K, D, p.T, (uint64_t)p.B * p.Hk, kDqBN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&B.tv, V, D, p.T, (uint64_t)p.B * p.Hk, kDqBN, 1)) != cudaSuccess) return e;
     if (p.L > 0) {
