@@ -162,9 +162,12 @@ moda_status moda_fwd(const moda_shape* shape,
  *   dQ, dK, dV, dKd, dVd   outputs (fully overwritten; dKd/dVd may be NULL if L = 0)
  *   ws, ws_bytes      workspace: at least moda_workspace_size(shape, 2) bytes;
  *                     with moda_workspace_size(shape, 1) bytes or more the
- *                     faster stored-dS path runs (the two paths round dS the
- *                     same way but compute it in different kernels, so their
- *                     results may differ in the last bits)
+ *                     faster stored-dS path runs (on token-major query rows,
+ *                     read through a head-strided tensor-map view of Q and dO;
+ *                     if the driver declines that view, the recomputing path
+ *                     runs instead).  The two paths round dS the same way but
+ *                     compute it in different kernels, so their results may
+ *                     differ in the last bits.
  * Deterministic: no floating-point atomics; repeated calls with the same
  * ws_bytes give identical bits.
  */
