@@ -208,6 +208,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kA_NumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
+    // The dQ kernel may start on SMs this grid has left: its depth blocks
+    // need nothing from this kernel, and it waits for this grid's completion
+    // before its first stored dS tile.
+    griddep_launch_dependents();
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nbh = a.B * a.Hk;
@@ -717,6 +721,10 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 if (i >= kDqStages &&
                     !mbar_wait(&bars[kB_KVEmpty + st], ((i / kDqStages) - 1) & 1, a.status, abort_flag))
                     break;
+                // this kernel may have started before the dK/dV kernel ended
+                // (programmatic dependent launch): the stored dS tiles are
+                // read only after that grid has completed
+                if (kStored && i == n_dep) griddep_wait();
                 unsigned char* dk = smem + Lay::kK + st * Lay::kKTile;
                 unsigned char* dv = smem + Lay::kV + st * Lay::kKTile;
                 const bool seq = !is_dep(i);
@@ -1086,12 +1094,32 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    // never complete before the dK/dV kernel (this one may have started early)
+    if (threadIdx.x == 0) griddep_wait();
 }
 
 // The stored-dS backward: d = 128, G in {1, 2, 4, 8} (Tq = 128 / G >= 16, a
 // power of two, so a dK/dV thread's 32 queries fall in whole chunks of one or
 // two dq tiles), and at most this many bytes of tiles.
 constexpr double kMaxStoredDsBytes = 16.0 * 1024 * 1024 * 1024;
+
+// Launch with programmatic stream serialization: the kernel may start before
+// the previous kernel in the stream has completed (see griddep_wait).
+template <typename Args>
+cudaError_t launch_dependent(void (*kernel)(Args), unsigned grid, unsigned threads, uint32_t smem,
+                             cudaStream_t stream, const Args& args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args);
+}
 
 int log2_exact(int x) {
     int l = 0;
@@ -1222,7 +1250,9 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
                 if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dq_kernel<D, true>), (int)smem)) !=
                     cudaSuccess)
                     return e;
-                dq_kernel<D, true><<<(unsigned)grid, kThreads, smem, stream>>>(B);
+                if ((e = launch_dependent(dq_kernel<D, true>, (unsigned)grid, kThreads, smem, stream, B)) !=
+                    cudaSuccess)
+                    return e;
                 launched = true;
             }
         }
@@ -1230,7 +1260,9 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
             if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(dq_kernel<D, false>), (int)smem)) !=
                 cudaSuccess)
                 return e;
-            dq_kernel<D, false><<<(unsigned)grid, kThreads, smem, stream>>>(B);
+            if ((e = launch_dependent(dq_kernel<D, false>, (unsigned)grid, kThreads, smem, stream, B)) !=
+                cudaSuccess)
+                return e;
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         phase_mark(3, stream);

@@ -133,6 +133,15 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
         : "memory");
 }
 
+// Programmatic dependent launch.  launch_dependents: this CTA lets a kernel
+// launched after it with programmatic stream serialization start; wait: until
+// the grid this kernel depends on has completed and its memory operations are
+// visible.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // L2 policy for data read exactly once (the depth tiles): its lines are the
 // first to be evicted, so streaming it does not push out the K/V tiles that
 // other query tiles read again.
