@@ -121,6 +121,7 @@ struct DkdvArgs {
     // t * G + g (tq / tdo are 4-D head-strided maps); otherwise the blocks are
     // 64 tokens of one head, head by head.
     int tb_log2, g_log2, n_tb;
+    int n_items, persist;                // key tiles; persist: CTAs walk several (snake_tile)
 };
 
 // Stored dS tiles.  Tile (bh, qt, kb) holds dS = P * (dP - D) (unscaled, bf16)
@@ -194,7 +195,7 @@ struct DkdvLayout {
 enum { kA_KVFull = 0, kA_QFull = 1, kA_QEmpty = 1 + kKvStages, kA_SFull = 1 + 2 * kKvStages,
        kA_DPFull = 3 + 2 * kKvStages, kA_PReady = 5 + 2 * kKvStages, kA_DSReady = 7 + 2 * kKvStages,
        kA_SFree = 9 + 2 * kKvStages, kA_Final = 11 + 2 * kKvStages, kA_DSRead = 12 + 2 * kKvStages,
-       kA_NumBars = 14 + 2 * kKvStages };
+       kA_AccFree = 14 + 2 * kKvStages, kA_NumBars = 15 + 2 * kKvStages };
 static_assert(kA_NumBars * 8 + 8 <= 256, "dK/dV barriers, TMEM address and abort flag fit the barrier area");
 
 // kTok: token-major query blocks (the stored-dS backward), see DkdvArgs.
@@ -215,24 +216,42 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nbh = a.B * a.Hk;
-    int kt, bh;                                             // small kt = most work: first
-    banded_item(static_cast<int>(blockIdx.x), a.n_kt, nbh, a.band, &kt, &bh);
-    const int b = bh / a.Hk;
-    const int hk = bh - b * a.Hk;
-    // Iteration it -> query block: its first token tq0 and, head by head, its
-    // head g (token-major blocks hold all G heads).  Causal: the first block
-    // that sees the key tile is the one holding token kt * BN.
-    const int qb0 = a.causal ? kt * (BN / kKvBQ) : 0;
-    const int nqb = a.n_qb - qb0;
-    const int tb0 = a.causal ? (kt * BN) >> a.tb_log2 : 0;
-    const int n_it = kTok ? a.n_tb - tb0 : a.G * nqb;
-    auto block_of = [&](int it, int* g, int* tq0) {
+    // Work items: key tiles (b * Hk + hk, kt), the longest (small kt) first
+    // within bands of heads (banded_item).  A persistent launch deals them to
+    // its CTAs in a snake over rounds of gridDim.x items (snake_tile);
+    // otherwise CTA c takes item c.  Every role walks the same items and keeps
+    // a running iteration count for ring stages, TMEM buffers and barrier
+    // phases; the next item's K/V load and first score products overlap the
+    // previous item's dK/dV read-out.
+    const int n_ctas = static_cast<int>(gridDim.x);
+    const int n_rounds = a.persist ? (a.n_items + n_ctas - 1) / n_ctas : 1;
+    auto item_of = [&](int rnd) {
+        return a.persist ? snake_tile(rnd, static_cast<int>(blockIdx.x), n_ctas) : static_cast<int>(blockIdx.x);
+    };
+    struct Item {
+        int kt, bh, b, hk, qb0, nqb, tb0, n_it;
+    };
+    // Iteration it of an item -> query block: its first token tq0 and, head by
+    // head, its head g (token-major blocks hold all G heads).  Causal: the
+    // first block that sees the key tile is the one holding token kt * BN.
+    auto decode = [&](int idx) {
+        Item I;
+        banded_item(idx, a.n_kt, nbh, a.band, &I.kt, &I.bh);
+        I.b = I.bh / a.Hk;
+        I.hk = I.bh - I.b * a.Hk;
+        I.qb0 = a.causal ? I.kt * (BN / kKvBQ) : 0;
+        I.nqb = a.n_qb - I.qb0;
+        I.tb0 = a.causal ? (I.kt * BN) >> a.tb_log2 : 0;
+        I.n_it = kTok ? a.n_tb - I.tb0 : a.G * I.nqb;
+        return I;
+    };
+    auto block_of = [&](const Item& I, int it, int* g, int* tq0) {
         if (kTok) {
             *g = 0;
-            *tq0 = (tb0 + it) << a.tb_log2;
+            *tq0 = (I.tb0 + it) << a.tb_log2;
         } else {
-            *g = it / nqb;
-            *tq0 = (qb0 + it - *g * nqb) * kKvBQ;
+            *g = it / I.nqb;
+            *tq0 = (I.qb0 + it - *g * I.nqb) * kKvBQ;
         }
     };
 
@@ -250,6 +269,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             mbar_init(&bars[kA_SFree + s], 1);
         }
         mbar_init(&bars[kA_Final], 1);
+        mbar_init(&bars[kA_AccFree], kKvMathWarps);         // dK/dV of an item read out
         for (int s = 0; s < 2; ++s) mbar_init(&bars[kA_DSRead + s], 4);   // one arrive per store warp
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -276,79 +296,102 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
     const uint32_t tmem = *tmem_holder;
 
     if (warp == 0) {
-        // producer, whole warp: per query block, the bias rows (lanes write
-        // rows lane and lane + 32), then Q and dO by TMA (lane 0)
+        // producer, whole warp: per item the K and V tiles, then per query
+        // block the bias rows (lanes write rows lane and lane + 32) and Q and
+        // dO by TMA (lane 0)
         if (lane == 0) {
             prefetch_tmap(&a.tk); prefetch_tmap(&a.tv); prefetch_tmap(&a.tq); prefetch_tmap(&a.tdo);
-            mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * Lay::kKTile);
-            for (int s = 0; s < Lay::kSlabs; ++s) {
-                tma_load_3d(smem + Lay::kK + s * kSlabBytes, &a.tk, &bars[kA_KVFull], s * 64, kt * BN, bh);
-                tma_load_3d(smem + Lay::kV + s * kSlabBytes, &a.tv, &bars[kA_KVFull], s * 64, kt * BN, bh);
-            }
         }
         const float inv_scale = 1.0f / a.scale;
-        // LSE and D of a query block are read one iteration ahead, so their
-        // global-load latency overlaps the wait for the stage to free up
         float nl[2], nd[2];
-        auto fetch_stats = [&](int it) {
-            int g, tq0;
-            block_of(it, &g, &tq0);
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int rr = lane + 32 * h2;                 // row of the block
-                const int gr = kTok ? (rr & (a.G - 1)) : g;
-                const int t = tq0 + (kTok ? rr >> a.g_log2 : rr);
-                const size_t qrow = static_cast<size_t>(b * a.Hq + hk * a.G + gr) * a.T + t;
-                nl[h2] = t < a.T ? a.LSE[qrow] : INFINITY;     // rows past T: p = 0
-                nd[h2] = t < a.T ? a.Drow[qrow] : 0.0f;
-            }
-        };
-        if (n_it > 0) fetch_stats(0);
-        int issued = 0;
-        for (int it = 0; it < n_it; ++it) {
-            const int st = it % kKvStages;
-            if (it >= kKvStages &&
-                !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + st], ((it / kKvStages) - 1) & 1,
-                                                   a.status, abort_flag)))
-                break;
-            int g, tq0;
-            block_of(it, &g, &tq0);
-            float cl[2] = {nl[0], nl[1]}, cd[2] = {nd[0], nd[1]};
-            if (it + 1 < n_it) fetch_stats(it + 1);
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int rr = lane + 32 * h2;                 // query row of the block
-                const float bl = -cl[h2] * inv_scale;
-                const float bd = -cd[h2];
-                const float lh = __bfloat162float(__float2bfloat16_rn(bl));
-                const float ll = bl == -INFINITY ? 0.0f : bl - lh;
-                const float dh = __bfloat162float(__float2bfloat16_rn(bd));
-                const float dl = bd - dh;
-                const uint32_t o0 = bias_chunk(rr, 0);
-                *reinterpret_cast<uint4*>(smem + Lay::kAL + st * Lay::kBiasQ + o0) = make_uint4(pack_bf16(lh, ll), 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(smem + Lay::kAD + st * Lay::kBiasQ + o0) = make_uint4(pack_bf16(dh, dl), 0u, 0u, 0u);
-            }
-            fence_proxy_async_smem();   // generic writes -> the tensor core's reads
-            __syncwarp();
+        int it0 = 0, n_done = 0, issued = 0;
+        bool ok = true;
+        for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+            const int idx = item_of(rnd);
+            if (idx >= a.n_items) continue;
+            const Item I = decode(idx);
+            // the item's K and V replace the previous item's once its last dK
+            // product (and so every product reading K or V) has completed
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[kA_QFull + st], 2 * Lay::kQTile);
-                for (int s = 0; s < Lay::kSlabs; ++s) {
-                    unsigned char* dq_ = smem + Lay::kQ + st * Lay::kQTile + s * kKvSlab;
-                    unsigned char* ddo = smem + Lay::kDO + st * Lay::kQTile + s * kKvSlab;
-                    if (kTok) {   // box (64, G, TB, 1): rows t * G + g
-                        tma_load_4d(dq_, &a.tq, &bars[kA_QFull + st], s * 64, 0, tq0, bh);
-                        tma_load_4d(ddo, &a.tdo, &bars[kA_QFull + st], s * 64, 0, tq0, bh);
-                    } else {
-                        const int qh = b * a.Hq + hk * a.G + g;
-                        tma_load_3d(dq_, &a.tq, &bars[kA_QFull + st], s * 64, tq0, qh);
-                        tma_load_3d(ddo, &a.tdo, &bars[kA_QFull + st], s * 64, tq0, qh);
+                if (n_done > 0 && !mbar_wait(&bars[kA_QEmpty + (it0 - 1) % kKvStages],
+                                             ((it0 - 1) / kKvStages) & 1, a.status, abort_flag))
+                    ok = false;
+                if (ok) {
+                    mbar_arrive_expect_tx(&bars[kA_KVFull], 2 * Lay::kKTile);
+                    for (int s = 0; s < Lay::kSlabs; ++s) {
+                        tma_load_3d(smem + Lay::kK + s * kSlabBytes, &a.tk, &bars[kA_KVFull], s * 64, I.kt * BN, I.bh);
+                        tma_load_3d(smem + Lay::kV + s * kSlabBytes, &a.tv, &bars[kA_KVFull], s * 64, I.kt * BN, I.bh);
                     }
                 }
             }
-            issued = it + 1;
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            // LSE and D of a query block are read one iteration ahead, so their
+            // global-load latency overlaps the wait for the stage to free up
+            auto fetch_stats = [&](int it) {
+                int g, tq0;
+                block_of(I, it, &g, &tq0);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int rr = lane + 32 * h2;                 // row of the block
+                    const int gr = kTok ? (rr & (a.G - 1)) : g;
+                    const int t = tq0 + (kTok ? rr >> a.g_log2 : rr);
+                    const size_t qrow = static_cast<size_t>(I.b * a.Hq + I.hk * a.G + gr) * a.T + t;
+                    nl[h2] = t < a.T ? a.LSE[qrow] : INFINITY;     // rows past T: p = 0
+                    nd[h2] = t < a.T ? a.Drow[qrow] : 0.0f;
+                }
+            };
+            if (I.n_it > 0) fetch_stats(0);
+            for (int it = 0; it < I.n_it; ++it) {
+                const int git = it0 + it;
+                const int st = git % kKvStages;
+                if (git >= kKvStages &&
+                    !__all_sync(0xffffffffu, mbar_wait(&bars[kA_QEmpty + st], ((git / kKvStages) - 1) & 1,
+                                                       a.status, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                int g, tq0;
+                block_of(I, it, &g, &tq0);
+                float cl[2] = {nl[0], nl[1]}, cd[2] = {nd[0], nd[1]};
+                if (it + 1 < I.n_it) fetch_stats(it + 1);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int rr = lane + 32 * h2;                 // query row of the block
+                    const float bl = -cl[h2] * inv_scale;
+                    const float bd = -cd[h2];
+                    const float lh = __bfloat162float(__float2bfloat16_rn(bl));
+                    const float ll = bl == -INFINITY ? 0.0f : bl - lh;
+                    const float dh = __bfloat162float(__float2bfloat16_rn(bd));
+                    const float dl = bd - dh;
+                    const uint32_t o0 = bias_chunk(rr, 0);
+                    *reinterpret_cast<uint4*>(smem + Lay::kAL + st * Lay::kBiasQ + o0) = make_uint4(pack_bf16(lh, ll), 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(smem + Lay::kAD + st * Lay::kBiasQ + o0) = make_uint4(pack_bf16(dh, dl), 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();   // generic writes -> the tensor core's reads
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars[kA_QFull + st], 2 * Lay::kQTile);
+                    for (int s = 0; s < Lay::kSlabs; ++s) {
+                        unsigned char* dq_ = smem + Lay::kQ + st * Lay::kQTile + s * kKvSlab;
+                        unsigned char* ddo = smem + Lay::kDO + st * Lay::kQTile + s * kKvSlab;
+                        if (kTok) {   // box (64, G, TB, 1): rows t * G + g
+                            tma_load_4d(dq_, &a.tq, &bars[kA_QFull + st], s * 64, 0, tq0, I.bh);
+                            tma_load_4d(ddo, &a.tdo, &bars[kA_QFull + st], s * 64, 0, tq0, I.bh);
+                        } else {
+                            const int qh = I.b * a.Hq + I.hk * a.G + g;
+                            tma_load_3d(dq_, &a.tq, &bars[kA_QFull + st], s * 64, tq0, qh);
+                            tma_load_3d(ddo, &a.tdo, &bars[kA_QFull + st], s * 64, tq0, qh);
+                        }
+                    }
+                }
+                issued = git + 1;
+            }
+            it0 += I.n_it;
+            ++n_done;
         }
+        // Let every load this warp started land before the CTA retires.
         if (lane == 0) {
-            mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
+            if (n_done > 0) mbar_wait(&bars[kA_KVFull], (n_done - 1) & 1, a.status, abort_flag);
             for (int it = max(0, issued - kKvStages); it < issued; ++it)
                 mbar_wait(&bars[kA_QFull + it % kKvStages], (it / kKvStages) & 1, a.status, abort_flag);
         }
@@ -366,87 +409,110 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
             const uint64_t kd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kK));
             const uint64_t vd0 = desc_kmajor_sw128(smem_u32(smem + Lay::kV));
             const uint64_t ad0 = desc_noswizzle(smem_u32(smem + Lay::kAA), kBiasLbo, kBiasSbo);
-            bool ok = mbar_wait(&bars[kA_KVFull], 0, a.status, abort_flag);
-            if (warp == 1) {
-                for (int it = 0; ok && it < n_it; ++it) {
-                    const int st = it % kKvStages;
-                    const int buf = it & 1;
-                    if (!mbar_wait(&bars[kA_QFull + st], (it / kKvStages) & 1, a.status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    // S^T(it) = K Q^T - LSE/scale into the S columns of buffer
-                    // buf, which held P^T(it-2): its dV product must be done
-                    if (it >= 2 && !mbar_wait(&bars[kA_SFree + buf], ((it - 2) >> 1) & 1, a.status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
-                    const uint64_t dd = desc_kmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile));
+            bool ok = true;
+            int it0 = 0, n_done = 0;
+            for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+                const int idx = item_of(rnd);
+                if (idx >= a.n_items) continue;
+                const Item I = decode(idx);
+                if (warp == 1) {
+                    // the item's K and V tiles
+                    if (!mbar_wait(&bars[kA_KVFull], n_done & 1, a.status, abort_flag)) { ok = false; break; }
+                    for (int it = 0; it < I.n_it; ++it) {
+                        const int git = it0 + it;
+                        const int st = git % kKvStages;
+                        const int buf = git & 1;
+                        if (!mbar_wait(&bars[kA_QFull + st], (git / kKvStages) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        // S^T = K Q^T - LSE/scale into the S columns of buffer buf,
+                        // which held P^T two iterations back: its dV product must be done
+                        if (git >= 2 &&
+                            !mbar_wait(&bars[kA_SFree + buf], ((git - 2) >> 1) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t qd = desc_kmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile));
+                        const uint64_t dd = desc_kmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile));
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
-                        const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                        umma_ss(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_ss(tmem + buf * 64, ad0,
-                            desc_noswizzle(smem_u32(smem + Lay::kAL + st * Lay::kBiasQ), kBiasLbo, kBiasSbo), id_s, 1u);
-                    umma_commit(&bars[kA_SFull + buf]);
-                    // dP^T(it) = V dO^T - D over dS^T(it-2): its dK product must be
-                    // done (the stage release of it-2) and, with stored dS, the
-                    // store warps must have read it
-                    if (it >= 2 && !mbar_wait(&bars[kA_QEmpty + (it - 2) % kKvStages], ((it - 2) / kKvStages) & 1,
-                                              a.status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (it >= 2 && a.dS &&
-                        !mbar_wait(&bars[kA_DSRead + buf], ((it - 2) >> 1) & 1, a.status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                            const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
+                            umma_ss(tmem + buf * 64, kd0 + offk, qd + offq, id_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_ss(tmem + buf * 64, ad0,
+                                desc_noswizzle(smem_u32(smem + Lay::kAL + st * Lay::kBiasQ), kBiasLbo, kBiasSbo),
+                                id_s, 1u);
+                        umma_commit(&bars[kA_SFull + buf]);
+                        // dP^T = V dO^T - D over dS^T of two iterations back: its dK
+                        // product must be done (that iteration's stage release)
+                        // and, with stored dS, the store warps must have read it
+                        if (git >= 2 && !mbar_wait(&bars[kA_QEmpty + (git - 2) % kKvStages],
+                                                   ((git - 2) / kKvStages) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (git >= 2 && a.dS &&
+                            !mbar_wait(&bars[kA_DSRead + buf], ((git - 2) >> 1) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
-                        const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
-                        umma_ss(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t offk = ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4;
+                            const uint64_t offq = ((kk >> 2) * kKvSlab + (kk & 3) * 32) >> 4;
+                            umma_ss(tmem + 128 + buf * 64, vd0 + offk, dd + offq, id_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_ss(tmem + 128 + buf * 64, ad0,
+                                desc_noswizzle(smem_u32(smem + Lay::kAD + st * Lay::kBiasQ), kBiasLbo, kBiasSbo),
+                                id_s, 1u);
+                        umma_commit(&bars[kA_DPFull + buf]);
                     }
-                    umma_ss(tmem + 128 + buf * 64, ad0,
-                            desc_noswizzle(smem_u32(smem + Lay::kAD + st * Lay::kBiasQ), kBiasLbo, kBiasSbo), id_s, 1u);
-                    umma_commit(&bars[kA_DPFull + buf]);
+                } else {
+                    for (int it = 0; it < I.n_it; ++it) {
+                        const int git = it0 + it;
+                        const int st = git % kKvStages;
+                        const int buf = git & 1;
+                        const uint32_t acc0 = it > 0 ? 1u : 0u;
+                        // dV += P^T dO (A: P^T from TMEM), then release the S columns
+                        if (!mbar_wait(&bars[kA_PReady + buf], (git >> 1) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        // an item's first products overwrite dV / dK: the math
+                        // warps must have read out the previous item's
+                        if (it == 0 && n_done > 0 &&
+                            !mbar_wait(&bars[kA_AccFree], (n_done - 1) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
+#pragma unroll
+                        for (int kk = 0; kk < kKvBQ / 16; ++kk)
+                            umma_ts(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g,
+                                    kk > 0 ? 1u : acc0);
+                        umma_commit(&bars[kA_SFree + buf]);
+                        // dK += dS^T Q, then release the Q/dO stage (and dS^T)
+                        if (!mbar_wait(&bars[kA_DSReady + buf], (git >> 1) & 1, a.status, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
+#pragma unroll
+                        for (int kk = 0; kk < kKvBQ / 16; ++kk)
+                            umma_ts(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g,
+                                    kk > 0 ? 1u : acc0);
+                        umma_commit(&bars[kA_QEmpty + st]);
+                    }
+                    umma_commit(&bars[kA_Final]);
                 }
-            } else {
-                for (int it = 0; ok && it < n_it; ++it) {
-                    const int st = it % kKvStages;
-                    const int buf = it & 1;
-                    const uint32_t acc0 = it > 0 ? 1u : 0u;
-                    // dV += P^T dO (A: P^T from TMEM), then release the S columns
-                    if (!mbar_wait(&bars[kA_PReady + buf], (it >> 1) & 1, a.status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t dmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kDO + st * Lay::kQTile), kKvSlab);
-#pragma unroll
-                    for (int kk = 0; kk < kKvBQ / 16; ++kk)
-                        umma_ts(tmem + 256, tmem + buf * 64 + kk * 8, dmn + kk * (2048 >> 4), id_g, kk > 0 ? 1u : acc0);
-                    umma_commit(&bars[kA_SFree + buf]);
-                    // dK += dS^T Q, then release the Q/dO stage (and dS^T)
-                    if (!mbar_wait(&bars[kA_DSReady + buf], (it >> 1) & 1, a.status, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t qmn = desc_mnmajor_sw128(smem_u32(smem + Lay::kQ + st * Lay::kQTile), kKvSlab);
-#pragma unroll
-                    for (int kk = 0; kk < kKvBQ / 16; ++kk)
-                        umma_ts(tmem + 384, tmem + 128 + buf * 64 + kk * 8, qmn + kk * (2048 >> 4), id_g,
-                                kk > 0 ? 1u : acc0);
-                    umma_commit(&bars[kA_QEmpty + st]);
-                }
-                umma_commit(&bars[kA_Final]);
+                it0 += I.n_it;
+                ++n_done;
             }
         }
         __syncwarp();
@@ -459,22 +525,31 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         if (a.dS) {
             const int quarter = warp & 3;
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-            const int k = kt * BN + quarter * 32 + lane;
-            for (int it = 0; it < n_it; ++it) {
-                int g, tq0;
-                block_of(it, &g, &tq0);
-                const int buf = it & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSReady + buf], (it >> 1) & 1, a.status,
-                                                       abort_flag))) break;
-                tc_fence_after();
-                uint32_t v[32];
-                tmem_ld32(lane_base + 128 + buf * 64, v);
-                tmem_wait_ld();
-                reg_fence<32>(v);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[kA_DSRead + buf]);
-                store_ds_row(a, bh, k, tq0, v);
+            bool ok = true;
+            int it0 = 0;
+            for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+                const int idx = item_of(rnd);
+                if (idx >= a.n_items) continue;
+                const Item I = decode(idx);
+                const int k = I.kt * BN + quarter * 32 + lane;
+                for (int it = 0; it < I.n_it; ++it) {
+                    int g, tq0;
+                    block_of(I, it, &g, &tq0);
+                    const int git = it0 + it;
+                    const int buf = git & 1;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DSReady + buf], (git >> 1) & 1, a.status,
+                                                           abort_flag))) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + 128 + buf * 64, v);
+                    tmem_wait_ld();
+                    reg_fence<32>(v);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[kA_DSRead + buf]);
+                    store_ds_row(a, I.bh, k, tq0, v);
+                }
+                it0 += I.n_it;
             }
         }
     } else {
@@ -485,90 +560,105 @@ __global__ void __launch_bounds__(kKvThreads, 1) dkdv_kernel(const __grid_consta
         const int sub = (warp - 2) >> 2;
         const int half = lane >> 4;
         const int kr = quarter * 32 + sub * 16 + (lane & 15);   // key row within the tile
-        const int k = kt * BN + kr;
         const int c0 = half * 32;                          // first query column of this thread
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32 + sub * 16) << 16);
         const float sl2 = a.scale_log2;
         bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            int g, tq0;
-            block_of(it, &g, &tq0);
-            const int buf = it & 1;
-            // P^T = 2^(scale*log2(e) * (s - LSE/scale)) once S^T is in
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFull + buf], (it >> 1) & 1, a.status,
-                                                   abort_flag))) { ok = false; break; }
-            tc_fence_after();
-            const bool diag = a.causal && tq0 < kt * BN + BN;   // some key after some query
-            uint32_t s[32], dp[32], pk[16], dk[16];
-            tmem_ld16x2_32<32>(lane_base + buf * 64, s);          // s - LSE/scale
-            tmem_wait_ld();
-            reg_fence<32>(s);
-            if (!diag) {                   // every column visible (CTA-uniform branch)
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[e] = __float_as_uint(ex2(__uint_as_float(s[e]) * sl2));
-            } else {
-                // visible columns: token >= k, i.e. c >= k - tq0 (head by head)
-                // or c >= (k - tq0) * G (token-major); a select, no branch per
-                // element (masked: score -inf, so P = dS = 0)
-                const int vlo = (kTok ? (k - tq0) * a.G : k - tq0) - c0;
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    s[e] = __float_as_uint(ex2((e >= vlo ? __uint_as_float(s[e]) : -INFINITY) * sl2));
-            }
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) pk[e / 2] = pack_bf16(__uint_as_float(s[e]), __uint_as_float(s[e + 1]));
-            // P^T (bf16 pairs) over the S columns this warp has read
-            __syncwarp();
-            tmem_st16x2_16<16>(lane_base + buf * 64, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kA_PReady + buf]);
-            // dS^T = P^T * (dP^T - D) once dP^T is in
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DPFull + buf], (it >> 1) & 1, a.status,
-                                                   abort_flag))) { ok = false; break; }
-            tc_fence_after();
-            tmem_ld16x2_32<32>(lane_base + 128 + buf * 64, dp);   // dP - D
-            tmem_wait_ld();
-            reg_fence<32>(dp);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2)
-                dk[e / 2] = pack_bf16(__uint_as_float(s[e]) * __uint_as_float(dp[e]),
-                                      __uint_as_float(s[e + 1]) * __uint_as_float(dp[e + 1]));
-            __syncwarp();
-            tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kA_DSReady + buf]);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_Final], 0, a.status, abort_flag));
-        if (ok) {
-            tc_fence_after();
-            // dK (scaled) then dV; this thread writes columns [half*D/2, (half+1)*D/2)
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                uint32_t gr[D / 2];
-#pragma unroll
-                for (int c = 0; c < D / 2; c += 32)
-                    tmem_ld16x2_32<D / 2>(lane_base + (which ? 256 : 384) + c, gr + c);
+        int it0 = 0, n_done = 0;
+        for (int rnd = 0; ok && rnd < n_rounds; ++rnd) {
+            const int idx = item_of(rnd);
+            if (idx >= a.n_items) continue;
+            const Item I = decode(idx);
+            const int k = I.kt * BN + kr;
+            for (int it = 0; it < I.n_it; ++it) {
+                int g, tq0;
+                block_of(I, it, &g, &tq0);
+                const int git = it0 + it;
+                const int buf = git & 1;
+                // P^T = 2^(scale*log2(e) * (s - LSE/scale)) once S^T is in
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_SFull + buf], (git >> 1) & 1, a.status,
+                                                       abort_flag))) { ok = false; break; }
+                tc_fence_after();
+                const bool diag = a.causal && tq0 < I.kt * BN + BN;   // some key after some query
+                uint32_t s[32], dp[32], pk[16], dk[16];
+                tmem_ld16x2_32<32>(lane_base + buf * 64, s);          // s - LSE/scale
                 tmem_wait_ld();
-                reg_fence<D / 2>(gr);
-                if (k < a.T) {
-                    const size_t row = static_cast<size_t>(bh) * a.T + k;
-                    uint4* dst = reinterpret_cast<uint4*>((which ? a.dV : a.dK) + row * D + half * (D / 2));
-                    const float sc = which ? 1.0f : a.scale;
+                reg_fence<32>(s);
+                if (!diag) {                   // every column visible (CTA-uniform branch)
 #pragma unroll
-                    for (int c = 0; c < D / 2; c += 8) {
-                        uint4 u;
-                        u.x = pack_bf16(__uint_as_float(gr[c]) * sc, __uint_as_float(gr[c + 1]) * sc);
-                        u.y = pack_bf16(__uint_as_float(gr[c + 2]) * sc, __uint_as_float(gr[c + 3]) * sc);
-                        u.z = pack_bf16(__uint_as_float(gr[c + 4]) * sc, __uint_as_float(gr[c + 5]) * sc);
-                        u.w = pack_bf16(__uint_as_float(gr[c + 6]) * sc, __uint_as_float(gr[c + 7]) * sc);
-                        dst[c / 8] = u;
+                    for (int e = 0; e < 32; ++e) s[e] = __float_as_uint(ex2(__uint_as_float(s[e]) * sl2));
+                } else {
+                    // visible columns: token >= k, i.e. c >= k - tq0 (head by head)
+                    // or c >= (k - tq0) * G (token-major); a select, no branch per
+                    // element (masked: score -inf, so P = dS = 0)
+                    const int vlo = (kTok ? (k - tq0) * a.G : k - tq0) - c0;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        s[e] = __float_as_uint(ex2((e >= vlo ? __uint_as_float(s[e]) : -INFINITY) * sl2));
+                }
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) pk[e / 2] = pack_bf16(__uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+                // P^T (bf16 pairs) over the S columns this warp has read
+                __syncwarp();
+                tmem_st16x2_16<16>(lane_base + buf * 64, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kA_PReady + buf]);
+                // dS^T = P^T * (dP^T - D) once dP^T is in
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[kA_DPFull + buf], (git >> 1) & 1, a.status,
+                                                       abort_flag))) { ok = false; break; }
+                tc_fence_after();
+                tmem_ld16x2_32<32>(lane_base + 128 + buf * 64, dp);   // dP - D
+                tmem_wait_ld();
+                reg_fence<32>(dp);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    dk[e / 2] = pack_bf16(__uint_as_float(s[e]) * __uint_as_float(dp[e]),
+                                          __uint_as_float(s[e + 1]) * __uint_as_float(dp[e + 1]));
+                __syncwarp();
+                tmem_st16x2_16<16>(lane_base + 128 + buf * 64, dk);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kA_DSReady + buf]);
+            }
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kA_Final], n_done & 1, a.status, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                // dK (scaled) then dV; this thread writes columns [half*D/2, (half+1)*D/2).
+                // Once both are in registers the next item's products may overwrite them.
+#pragma unroll
+                for (int which = 0; which < 2; ++which) {
+                    uint32_t gr[D / 2];
+#pragma unroll
+                    for (int c = 0; c < D / 2; c += 32)
+                        tmem_ld16x2_32<D / 2>(lane_base + (which ? 256 : 384) + c, gr + c);
+                    tmem_wait_ld();
+                    reg_fence<D / 2>(gr);
+                    if (which == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars[kA_AccFree]);
+                    }
+                    if (k < a.T) {
+                        const size_t row = static_cast<size_t>(I.bh) * a.T + k;
+                        uint4* dst = reinterpret_cast<uint4*>((which ? a.dV : a.dK) + row * D + half * (D / 2));
+                        const float sc = which ? 1.0f : a.scale;
+#pragma unroll
+                        for (int c = 0; c < D / 2; c += 8) {
+                            uint4 u;
+                            u.x = pack_bf16(__uint_as_float(gr[c]) * sc, __uint_as_float(gr[c + 1]) * sc);
+                            u.y = pack_bf16(__uint_as_float(gr[c + 2]) * sc, __uint_as_float(gr[c + 3]) * sc);
+                            u.z = pack_bf16(__uint_as_float(gr[c + 4]) * sc, __uint_as_float(gr[c + 5]) * sc);
+                            u.w = pack_bf16(__uint_as_float(gr[c + 6]) * sc, __uint_as_float(gr[c + 7]) * sc);
+                            dst[c / 8] = u;
+                        }
                     }
                 }
             }
+            it0 += I.n_it;
+            ++n_done;
         }
     }
     tc_fence_before();
@@ -1196,7 +1286,16 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
         const void* fn = stored ? reinterpret_cast<const void*>(dkdv_kernel<D, true>)
                                 : reinterpret_cast<const void*>(dkdv_kernel<D, false>);
         if ((e = set_max_dynamic_smem(fn, (int)smem)) != cudaSuccess) return e;
-        const long long grid = (long long)p.B * p.Hk * A.n_kt;
+        // One CTA per SM walks a snake of the longest-first key tiles when there
+        // are more tiles than SMs and the order is longest-first overall (one
+        // band of heads: the snake balances a decreasing order); otherwise one
+        // CTA per tile, which the hardware schedules greedily.
+        const long long n_items = (long long)p.B * p.Hk * A.n_kt;
+        if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
+        const long long sms = device_sm_count() > 0 ? device_sm_count() : 1;
+        A.n_items = static_cast<int>(n_items);
+        A.persist = n_items > sms && A.band >= p.B * p.Hk ? 1 : 0;
+        const long long grid = A.persist ? sms : n_items;
         if (stored)
             dkdv_kernel<D, true><<<(unsigned)grid, kKvThreads, smem, stream>>>(A);
         else
