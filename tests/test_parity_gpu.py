@@ -328,3 +328,27 @@ def test_fwd_bwd_many_tiles_per_cta():
     assert err_stats(f64(out["LSE"]), LSE)[0] <= LSE_MAX_ABS
     for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(w, x)):
         assert_grad_close(f64(out[name]), r, name)
+
+
+# (B, Hq, Hk, d, T, L): stored dS with more tiles than SMs and ragged ends.
+# The first case has 216 key tiles, so the dK/dV kernel runs persistent CTAs
+# that walk several key tiles each (ring, TMEM-buffer and accumulator phases
+# cross item boundaries); all three have more query tiles than SMs, with a
+# ragged last query tile whose stored dS rows past T are never written.
+PERSISTENT_BWD = [
+    (3, 16, 8, 128, 1100, 5),     # G = 2: 216 key tiles, 432 query tiles
+    (2, 16, 4, 128, 1200, 7),     # G = 4: 304 query tiles, the last one half full
+    (1, 16, 2, 128, 1300, 3),     # G = 8: 164 query tiles of 16 tokens
+]
+
+
+@pytest.mark.parametrize("case", PERSISTENT_BWD, ids=lambda c: "B%d_Hq%d_Hk%d_d%d_T%d_L%d" % c)
+def test_bwd_persistent_tiles(case):
+    w = small_w(*case, backward=True)
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x, ws_mode=1)
+    for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(w, x)):
+        assert_grad_close(f64(out[name]), r, name)
+    again = run_gpu(w, x, ws_mode=1)
+    for name in ("dQ", "dK", "dV", "dKd", "dVd"):
+        assert torch.equal(out[name], again[name]), f"{name} not repeatable"
