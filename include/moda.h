@@ -74,11 +74,26 @@ typedef enum moda_dtype {
  * [t*L, (t+1)*L).  CHUNKED is the chunk-aware view [B, Hk, T/C, C*L, d]: with
  * C counted in tokens, chunk c holds rows [c*C*L, (c+1)*C*L) of the FLAT
  * tensor, so it is the same bytes; CHUNKED only adds the check T % C == 0.
- * Results are bitwise identical for both layouts and every C.
+ *
+ * LAYER is the natural layer-major depth cache itself (the input of
+ * moda_repack_depth): Kd and Vd are [L, B, Hk, T, d], row (l, b, hk, t)
+ * holding depth row t*L + l of (b, hk).  moda_fwd and moda_bwd read it in
+ * place -- the tensor-map view (d, layer, token, b*Hk + hk) lands a box of
+ * whole tokens in shared memory as rows t*L + l, so the transpose of the
+ * repack happens inside the depth-tile loads -- and moda_bwd writes dKd and
+ * dVd in the same layer-major layout.  Supported for bf16 when every depth
+ * block holds whole tokens: with Tq = 128 / G and n(c) = min(c, Tq*L
+ * rounded up to a multiple of 16), L must divide n(128) and n(64) (any power
+ * of two L <= 64 qualifies); other shapes get MODA_ERR_UNSUPPORTED (repack
+ * to FLAT instead).  The fp32 path takes FLAT or CHUNKED only.
+ *
+ * Results are bitwise identical for all three layouts and every C (dKd, dVd
+ * in the layout of Kd, Vd).
  */
 typedef enum moda_depth_layout {
     MODA_DEPTH_FLAT = 0,
-    MODA_DEPTH_CHUNKED = 1
+    MODA_DEPTH_CHUNKED = 1,
+    MODA_DEPTH_LAYER = 2
 } moda_depth_layout;
 
 /* moda_shape.flags bits. */

@@ -27,6 +27,7 @@ MODA_BF16 = 0
 MODA_FP32 = 1
 MODA_DEPTH_FLAT = 0
 MODA_DEPTH_CHUNKED = 1
+MODA_DEPTH_LAYER = 2
 MODA_FLAG_NONCAUSAL = 1
 
 # Every symbol include/moda.h declares.

@@ -48,7 +48,8 @@ moda_status validate(const moda_shape* s, Problem* p) {
     if (!s) return fail(MODA_ERR_INVALID_ARG, "shape is NULL");
     if (s->dtype != MODA_BF16 && s->dtype != MODA_FP32)
         return fail(MODA_ERR_INVALID_ARG, "unknown dtype %d", (int)s->dtype);
-    if (s->depth_layout != MODA_DEPTH_FLAT && s->depth_layout != MODA_DEPTH_CHUNKED)
+    if (s->depth_layout != MODA_DEPTH_FLAT && s->depth_layout != MODA_DEPTH_CHUNKED &&
+        s->depth_layout != MODA_DEPTH_LAYER)
         return fail(MODA_ERR_INVALID_ARG, "unknown depth layout %d", (int)s->depth_layout);
     if (s->B < 0 || s->T < 0 || s->L < 0)
         return fail(MODA_ERR_INVALID_ARG, "B=%d T=%d L=%d must be >= 0", s->B, s->T, s->L);
@@ -79,6 +80,21 @@ moda_status validate(const moda_shape* s, Problem* p) {
     } else if (s->d > 128) {
         return fail(MODA_ERR_UNSUPPORTED, "fp32 path supports d <= 128 (d=%d)", s->d);
     }
+    const bool layer = s->depth_layout == MODA_DEPTH_LAYER && s->L > 0;
+    if (layer) {
+        // whole tokens per depth block: the forward's blocks of n(128) rows and
+        // the dQ kernel's of n(64) rows, n(c) = min(c, Tq*L rounded up to 16)
+        if (s->dtype != MODA_BF16)
+            return fail(MODA_ERR_UNSUPPORTED, "the layer-major depth layout needs the bf16 path");
+        const long long dep = (long long)(128 / G) * s->L;
+        const long long r16 = (dep + 15) / 16 * 16;
+        const long long n128 = r16 < 128 ? r16 : 128, n64 = r16 < 64 ? r16 : 64;
+        if (n128 % s->L != 0 || n64 % s->L != 0)
+            return fail(MODA_ERR_UNSUPPORTED,
+                        "layer-major depth layout: L=%d does not split the depth blocks (%lld, %lld rows) "
+                        "into whole tokens; repack to the flat layout",
+                        s->L, n128, n64);
+    }
     // 64-bit element counts must stay addressable; the kernels index rows with
     // 32-bit (b*H + h) and token coordinates.
     const double rows_q = double(s->B) * s->Hq * s->T;
@@ -91,6 +107,7 @@ moda_status validate(const moda_shape* s, Problem* p) {
     p->elem_bytes = s->dtype == MODA_BF16 ? 2 : 4;
     p->causal = (s->flags & MODA_FLAG_NONCAUSAL) ? 0 : 1;
     p->win_lo = s->depth_window > 0 ? s->L - s->depth_window : 0;
+    p->depth_layer = layer ? 1 : 0;
     return MODA_OK;
 }
 
@@ -161,7 +178,13 @@ size_t moda_workspace_size(const moda_shape* shape, int for_bwd) {
 moda_status moda_repack_depth(const moda_shape* shape, const void* src, void* dst,
                               moda_stream_t stream) {
     Problem p;
-    moda_status st = validate(shape, &p);
+    // the repack's layouts are fixed (layer-major in, token-major out)
+    moda_shape flat;
+    if (shape) {
+        flat = *shape;
+        flat.depth_layout = MODA_DEPTH_FLAT;
+    }
+    moda_status st = validate(shape ? &flat : nullptr, &p);
     if (st != MODA_OK) return st;
     if (p.B == 0 || p.T == 0 || p.L == 0) return MODA_OK;
     if ((st = check_ptrs({{src, "src"}, {dst, "dst"}})) != MODA_OK) return st;
@@ -226,7 +249,13 @@ namespace {
 // Decoding limits on top of the shared shape checks.
 moda_status validate_decode(const moda_shape* shape, moda::Problem* p) {
     using namespace moda;
-    moda_status st = validate(shape, p);
+    // the depth layout has no effect on decoding (Kd, Vd are the new token's rows)
+    moda_shape flat;
+    if (shape) {
+        flat = *shape;
+        flat.depth_layout = MODA_DEPTH_FLAT;
+    }
+    moda_status st = validate(shape ? &flat : nullptr, p);
     if (st != MODA_OK) return st;
     if (p->B > 0 && p->T < 1) return fail(MODA_ERR_INVALID_ARG, "decoding needs T >= 1 cached keys");
     if (p->d != 64 && p->d != 128)

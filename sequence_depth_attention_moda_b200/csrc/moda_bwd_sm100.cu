@@ -689,6 +689,7 @@ struct DqArgs {
     const unsigned char* dS;             // stored dS tiles (written by the dK/dV kernel), kStored only
     int n_kb;                            // 64-key blocks per head
     int g_log2;                          // kStored: G = 1 << g_log2
+    int layer;                           // Kd, Vd, dKd, dVd layer-major [L, B, Hk, T, d]
 };
 
 constexpr int kDqBN = 64;            // rows per key / depth block
@@ -840,6 +841,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     if (seq) {
                         tma_load_3d(dk + s * kDqSlab, mk, &bars[kB_KVFull + st], s * 64, row0, bh);
                         tma_load_3d(dv + s * kDqSlab, mv, &bars[kB_KVFull + st], s * 64, row0, bh);
+                    } else if (a.layer) {   // box (64, L, dep_rows / L, 1): whole tokens from row0 / L
+                        tma_load_4d_hint(dk + s * kDqSlab, mk, &bars[kB_KVFull + st], s * 64, 0, row0 / a.L, bh, once);
+                        tma_load_4d_hint(dv + s * kDqSlab, mv, &bars[kB_KVFull + st], s * 64, 0, row0 / a.L, bh, once);
                     } else {   // depth tiles are read exactly once
                         tma_load_3d_hint(dk + s * kDqSlab, mk, &bars[kB_KVFull + st], s * 64, row0, bh, once);
                         tma_load_3d_hint(dv + s * kDqSlab, mv, &bars[kB_KVFull + st], s * 64, row0, bh, once);
@@ -1036,13 +1040,35 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             if (r < D) {
                 const int row0 = jd * a.dep_rows + c0;
                 const int nvalid = min(a.dep_rows, dep_total - jd * a.dep_rows) - c0;
-                __nv_bfloat16* gk = a.dKd + (dep_base + row0) * D + r;
-                __nv_bfloat16* gv = a.dVd + (dep_base + row0) * D + r;
+                if (a.layer) {
+                    // depth row q of the tile = token t0 + q / L, layer q % L, at
+                    // row (l * B * Hk + bh) * T + t of the layer-major tensors
+                    const size_t lstride = static_cast<size_t>(a.B) * a.Hk * a.T * D;
+                    int tq = row0 / a.L;
+                    int l = row0 - tq * a.L;
+                    size_t off = static_cast<size_t>(l) * lstride + (static_cast<size_t>(bh) * a.T + t0 + tq) * D + r;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    if (c < nvalid) {
-                        gk[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
-                        gv[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xv[c]));
+                    for (int c = 0; c < 32; ++c) {
+                        if (c < nvalid) {
+                            a.dKd[off] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
+                            a.dVd[off] = __float2bfloat16_rn(__uint_as_float(xv[c]));
+                        }
+                        if (++l == a.L) {
+                            l = 0;
+                            off += D - static_cast<size_t>(a.L - 1) * lstride;
+                        } else {
+                            off += lstride;
+                        }
+                    }
+                } else {
+                    __nv_bfloat16* gk = a.dKd + (dep_base + row0) * D + r;
+                    __nv_bfloat16* gv = a.dVd + (dep_base + row0) * D + r;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        if (c < nvalid) {
+                            gk[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
+                            gv[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xv[c]));
+                        }
                     }
                 }
             }
@@ -1332,7 +1358,17 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
     }
     if ((e = make_tma_3d_bf16(&B.tk, K, D, p.T, (uint64_t)p.B * p.Hk, kDqBN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&B.tv, V, D, p.T, (uint64_t)p.B * p.Hk, kDqBN, 1)) != cudaSuccess) return e;
-    if (p.L > 0) {
+    B.layer = p.depth_layer;
+    if (p.L > 0 && p.depth_layer) {
+        // layer-major cache [L, B, Hk, T, d] viewed as (d, layer, token, b * Hk + hk)
+        if (B.dep_rows % p.L != 0) return cudaErrorInvalidValue;
+        const uint64_t nbh = (uint64_t)p.B * p.Hk;
+        const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.L, (uint64_t)p.T, nbh};
+        const uint64_t strides[3] = {nbh * p.T * D * 2, (uint64_t)D * 2, (uint64_t)p.T * D * 2};
+        const uint32_t box[4] = {64, (uint32_t)p.L, (uint32_t)(B.dep_rows / p.L), 1};
+        if ((e = make_tma_4d_bf16(&B.tkd, Kd, dims, strides, box)) != cudaSuccess) return e;
+        if ((e = make_tma_4d_bf16(&B.tvd, Vd, dims, strides, box)) != cudaSuccess) return e;
+    } else if (p.L > 0) {
         const uint64_t rows = (uint64_t)p.T * p.L;
         if ((e = make_tma_3d_bf16(&B.tkd, Kd, D, rows, (uint64_t)p.B * p.Hk, B.dep_rows, 1)) != cudaSuccess) return e;
         if ((e = make_tma_3d_bf16(&B.tvd, Vd, D, rows, (uint64_t)p.B * p.Hk, B.dep_rows, 1)) != cudaSuccess) return e;

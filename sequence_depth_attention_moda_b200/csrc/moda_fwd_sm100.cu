@@ -79,6 +79,7 @@ struct FwdArgs {
     int n_tiles;      // B * Hk * n_qt query tiles, longest first within a band of heads
     int band;         // (b, KV head) pairs per band (banded_item)
     int tok_major;    // query tile rows token-major (r = t * G + g), else head-major (r = g * Tq + t)
+    int layer;        // depth tiles from the layer-major cache (4-D view, dep_rows / L whole tokens)
     float scale_log2;
 };
 
@@ -241,6 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1) moda_fwd_sm100_kernel(const __gri
                     for (int s = 0; s < Lay::kSlabs; ++s) {
                         if (seq)
                             tma_load_3d(dst + s * kSlabBytes, m_seq, &full[st], s * 64, row0, T.bh);
+                        else if (a.layer)   // box (64, L, dep_rows / L, 1) from token row0 / L
+                            tma_load_4d_hint(dst + s * kSlabBytes, m_dep, &full[st], s * 64, 0, row0 / a.L, T.bh,
+                                             once);
                         else
                             tma_load_3d_hint(dst + s * kSlabBytes, m_dep, &full[st], s * 64, row0, T.bh, once);
                     }
@@ -574,7 +578,19 @@ cudaError_t launch_d(const Problem& p, const void* Q, const void* K, const void*
         return e;
     if ((e = make_tma_3d_bf16(&a.tk, K, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
     if ((e = make_tma_3d_bf16(&a.tv, V, D, p.T, (uint64_t)p.B * p.Hk, BN, 1)) != cudaSuccess) return e;
-    if (p.L > 0) {
+    a.layer = p.depth_layer;
+    if (p.L > 0 && p.depth_layer) {
+        // layer-major cache [L, B, Hk, T, d] viewed as (d, layer, token, b * Hk + hk):
+        // a box of dep_rows / L whole tokens lands as rows t * L + l, the same
+        // shared-memory tile as the token-major layout's dep_rows rows
+        if (a.dep_rows % p.L != 0) return cudaErrorInvalidValue;
+        const uint64_t nbh = (uint64_t)p.B * p.Hk;
+        const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.L, (uint64_t)p.T, nbh};
+        const uint64_t strides[3] = {nbh * p.T * D * 2, (uint64_t)D * 2, (uint64_t)p.T * D * 2};
+        const uint32_t box[4] = {64, (uint32_t)p.L, (uint32_t)(a.dep_rows / p.L), 1};
+        if ((e = make_tma_4d_bf16(&a.tkd, Kd, dims, strides, box)) != cudaSuccess) return e;
+        if ((e = make_tma_4d_bf16(&a.tvd, Vd, dims, strides, box)) != cudaSuccess) return e;
+    } else if (p.L > 0) {
         const uint64_t rows = (uint64_t)p.T * p.L;
         if ((e = make_tma_3d_bf16(&a.tkd, Kd, D, rows, (uint64_t)p.B * p.Hk, a.dep_rows, 1)) != cudaSuccess) return e;
         if ((e = make_tma_3d_bf16(&a.tvd, Vd, D, rows, (uint64_t)p.B * p.Hk, a.dep_rows, 1)) != cudaSuccess) return e;

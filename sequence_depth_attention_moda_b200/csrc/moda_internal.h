@@ -18,6 +18,7 @@ struct Problem {
     int elem_bytes;     // 2 (bf16) or 4 (fp32)
     int causal;         // 1: key j visible to row t iff j <= t; 0: all keys
     int win_lo;         // first visible depth row of a token (L - window, or 0)
+    int depth_layer;    // 1: Kd, Vd (and dKd, dVd) layer-major [L, B, Hk, T, d]
 };
 
 // Kernel-side status bits written into the per-device status word.

@@ -122,6 +122,16 @@ __device__ __forceinline__ void tma_load_3d_hint(void* dst, const void* map, uin
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* map, uint64_t* bar, int c0,
+                                                 int c1, int c2, int c3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)),
+        "l"(policy)
+        : "memory");
+}
+
 // Untiled bulk copy of `bytes` contiguous bytes global -> shared with an L2
 // cache policy (both addresses 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,

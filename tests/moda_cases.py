@@ -93,7 +93,10 @@ def run_gpu(w: Workload, x: Dict[str, torch.Tensor], backward=None, layout=moda.
     dt = x["Q"].dtype
     gd = Guarded()
     out = {}
-    if w.L > 0:
+    layer = layout == moda.MODA_DEPTH_LAYER
+    if w.L > 0 and layer:      # the layer-major cache, read in place
+        Kd, Vd = x["Kd_layer"], x["Vd_layer"]
+    elif w.L > 0:
         Kd = gd.empty("Kd", (w.B, w.Hk, w.T * w.L, w.d), dt, dev)
         Vd = gd.empty("Vd", (w.B, w.Hk, w.T * w.L, w.d), dt, dev)
         moda.moda_repack_depth(sh, x["Kd_layer"], Kd)
@@ -117,6 +120,13 @@ def run_gpu(w: Workload, x: Dict[str, torch.Tensor], backward=None, layout=moda.
                       ws, nws)
         out.update(dQ=dQ, dK=dK, dV=dV, dKd=dKd, dVd=dVd)
     gd.check()
+    if layer and w.L > 0 and out.get("dKd") is not None:
+        # depth gradients came back layer-major [L, B, Hk, T, d]: token-major
+        # copies for the comparisons, the raw tensors beside them
+        def tm(t):
+            return t.permute(1, 2, 3, 0, 4).reshape(w.B, w.Hk, w.T * w.L, w.d).contiguous()
+        out["dKd_layer"], out["dVd_layer"] = out["dKd"], out["dVd"]
+        out["dKd"], out["dVd"] = tm(out["dKd"]), tm(out["dVd"])
     return out
 
 

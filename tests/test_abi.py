@@ -67,6 +67,10 @@ FAKE = 0x10000   # aligned fake device address: never dereferenced (validation f
     (dict(flags=2), 1),                                                  # unknown flag
     (dict(depth_window=3), 1),                                           # window > L
     (dict(depth_window=-1), 1),
+    (dict(depth_layout=3), 1),                                           # unknown layout
+    (dict(depth_layout=2, L=3), 3),                                      # layer-major: 128 % 3
+    (dict(depth_layout=2, L=24), 3),                                     # layer-major: 64 % 24
+    (dict(depth_layout=2, L=2, dtype=1), 3),                             # layer-major needs bf16
 ])
 def test_fwd_rejects_bad_shapes(lib, kw, status):
     base = dict(B=1, Hq=4, Hk=2, T=64, d=128, L=2, C=16)
@@ -252,3 +256,24 @@ def test_binding_rejects_wrong_dtype_and_short_tensors(lib):
                          torch.zeros(1, 4), None, 0)
     with pytest.raises(moda.MoDAError, match="dst holds"):
         moda.moda_repack_depth(sh, torch.zeros(2, 1, 2, 64, 128, **bf), Kd[:, :1])
+
+
+def test_layer_layout_limits(lib):
+    """The layer-major depth layout is accepted exactly when the forward's
+    128-row and the dQ kernel's 64-row depth blocks hold whole tokens; the
+    decoding and repack entry points ignore the layout field."""
+    def ok(**kw):
+        base = dict(B=1, Hq=4, Hk=2, T=64, d=128, L=2, C=0, depth_layout=moda.MODA_DEPTH_LAYER)
+        base.update(kw)
+        sh = moda.make_shape(**base)
+        return lib.moda_workspace_size(ctypes.byref(sh), 1) != ctypes.c_size_t(-1).value
+    for L in (1, 2, 4, 8, 16, 32, 64):
+        assert ok(L=L), L
+    assert ok(L=0, dtype=moda.MODA_FP32)                 # no depth rows: nothing to read
+    assert not ok(L=48) and not ok(L=3) and not ok(L=128)
+    # G = 8: 16 tokens per query tile, blocks of min(c, 16 L rounded to 16) rows
+    assert ok(Hq=16, Hk=2, L=3)                          # 48-row blocks: 16 tokens of 3
+    assert not ok(Hq=16, Hk=2, L=5)                      # 80 rows: 64-row dQ blocks, 64 % 5
+    assert not ok(Hq=16, Hk=2, L=6)                      # 96 rows: 64-row dQ blocks, 64 % 6
+    sh = moda.make_shape(B=1, Hq=4, Hk=2, T=64, d=128, L=3, C=0, depth_layout=moda.MODA_DEPTH_LAYER)
+    assert lib.moda_decode_workspace_size(ctypes.byref(sh)) != ctypes.c_size_t(-1).value

@@ -352,3 +352,45 @@ def test_bwd_persistent_tiles(case):
     again = run_gpu(w, x, ws_mode=1)
     for name in ("dQ", "dK", "dV", "dKd", "dVd"):
         assert torch.equal(out[name], again[name]), f"{name} not repeatable"
+
+
+# (B, Hq, Hk, d, T, L, causal, window): the layer-major depth layout, read in
+# place through 4-D tensor-map views (no repack), against the flat layout
+LAYER_CASES = [
+    (1, 8, 2, 128, 513, 16, True, 0),     # G = 4, ragged last tile
+    (2, 4, 4, 128, 300, 8, True, 0),      # G = 1: 128 tokens per query tile
+    (1, 16, 2, 128, 200, 3, True, 0),     # G = 8: 48-row depth blocks of 16 tokens
+    (2, 4, 2, 64, 257, 4, True, 0),       # d = 64: the recomputing dQ kernel
+    (1, 8, 2, 128, 300, 8, False, 3),     # non-causal, depth window
+    (1, 6, 2, 128, 100, 2, True, 0),      # G = 3: head-major rows, recomputing dQ
+]
+
+
+@pytest.mark.parametrize("case", LAYER_CASES, ids=lambda c: "B%d_Hq%d_Hk%d_d%d_T%d_L%d_c%d_w%d" % c)
+def test_layer_layout_small(case):
+    """The layer-major cache read in place gives the flat layout's results bit
+    for bit (the same shared-memory depth tiles), dK_d / dV_d written back
+    layer-major; both backward workspaces; and the oracle agrees."""
+    B, Hq, Hk, d, T, L, causal, window = case
+    w = small_w(B, Hq, Hk, d, T, L, backward=True).with_(causal=causal, window=window)
+    x = I.make_inputs(w, device=DEV)
+    for mode in (1, 2):
+        flat = run_gpu(w, x, ws_mode=mode)
+        lay = run_gpu(w, x, layout=moda.MODA_DEPTH_LAYER, ws_mode=mode)
+        for k in ("O", "LSE", "dQ", "dK", "dV", "dKd", "dVd"):
+            assert torch.equal(flat[k], lay[k]), f"ws_mode {mode} {k}"
+    O, LSE = oracle_fwd_full(w, x)
+    assert_out_close(f64(lay["O"]), O, "bf16", "O")
+    for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(w, x)):
+        assert_grad_close(f64(lay[name]), r, name)
+
+
+def test_layer_layout_full_size():
+    """layer_1p5b_T4k with the layer-major cache: bitwise the flat layout's
+    outputs and gradients (the launch configuration the benchmark times)."""
+    w = I.LAYER_1P5B
+    x = I.make_inputs(w, device=DEV)
+    flat = run_gpu(w, x)
+    lay = run_gpu(w, x, layout=moda.MODA_DEPTH_LAYER)
+    for k in ("O", "LSE", "dQ", "dK", "dV", "dKd", "dVd"):
+        assert torch.equal(flat[k], lay[k]), k
