@@ -670,7 +670,7 @@ def run_ours(args):
         long_res = {}
         for L in (LONG.L, 0):
             wl = LONG.with_(L=L)
-            rl = Runner(wl, xl, backward=False)
+            rl = Runner(wl, xl, backward=False, layer=False)   # the forward on token-major depth rows
             msl, callsl = time_steps(rl, max(3, args.steps // 4), 2, world, per_call=True)
             tf = wl.fwd_flops() / (callsl["fwd"] * 1e-3) / 1e12
             long_res[f"L{L}"] = {"fwd_tflops": round(tf, 1),
@@ -800,7 +800,7 @@ def config_measure(w: I.Workload, peaks, flush: torch.Tensor, runs: int = 20, tw
     x = I.make_inputs(w, device="cuda", grad_out=w.backward)
 
     def one(wl):
-        r = Runner(wl, x, backward=wl.backward)
+        r = Runner(wl, x, backward=wl.backward, layer=False)   # repack and kernels timed one by one
         r.step()                                   # fills the token-major depth tensors
         xx = r.x
         fwd = lambda: moda.moda_fwd(r.sh, xx["Q"], xx["K"], xx["V"], r.Kd, r.Vd, r.O, r.LSE)
