@@ -1111,8 +1111,8 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         if (c < nvalid) {
-                            gk[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale);
-                            gv[static_cast<size_t>(c) * D] = __float2bfloat16_rn(__uint_as_float(xv[c]));
+                            st_cs_bf16(gk + static_cast<size_t>(c) * D, __float2bfloat16_rn(__uint_as_float(xk[c]) * a.scale));
+                            st_cs_bf16(gv + static_cast<size_t>(c) * D, __float2bfloat16_rn(__uint_as_float(xv[c])));
                         }
                     }
                 }
