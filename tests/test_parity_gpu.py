@@ -394,3 +394,13 @@ def test_layer_layout_full_size():
     lay = run_gpu(w, x, layout=moda.MODA_DEPTH_LAYER)
     for k in ("O", "LSE", "dQ", "dK", "dV", "dKd", "dVd"):
         assert torch.equal(flat[k], lay[k]), k
+
+
+def test_layer_layout_long_context_forward():
+    """long_context_T64k forward from the layer-major cache (1 KB per layer
+    plane per depth block): bitwise the flat layout's O and LSE."""
+    w = I.LONG_64K
+    x = I.make_inputs(w, device=DEV, grad_out=False)
+    flat = run_gpu(w, x, backward=False)
+    lay = run_gpu(w, x, backward=False, layout=moda.MODA_DEPTH_LAYER)
+    assert torch.equal(flat["O"], lay["O"]) and torch.equal(flat["LSE"], lay["LSE"])

@@ -52,6 +52,26 @@ def test_noalloc_matches_workspace_backward_twice(w):
             assert_grad_close(f64(got[k]), f64(fast[k]), f"call {call} {k} vs the stored-dS path")
 
 
+def test_noalloc_layer_major_depth():
+    """With the layer-major depth layout (caches read in place, dKd / dVd
+    written layer-major) the no-allocation backward gives moda_bwd's bits."""
+    w = W_BF16.with_(L=8)
+    x = I.make_inputs(w, device="cuda")
+    ref = run_gpu(w, x, layout=moda.MODA_DEPTH_LAYER, ws_mode=2)
+    sh = shape_of(w, moda.MODA_DEPTH_LAYER)
+    gd = Guarded()
+    g = {"dQ": gd.like("dQ", x["Q"]), "dK": gd.like("dK", x["K"]), "dV": gd.like("dV", x["V"]),
+         "dKd": gd.like("dKd", x["Kd_layer"]), "dVd": gd.like("dVd", x["Vd_layer"])}
+    moda.moda_bwd_noalloc(sh, x["Q"], x["K"], x["V"], x["Kd_layer"], x["Vd_layer"], ref["O"], ref["LSE"],
+                          x["dO"], g["dQ"], g["dK"], g["dV"], g["dKd"], g["dVd"])
+    gd.check()
+    torch.cuda.synchronize()
+    moda.moda_check_status()
+    for k in ("dQ", "dK", "dV"):
+        assert torch.equal(g[k], ref[k]), k
+    assert torch.equal(g["dKd"], ref["dKd_layer"]) and torch.equal(g["dVd"], ref["dVd_layer"])
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
     # 4,194,305 query rows > the 4,194,304-row built-in scratch: rejected
     # before anything is queued (the pointers are never touched).
