@@ -404,3 +404,24 @@ def test_layer_layout_long_context_forward():
     flat = run_gpu(w, x, backward=False)
     lay = run_gpu(w, x, backward=False, layout=moda.MODA_DEPTH_LAYER)
     assert torch.equal(flat["O"], lay["O"]) and torch.equal(flat["LSE"], lay["LSE"])
+
+
+def test_bench_step_every_slice():
+    """layer_1p5b_T4k exactly as the benchmark step runs it (layer-major depth
+    caches read in place, full backward workspace): O, LSE and all five
+    gradients of every (b, hk) slice against the oracle."""
+    w = I.LAYER_1P5B
+    x = I.make_inputs(w, device=DEV)
+    out = run_gpu(w, x, layout=moda.MODA_DEPTH_LAYER, ws_mode=1)
+    G = w.G
+    for b in range(w.B):
+        for hk in range(w.Hk):
+            ws, xs = slice_workload(w, x, b, hk)
+            O, LSE = oracle_fwd_full(ws, xs)
+            assert_out_close(f64(out["O"][b:b + 1, hk * G:(hk + 1) * G]), O, "bf16", f"slice ({b},{hk}) O")
+            assert err_stats(f64(out["LSE"][b:b + 1, hk * G:(hk + 1) * G]), LSE)[0] <= LSE_MAX_ABS
+            got = {"dQ": out["dQ"][b:b + 1, hk * G:(hk + 1) * G], "dK": out["dK"][b:b + 1, hk:hk + 1],
+                   "dV": out["dV"][b:b + 1, hk:hk + 1], "dKd": out["dKd"][b:b + 1, hk:hk + 1],
+                   "dVd": out["dVd"][b:b + 1, hk:hk + 1]}
+            for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(ws, xs)):
+                assert_grad_close(f64(got[name]), r, f"slice ({b},{hk}) {name}")
