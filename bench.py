@@ -814,8 +814,18 @@ def config_measure(w: I.Workload, peaks, flush: torch.Tensor, runs: int = 20, tw
                 moda.moda_repack_depth(r.sh, xx["Kd_layer"], r.Kd)
                 moda.moda_repack_depth(r.sh, xx["Vd_layer"], r.Vd)
             res["repack_ms"] = _median_ms(rep, runs, flush)
-        moda.moda_check_status()
         del r
+        if wl.L and layer_supported(wl):
+            # the same calls reading the layer-major caches in place (no repack)
+            rl = Runner(wl, x, backward=wl.backward, layer=True)
+            fwd_l = lambda: moda.moda_fwd(rl.sh, xx["Q"], xx["K"], xx["V"], rl.Kd, rl.Vd, rl.O, rl.LSE)
+            res["fwd_layer_ms"] = _median_ms(fwd_l, runs, flush)
+            if wl.backward:
+                bwd_l = lambda: moda.moda_bwd(rl.sh, xx["Q"], xx["K"], xx["V"], rl.Kd, rl.Vd, rl.O, rl.LSE,
+                                              xx["dO"], rl.dQ, rl.dK, rl.dV, rl.dKd, rl.dVd, rl.ws, rl.nws)
+                res["bwd_layer_ms"] = _median_ms(bwd_l, runs, flush)
+            del rl
+        moda.moda_check_status()
         return res
 
     def roof(flops, nbytes, ms):
@@ -841,6 +851,19 @@ def config_measure(w: I.Workload, peaks, flush: torch.Tensor, runs: int = 20, tw
         rb = 2 * 2 * dep_el * e
         out["repack"] = {"ms": round(m["repack_ms"], 4), "gbs": round(rb / (m["repack_ms"] * 1e-3) / 1e9, 1),
                          "frac_of_hbm": round(rb / (m["repack_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    if "fwd_layer_ms" in m:
+        # layer-major caches read in place: the repack's transpose inside the
+        # depth-tile loads; its time against repack + the token-major calls
+        lm = {"fwd_ms": round(m["fwd_layer_ms"], 4)}
+        flat = m["repack_ms"] + m["fwd_ms"]
+        lay = m["fwd_layer_ms"]
+        if w.backward:
+            lm["bwd_ms"] = round(m["bwd_layer_ms"], 4)
+            flat += m["bwd_ms"]
+            lay += m["bwd_layer_ms"]
+        lm["calls_ms"] = round(lay, 4)
+        lm["repack_plus_token_major_calls_ms"] = round(flat, 4)
+        out["layer_major"] = lm
     if twin and w.L:
         m0 = one(w.with_(L=0))
         out["L0_fwd_ms"] = round(m0["fwd_ms"], 4)
