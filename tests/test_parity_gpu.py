@@ -425,3 +425,20 @@ def test_bench_step_every_slice():
                    "dVd": out["dVd"][b:b + 1, hk:hk + 1]}
             for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(ws, xs)):
                 assert_grad_close(f64(got[name]), r, f"slice ({b},{hk}) {name}")
+
+
+def test_layer_layout_persistent_and_modes():
+    """Layer-major caches with persistent dK/dV (216 key tiles), more query
+    tiles than SMs and a ragged end, causal and non-causal with a depth
+    window: bitwise the flat layout, and the oracle agrees."""
+    for causal, window in ((True, 0), (False, 3)):
+        w = small_w(3, 16, 8, 128, 1100, 4, backward=True).with_(causal=causal, window=window)
+        x = I.make_inputs(w, device=DEV)
+        flat = run_gpu(w, x, ws_mode=1)
+        lay = run_gpu(w, x, layout=moda.MODA_DEPTH_LAYER, ws_mode=1)
+        for k in ("O", "LSE", "dQ", "dK", "dV", "dKd", "dVd"):
+            assert torch.equal(flat[k], lay[k]), f"causal={causal} {k}"
+        O, _ = oracle_fwd_full(w, x)
+        assert_out_close(f64(lay["O"]), O, "bf16", f"causal={causal} O")
+        for name, r in zip(("dQ", "dK", "dV", "dKd", "dVd"), oracle_bwd_full(w, x)):
+            assert_grad_close(f64(lay[name]), r, f"causal={causal} {name}")
