@@ -127,7 +127,7 @@ cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t
 // A 4-D bf16 tensor map (dims[0] = d, innermost; byte strides of dims 1..3),
 // box `box` with 128-byte swizzle (box[0] = 64: one 128-byte row).  The
 // strides need not grow with the dimension: the forward reads a query tile
-// token-major (heads inner to tokens) through one.  Not memoised.
+// token-major (heads inner to tokens) through one.  Memoised like the 3-D maps.
 cudaError_t make_tma_4d_bf16(TmaMap* out, const void* base, const uint64_t dims[4],
                              const uint64_t strides_bytes[3], const uint32_t box[4]);
 

@@ -83,6 +83,26 @@ cudaError_t encode_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t r
     return cudaSuccess;
 }
 
+// The same for the 4-D maps (token-major views of Q and dO, the layer-major
+// depth caches): keyed by base, extents, strides and box.
+struct Map4Key {
+    uint64_t base, dims[4], strides[3];
+    uint32_t box[4];
+    bool operator==(const Map4Key& o) const {
+        return std::memcmp(this, &o, sizeof(Map4Key)) == 0;
+    }
+};
+struct Map4KeyHash {
+    size_t operator()(const Map4Key& k) const {
+        uint64_t h = k.base * 0x9E3779B97F4A7C15ull;
+        for (int i = 0; i < 4; ++i) h = (h ^ k.dims[i]) * 0x100000001B3ull;
+        for (int i = 0; i < 3; ++i) h = (h ^ k.strides[i]) * 0x100000001B3ull;
+        for (int i = 0; i < 4; ++i) h = (h ^ k.box[i]) * 0x100000001B3ull;
+        return static_cast<size_t>(h ^ (h >> 29));
+    }
+};
+std::unordered_map<Map4Key, TmaMap, Map4KeyHash> g_map4_cache;
+
 std::mutex g_attr_mutex;
 std::vector<std::tuple<int, const void*, int>> g_attr_done;
 
@@ -109,6 +129,19 @@ cudaError_t make_tma_3d_bf16(TmaMap* out, const void* base, uint64_t d, uint64_t
 
 cudaError_t make_tma_4d_bf16(TmaMap* out, const void* base, const uint64_t dims[4],
                              const uint64_t strides_bytes[3], const uint32_t box[4]) {
+    Map4Key key;
+    std::memset(&key, 0, sizeof(key));
+    key.base = reinterpret_cast<uint64_t>(base);
+    for (int i = 0; i < 4; ++i) key.dims[i] = dims[i], key.box[i] = box[i];
+    for (int i = 0; i < 3; ++i) key.strides[i] = strides_bytes[i];
+    {
+        std::lock_guard<std::mutex> lk(g_map_mutex);
+        auto it = g_map4_cache.find(key);
+        if (it != g_map4_cache.end()) {
+            *out = it->second;
+            return cudaSuccess;
+        }
+    }
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     CUtensorMap map;
@@ -122,6 +155,9 @@ cudaError_t make_tma_4d_bf16(TmaMap* out, const void* base, const uint64_t dims[
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     std::memcpy(out->bytes, &map, sizeof(map));
+    std::lock_guard<std::mutex> lk(g_map_mutex);
+    if (g_map4_cache.size() >= kMapCacheEntries) g_map4_cache.clear();
+    g_map4_cache.emplace(key, *out);
     return cudaSuccess;
 }
 
