@@ -288,7 +288,7 @@ const char* moda_status_string(moda_status status);
 const char* moda_last_error_message(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
-int moda_version(void);   /* 10100: adds flags and depth_window to moda_shape */
+int moda_version(void);   /* 10200: adds MODA_DEPTH_LAYER (10100: flags and depth_window in moda_shape) */
 
 #ifdef __cplusplus
 }  /* extern "C" */

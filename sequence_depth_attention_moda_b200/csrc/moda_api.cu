@@ -335,6 +335,6 @@ moda_status moda_set_phase_events(void* const* events, int n) {
     return MODA_OK;
 }
 
-int moda_version(void) { return 10100; }
+int moda_version(void) { return 10200; }
 
 }  // extern "C"
